@@ -1,0 +1,371 @@
+"""Plain CPU oracle for single-token MLA decode over the latent KV cache.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
+reference legs call it.  It shares no code, table or constant with the CUDA
+library under ``mla_latent_kv_nope_b200/``; the only thing the two sides share is
+the seeded input generator, which holds none of the method's arithmetic.
+
+Everything is float64 numpy.  bf16 inputs are upcast exactly before use; the
+oracle never rounds intermediate values.  Matrix products use numpy's matmul as
+a library primitive; nothing is blocked, fused or reordered beyond what each
+definition states, so every function can be read against the equation it cites.
+
+Sources (cited by page title and section, as the pages name them):
+
+* [MLA-とは] "Multi-head Latent Attention（MLA）とは？KVキャッシュを圧縮する
+  DeepSeekの注意機構を完全解説" (disassemble-channel.com), sections
+  "MLAの発想", "行列吸収", "Value側の吸収", "RoPEが吸収を壊す",
+  "Decoupled RoPE", "KVキャッシュ容量の比較", "実装上のトレードオフ".
+* [attention-variants] youngju.dev "model internals: attention variants",
+  sections "MLA: キャッシュする対象そのものを変える" and "一つの表で比べる".
+* [yuuk-wiki] notes.yuuk.io wiki "Multi-Head Latent Attention", section
+  "横断的知見" (MQA as the special case of MLA).
+
+Conventions (column vectors, y = W x, as [MLA-とは] states in its preamble):
+
+* ``W_UK[i]`` and ``W_UV[i]`` are the per-head blocks W^UK_i, W^UV_i in
+  R^{d_h x d_c}, stored as arrays of shape [H, d_h, d_c] ([MLA-とは] "MLAの発想",
+  the equation k^C = W^UK c^KV and the row-block definition after it).
+* A latent cache row is [c^KV (d_c) || k^R (d_r)]; k^R is stored already
+  rotated ([MLA-とは] "Decoupled RoPE", the two-part cache figure text).
+* ``W_DKV`` is the vertical concatenation [W^DKV ; W^KR] of shape
+  [d_c + d_r, hidden]: rows [0, d_c) give c^KV, rows [d_c, d_c + d_r) give
+  the pre-rotation k^R (both are applied to h, [MLA-とは] "Decoupled RoPE",
+  equation for k^R_j).
+
+Every function here has at least one independent pin in
+``tests/test_oracle_pins.py``; none is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "rope",
+    "rms_norm",
+    "down_project",
+    "cache_append",
+    "absorb_q",
+    "head_logits",
+    "softmax_lse",
+    "materialised_values",
+    "mla_decode_materialised",
+    "latent_attention",
+    "combine_partials",
+    "out_proj",
+    "cache_elems_per_token",
+    "mults_per_cached_token",
+]
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# RoPE and RMSNorm
+# ---------------------------------------------------------------------------
+def rope(x, pos, base: float = 10000.0) -> np.ndarray:
+    """Rotary embedding with half-split pairing, [MLA-とは] "RoPEが吸収を壊す".
+
+    The page defines the rotation used throughout its checks: for a vector of
+    even length d, with half = d/2 and angle theta_k = pos / base^(2k/d) for
+    k < half, the pair (x[k], x[k+half]) is rotated by theta_k:
+
+        y[k]        = x[k] cos(theta_k) - x[k+half] sin(theta_k)
+        y[k+half]   = x[k] sin(theta_k) + x[k+half] cos(theta_k)
+
+    ``x`` may carry leading batch axes; ``pos`` is a scalar or broadcasts
+    against those axes.  Angles and trigonometry are evaluated in float64.
+    """
+    x = _f64(x)
+    d = x.shape[-1]
+    if d == 0:
+        return x.copy()
+    if d % 2:
+        raise ValueError("rope needs an even last dimension")
+    half = d // 2
+    k = np.arange(half, dtype=np.float64)
+    inv_freq = 1.0 / (float(base) ** (2.0 * k / d))
+    pos = _f64(pos)
+    theta = pos[..., None] * inv_freq  # broadcasts over leading axes
+    c, s = np.cos(theta), np.sin(theta)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1)
+
+
+def rms_norm(x, gamma=None, eps: float = 1e-6) -> np.ndarray:
+    """RMSNorm of the latent before it is cached, [MLA-とは] "実装上のトレードオフ"
+    (正規化の扱い): a per-token scalar division by the root mean square,
+    followed by the learned diagonal gain.
+
+        y = x / sqrt(mean(x^2) + eps) * gamma
+
+    ``eps`` is not given by the pages; the library's default is 1e-6.
+    """
+    x = _f64(x)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    y = x / np.sqrt(ms + float(eps))
+    if gamma is not None:
+        y = y * _f64(gamma)
+    return y
+
+
+# ---------------------------------------------------------------------------
+# Cache append: down-projection, latent RMSNorm, decoupled RoPE key
+# ---------------------------------------------------------------------------
+def down_project(h, W_DKV) -> np.ndarray:
+    """x = [W^DKV ; W^KR] h for each row of ``h`` ([MLA-とは] "MLAの発想",
+    c^KV_t = W^DKV h_t, and "Decoupled RoPE", k^R_j = R_j W^KR h_j before R_j).
+
+    h: [B, hidden]; W_DKV: [d_c + d_r, hidden] -> [B, d_c + d_r].
+    """
+    return _f64(h) @ _f64(W_DKV).T
+
+
+def cache_append(cache, seqlens, h, W_DKV, d_c: int, gamma=None,
+                 eps: float = 1e-6, rope_base: float = 10000.0):
+    """Append one token per sequence to the latent cache.
+
+    For each sequence b with current length L_b (the new token's position):
+      x = W_DKV h_b                                   (down-projection)
+      c = RMSNorm(x[0:d_c]) * gamma                    (latent RMSNorm)
+      k = RoPE(x[d_c:], pos = L_b)                     (decoupled key, rotated)
+      cache[b, L_b, :] = [c || k];  L_b += 1
+    ([MLA-とは] "MLAの発想" eq. c^KV; "Decoupled RoPE" eq. k^R_j = R_j W^KR h_j
+    and the statement that the cache holds the already-rotated k^R;
+    "実装上のトレードオフ" 正規化の扱い for caching the normalised latent.)
+
+    Returns (new_cache float64 copy, new_seqlens int64 copy, rows [B, R] float64).
+    Raises IndexError if a sequence is already at capacity (nothing written).
+    """
+    cache = _f64(cache).copy()
+    seqlens = np.asarray(seqlens, dtype=np.int64).copy()
+    B, cap, R = cache.shape
+    x = down_project(h, W_DKV)
+    if x.shape != (B, R):
+        raise ValueError("W_DKV rows must equal the cache row width")
+    c = rms_norm(x[:, :d_c], gamma, eps)
+    rows = np.empty((B, R), dtype=np.float64)
+    for b in range(B):
+        L = int(seqlens[b])
+        if L >= cap:
+            raise IndexError(f"sequence {b} is at capacity {cap}")
+        k = rope(x[b, d_c:], L, rope_base)
+        rows[b] = np.concatenate([c[b], k])
+        cache[b, L] = rows[b]
+        seqlens[b] = L + 1
+    return cache, seqlens, rows
+
+
+# ---------------------------------------------------------------------------
+# Materialised MHA decode (the plain definition the absorbed form must equal)
+# ---------------------------------------------------------------------------
+def head_logits(q_nope_i, q_pe_i, q_pos, W_UK_i, c, k_pe,
+                rope_base: float = 10000.0) -> np.ndarray:
+    """Raw (unscaled) attention logits of one head against L cached tokens,
+    with K materialised.
+
+    q = [q^C ; RoPE(q^R, q_pos)]       ([MLA-とは] "Decoupled RoPE", q_{t,i})
+    k_j = [W^UK_i c_j ; k^R_j]          (k^C = W^UK c^KV, "MLAの発想";
+                                         k^R_j shared by all heads, stored rotated)
+    logit_j = q . k_j                   ("Decoupled RoPE", the split dot product)
+
+    q_nope_i: [d_h]; q_pe_i: [d_r]; W_UK_i: [d_h, d_c]; c: [L, d_c];
+    k_pe: [L, d_r].  Returns [L].
+    """
+    q = np.concatenate([_f64(q_nope_i), rope(q_pe_i, q_pos, rope_base)])
+    kC = _f64(c) @ _f64(W_UK_i).T  # [L, d_h]: rows are k^C_j = W^UK_i c_j
+    K = np.concatenate([kC, _f64(k_pe)], axis=1)  # [L, d_h + d_r]
+    return K @ q
+
+
+def softmax_lse(s):
+    """Softmax of a logit vector with max subtraction, and its log-sum-exp.
+
+    An empty vector gives (empty weights, -inf)."""
+    s = _f64(s)
+    if s.size == 0:
+        return s.copy(), -math.inf
+    m = np.max(s)
+    e = np.exp(s - m)
+    z = np.sum(e)
+    return e / z, float(m + math.log(z))
+
+
+def materialised_values(p, c, W_UV_i) -> np.ndarray:
+    """o = sum_j p_j v_j with v_j = W^UV_i c_j materialised per cached token
+    ([MLA-とは] "Value側の吸収", first equation for o_{t,i}).
+
+    p: [L]; c: [L, d_c]; W_UV_i: [d_v, d_c] -> [d_v]."""
+    V = _f64(c) @ _f64(W_UV_i).T  # [L, d_v]: rows are v^C_j
+    return _f64(p) @ V
+
+
+def mla_decode_materialised(q_nope, q_pe, q_pos, W_UK, W_UV, cache, seqlens,
+                            softmax_scale: float, rope_base: float = 10000.0):
+    """Single-token decode as plain multi-head attention with K and V
+    materialised from the latent cache (what the absorbed kernel must equal).
+
+    For every sequence b and head i:
+      s_j = scale * (q . k_j)  for j < L_b                  (head_logits)
+      p = softmax(s); lse = log sum_j exp(s_j)
+      out[b,i]   = sum_j p_j W^UV_i c_j                     ("Value側の吸収")
+      o_lat[b,i] = sum_j p_j c_j                            (latent-space sum)
+    scale is 1/sqrt(d_h + d_r) in the configs ([MLA-とは] "Decoupled RoPE",
+    softmax scaling by the concatenated dimension).
+
+    q_nope: [B,H,d_h]; q_pe: [B,H,d_r]; q_pos: [B] ints; W_UK: [H,d_h,d_c];
+    W_UV: [H,d_v,d_c]; cache: [B,cap,d_c+d_r]; seqlens: [B].
+    Returns out [B,H,d_v], o_lat [B,H,d_c], lse [B,H] (float64).
+    An empty sequence gives out = 0, o_lat = 0, lse = -inf.
+    """
+    q_nope, q_pe = _f64(q_nope), _f64(q_pe)
+    W_UK, W_UV, cache = _f64(W_UK), _f64(W_UV), _f64(cache)
+    B, H, _ = q_nope.shape
+    d_c = W_UK.shape[2]
+    d_v = W_UV.shape[1]
+    out = np.zeros((B, H, d_v))
+    o_lat = np.zeros((B, H, d_c))
+    lse = np.full((B, H), -math.inf)
+    for b in range(B):
+        L = int(seqlens[b])
+        if L == 0:
+            continue
+        c = cache[b, :L, :d_c]
+        k_pe = cache[b, :L, d_c:]
+        for i in range(H):
+            s = softmax_scale * head_logits(q_nope[b, i], q_pe[b, i],
+                                            q_pos[b], W_UK[i], c, k_pe,
+                                            rope_base)
+            p, lse[b, i] = softmax_lse(s)
+            out[b, i] = materialised_values(p, c, W_UV[i])
+            o_lat[b, i] = p @ c
+    return out, o_lat, lse
+
+
+# ---------------------------------------------------------------------------
+# The absorbed quantities, each by its own plain definition
+# ---------------------------------------------------------------------------
+def absorb_q(q_nope, q_pe, W_UK, q_pos, rope_base: float = 10000.0):
+    """q_cat[b,i] = [ W^UK_i^T q^C_{b,i} ; RoPE(q^R_{b,i}, q_pos[b]) ].
+
+    The first block is q~ := W^UK_i^T q_{t,i} in R^{d_c} ([MLA-とは] "行列吸収",
+    the per-step equation for q~); the second is the rotated decoupled query
+    ("Decoupled RoPE", q^R = R_t W^QR c^Q).  If ``q_pos`` is None the q_pe
+    input is taken as already rotated.
+    Returns [B, H, d_c + d_r] float64.
+    """
+    q_nope, q_pe, W_UK = _f64(q_nope), _f64(q_pe), _f64(W_UK)
+    q_tilde = np.einsum("bir,ird->bid", q_nope, W_UK)
+    if q_pos is None:
+        q_rot = q_pe.copy()
+    else:
+        q_rot = rope(q_pe, _f64(q_pos)[:, None], rope_base)
+    return np.concatenate([q_tilde, q_rot], axis=-1)
+
+
+def latent_attention(q_cat, cache, seqlens, softmax_scale: float,
+                     d_c: int, key_range=None):
+    """Attention of the absorbed query over the latent rows, i.e. MQA whose
+    one shared key is the whole row [c || k^R] and whose shared value is c
+    ([MLA-とは] "実装上のトレードオフ": the absorbed form is MQA with head dim
+    d_c + d_r; "Value側の吸収": the weighted sum is taken in latent space).
+
+      s_j = scale * (q_cat[b,i] . row_j)   for j in the key range
+      o_lat[b,i] = sum_j softmax(s)_j c_j,  lse[b,i] = log sum_j exp(s_j)
+
+    ``key_range`` (optional) is a (start, stop) pair per sequence, used to
+    produce split-KV partials; by default it is [0, L_b).
+    Returns o_lat [B,H,d_c], lse [B,H] (float64).  Empty ranges give 0 / -inf.
+    """
+    q_cat, cache = _f64(q_cat), _f64(cache)
+    B, H, _ = q_cat.shape
+    o_lat = np.zeros((B, H, d_c))
+    lse = np.full((B, H), -math.inf)
+    for b in range(B):
+        lo, hi = (0, int(seqlens[b])) if key_range is None else key_range[b]
+        if hi <= lo:
+            continue
+        rows = cache[b, lo:hi]  # [n, R]
+        S = softmax_scale * (q_cat[b] @ rows.T)  # [H, n]
+        for i in range(H):
+            p, lse[b, i] = softmax_lse(S[i])
+            o_lat[b, i] = p @ rows[:, :d_c]
+    return o_lat, lse
+
+
+def combine_partials(o_parts, lse_parts):
+    """Merge split-KV partial results by their log-sum-exp.
+
+    Each partial s holds o_s = softmax over its key chunk applied to the values
+    and lse_s = log of its chunk's exp-sum.  The whole-sequence result is
+        lse = log sum_s exp(lse_s),   o = sum_s exp(lse_s - lse) o_s,
+    with partials whose lse_s = -inf (empty chunks) contributing nothing and
+    an all-empty set giving o = 0, lse = -inf.  (Split-KV is not described on
+    the pages; this is the plain identity that makes chunked softmax equal the
+    unchunked one, pinned in the tests against unsplit attention.)
+
+    o_parts: [..., S, D]; lse_parts: [..., S] -> o [..., D], lse [...].
+    """
+    o_parts, lse_parts = _f64(o_parts), _f64(lse_parts)
+    m = np.max(lse_parts, axis=-1, keepdims=True)
+    finite = np.isfinite(m)
+    m_safe = np.where(finite, m, 0.0)
+    w = np.where(np.isfinite(lse_parts), np.exp(lse_parts - m_safe), 0.0)
+    z = np.sum(w, axis=-1, keepdims=True)
+    z_safe = np.where(z > 0, z, 1.0)
+    o = np.einsum("...s,...sd->...d", w / z_safe, np.where(
+        np.isfinite(lse_parts)[..., None], o_parts, 0.0))
+    lse = np.where(finite[..., 0], m_safe[..., 0] + np.log(z_safe[..., 0]),
+                   -math.inf)
+    return o, lse
+
+
+def out_proj(o_lat, W_UV) -> np.ndarray:
+    """out[b,i] = W^UV_i o_lat[b,i]: the value up-projection applied once,
+    after the latent-space weighted sum ([MLA-とは] "Value側の吸収", second
+    equation for o_{t,i}).  o_lat: [B,H,d_c]; W_UV: [H,d_v,d_c] -> [B,H,d_v]."""
+    return np.einsum("ivd,bid->biv", _f64(W_UV), _f64(o_lat))
+
+
+# ---------------------------------------------------------------------------
+# Closed forms: cache size and multiply counts
+# ---------------------------------------------------------------------------
+def cache_elems_per_token(kind: str, layers: int, n_h: int = 0, d_h: int = 0,
+                          n_g: int = 0, d_c: int = 0, d_r: int = 0) -> int:
+    """KV-cache elements per token over all layers.
+
+    MHA 2 n_h d_h l; GQA 2 n_g d_h l; MQA 2 d_h l; MLA (d_c + d_h^R) l
+    ([MLA-とは] "KVキャッシュはなぜ推論の急所なのか" and "KVキャッシュ容量の比較";
+    [attention-variants] "MLA: キャッシュする対象そのものを変える").
+    """
+    if kind == "MHA":
+        return 2 * n_h * d_h * layers
+    if kind == "GQA":
+        return 2 * n_g * d_h * layers
+    if kind == "MQA":
+        return 2 * d_h * layers
+    if kind == "MLA":
+        return (d_c + d_r) * layers
+    raise ValueError(kind)
+
+
+def mults_per_cached_token(form: str, n_h: int, d_h: int, d_c: int) -> int:
+    """Multiplies per cached token per layer for the key side.
+
+    naive: n_h d_h d_c (re-projecting every cached latent); absorbed: n_h d_c
+    (one d_c-long dot product per head); MHA: n_h d_h
+    ([MLA-とは] "行列吸収" closing paragraph and "実装上のトレードオフ", FLOPは増える).
+    """
+    if form == "naive":
+        return n_h * d_h * d_c
+    if form == "absorbed":
+        return n_h * d_c
+    if form == "MHA":
+        return n_h * d_h
+    raise ValueError(form)
