@@ -1,0 +1,464 @@
+"""Benchmark one MLA decode layer step on B200.
+
+A step is the whole decode path for one token per sequence: cache append
+(down-projection, latent RMSNorm, RoPE key), query absorption, split-KV latent
+decode, log-sum-exp combine and the W^UV output projection, on synthetic
+inputs already resident in HBM.  Sequence lengths are reset after each step so
+every step appends at the same position and attends over N + 1 rows.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the float64 CPU oracle, bounded sample)
+
+Multi-GPU: one process per GPU under torch.distributed.run; sequences are
+independent, so each rank runs its own batch with no data-path collective
+(weak scaling); time = max over ranks of the CUDA-event time.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode tokens/s and latent-cache GB/s, TFLOP/s as % of B200 roofline"
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(
+            j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def _decode_source_hash():
+    h = hashlib.sha256()
+    for name in ("k_decode_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "mla_latent_kv_nope_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(workload):
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu
+    summary, only if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        e = j[workload]
+        if e.get("source_hash") == _decode_source_hash():
+            return float(e["traffic_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (getattr(self, "out", "") or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), hw=f[5], hwt=f[6], swt=f[7],
+                                 pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        sms = sorted(r["sm"] for r in rows)
+        reasons = set()
+        for r in rows:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                            ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": rows[0]["smax"],
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+def _algorithmic(w, lens_after):
+    """Latent-cache bytes and FLOPs of one decode launch (cache read once;
+    QK^T over d_c + d_r and P.c over d_c per head and cached row)."""
+    rows = int(sum(int(x) for x in lens_after))
+    elem = 2 if w.dtype == "bf16" else 4
+    return rows * w.R * elem, 2.0 * w.H * rows * (w.R + w.d_c), rows
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import mla_latent_kv_nope_b200 as mla
+    from mla_latent_kv_nope_b200 import inputs
+    from mla_latent_kv_nope_b200.build import build
+
+    if rank == 0:
+        build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = inputs.WORKLOADS[args.workload].scaled(seed=rank)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dims = mla.Dims(w.B, w.H, w.d_c, w.d_r, w.d_nope, w.d_v, w.capacity, w.dtype)
+
+    lens = inputs.seqlens(w)
+    cache = torch.empty(w.B, w.capacity, w.R, dtype=dt, device=dev)
+    inputs.fill_cache(w, cache, lens, fill_rest=0.0)
+    seq0 = torch.from_numpy(lens).to(dev)
+    seq = seq0.clone()
+    qn, qp = inputs.query(w)
+    Wuk, Wuv = inputs.weights(w)
+    h, Wdkv = inputs.append_inputs(w)
+    T = lambda a: torch.from_numpy(a).to(dev, dt)  # noqa: E731
+    q_nope, q_pe, W_UK, W_UV, hh, W_DKV = map(T, (qn, qp, Wuk, Wuv, h, Wdkv))
+    q_pos = seq0.clone()  # the appended token's position
+    step = mla.DecodeStep(dims, W_UK, W_UV, W_DKV, num_splits=args.splits)
+    stream = torch.cuda.current_stream()
+
+    cache_bytes = cache.numel() * cache.element_size()
+    flush = None
+    if cache_bytes < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    ev_dec = []
+
+    def one_step(record=False):
+        if flush is not None:
+            flush.zero_()
+        step.append(hh, cache, seq)
+        mla.absorb_q(dims, q_nope, q_pe, W_UK, q_pos, step.q_cat, step.rope_base)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        step.splits_used = mla.decode(dims, step.q_cat, cache, seq, step.scale, step.ws,
+                                      step.num_splits)
+        mla.combine(dims, seq, step.ws, step.splits_used, step.o_lat, step.lse)
+        if record:
+            e1.record(stream)
+            ev_dec.append((e0, e1))
+        mla.out_proj(dims, step.o_lat, W_UV, step.out)
+        seq.copy_(seq0)
+
+    # Decode-kernel-only events (for the roofline): separate pass so that
+    # the step timing has no extra event records inside it.
+    def decode_only(n):
+        evs = []
+        step.append(hh, cache, seq)
+        mla.absorb_q(dims, q_nope, q_pe, W_UK, q_pos, step.q_cat, step.rope_base)
+        for _ in range(n):
+            if flush is not None:
+                flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mla.decode(dims, step.q_cat, cache, seq, step.scale, step.ws, step.num_splits)
+            e1.record(stream)
+            e2 = torch.cuda.Event(enable_timing=True)
+            mla.combine(dims, seq, step.ws, step.splits_used, step.o_lat, step.lse)
+            e2.record(stream)
+            evs.append((e0, e1, e2))
+        torch.cuda.synchronize()
+        seq.copy_(seq0)
+        return ([a.elapsed_time(b) for a, b, _ in evs], [a.elapsed_time(c) for a, _, c in evs])
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    if mla.get_device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            one_step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_total = t0.elapsed_time(t1)
+        dec_ms, decomb_ms = decode_only(max(args.steps, 5))
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+
+    # e2e through the public API with host buffers: pinned H2D of the step's
+    # inputs (q_nope, q_pe, q_pos, h) and D2H of the output, every step.
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    h_qn, h_qp, h_pos, h_h = pin(q_nope), pin(q_pe), pin(q_pos), pin(hh)
+    h_out = torch.empty(step.out.shape, dtype=dt).pin_memory()
+    bi = sum(t.numel() * t.element_size() for t in (h_qn, h_qp, h_pos, h_h))
+    bo = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        q_nope.copy_(h_qn, non_blocking=True)
+        q_pe.copy_(h_qp, non_blocking=True)
+        q_pos.copy_(h_pos, non_blocking=True)
+        hh.copy_(h_h, non_blocking=True)
+        if flush is not None:
+            flush.zero_()
+        step(q_nope, q_pe, q_pos, cache, seq, h=hh)
+        h_out.copy_(step.out, non_blocking=True)
+        seq.copy_(seq0)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / args.steps
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    if mla.get_device_status() != 0:
+        raise RuntimeError("device status error during timing")
+
+    if rank != 0:
+        return None
+    hbm, tf_burst, tf_sus, peak_src = _peaks()
+    lens_after = lens + 1
+    byts, flops, rows = _algorithmic(w, lens_after)
+    dec_avg = sum(dec_ms) / len(dec_ms)
+    decomb_avg = sum(decomb_ms) / len(decomb_ms)
+    achieved_gbs = byts / (dec_avg * 1e-3) / 1e9
+    achieved_tf = flops / (dec_avg * 1e-3) / 1e12
+    t_roof = max(byts / (hbm * 1e9), flops / (tf_burst * 1e12))
+    bound = "hbm" if byts / (hbm * 1e9) >= flops / (tf_burst * 1e12) else "tensor"
+    tokens = w.B * world
+    res = {
+        "metric": METRIC,
+        "value": tokens / (ms_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded; N(0,1) latents/queries, N(0,0.02^2) weights)",
+        "config": {
+            "workload": f"{w.name}: B={w.B} H={w.H} d_c={w.d_c} d_r={w.d_r} "
+                        f"d_nope={w.d_nope} d_v={w.d_v} N={w.N}"
+                        f"{' ragged' if w.ragged else ''} per GPU, append hidden={w.hidden}",
+            "global_batch": w.B * world,
+            "seq_len": int(lens_after.max()),
+            "parallelism": f"dp{world}",
+            "l2": ("inputs exceed L2 (cache %.0f MB)" % (cache_bytes / 1e6)) if flush is None
+                  else "L2 flushed between steps",
+            "num_splits": step.splits_used,
+        },
+        "decode_only": {
+            "ms": dec_avg, "ms_with_combine": decomb_avg,
+            "tokens_per_s": w.B / (decomb_avg * 1e-3),
+            "latent_cache_GBps": achieved_gbs, "TFLOPs": achieved_tf,
+            "roofline_us": t_roof * 1e6,
+            "frac_of_roofline": t_roof / (dec_avg * 1e-3),
+            "frac_of_roofline_with_combine": t_roof / (decomb_avg * 1e-3),
+            "hbm_frac": achieved_gbs / hbm, "tensor_frac_burst": achieved_tf / tf_burst,
+            "tensor_frac_sustained": achieved_tf / tf_sus,
+        },
+        "roofline": {
+            "kernel": "mla_decode (split-KV latent attention)",
+            "bound": bound,
+            "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
+            "peak": hbm if bound == "hbm" else tf_burst,
+            "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "frac": (achieved_gbs / hbm) if bound == "hbm" else (achieved_tf / tf_burst),
+            "traffic": _ncu_traffic(args.workload),
+            "algorithmic_bytes_per_launch": byts,
+            "algorithmic_flops_per_launch": flops,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured"
+                           else "fallback",
+        },
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_oracle_baseline(w, args.cpu_seconds)
+    return res
+
+
+# ---------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_baseline(w, budget_s=15.0):
+    """The float64 materialised-MHA oracle, as it stands, on a bounded sample
+    of the same workload: whole (sequence, head) pairs, one appended token
+    each, until about ``budget_s`` of CPU time; scaled to tokens/s by the
+    number of (sequence, head) pairs in a step."""
+    import numpy as np
+
+    from mla_latent_kv_nope_b200 import inputs
+    from oracle import mla_oracle as O
+
+    lens = inputs.seqlens(w)
+    qn, qp = inputs.query(w)
+    Wuk, Wuv = inputs.weights(w)
+    h, Wdkv = inputs.append_inputs(w)
+    f = lambda a: a.astype(np.float64)  # noqa: E731
+    done, spent = [], 0.0
+    rng = np.random.default_rng(0)
+    order = [(int(b), int(i)) for b, i in zip(rng.integers(0, w.B, 4096), rng.integers(0, w.H, 4096))]
+    cache_cache = {}
+    for b, i in order:
+        L = int(lens[b])
+        if b not in cache_cache:
+            c = np.zeros((1, L + 1, w.R))
+            c[0, :L] = inputs.cache_rows(w, b, L)
+            cache_cache = {b: c}
+        c = cache_cache[b]
+        t0 = time.perf_counter()
+        c2, L2, _ = O.cache_append(c, np.array([L]), f(h[b:b + 1]), f(Wdkv), w.d_c, eps=w.eps)
+        O.mla_decode_materialised(f(qn[b:b + 1, i:i + 1]), f(qp[b:b + 1, i:i + 1]), [L],
+                                  f(Wuk[i:i + 1]), f(Wuv[i:i + 1]), c2, L2, w.softmax_scale)
+        spent += time.perf_counter() - t0
+        done.append((b, i))
+        if spent >= budget_s:
+            break
+    per_pair = spent / len(done)
+    step_s = per_pair * w.B * w.H
+    return {"value": w.B / step_s, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{len(done)} (sequence, head) pairs of one step ({spent:.1f} s CPU), "
+                      f"each append + materialised attention over its full length; "
+                      f"scaled by B*H = {w.B * w.H} pairs per step"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle on this arm's workload (rank 0 only)."""
+    if rank != 0:
+        return None
+    from mla_latent_kv_nope_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for k in range(args.warmup + args.steps):
+        r = cpu_oracle_baseline(w, budget)
+        if k >= args.warmup:
+            vals.append(r)
+    v = sum(r["value"] for r in vals) / len(vals)
+    ms = w.B / v * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.N + 1,
+                   "parallelism": "cpu"},
+        "cpu_baseline": {"kind": "oracle", "cores": vals[-1]["cores"], "sample": vals[-1]["sample"],
+                         "value": v, "unit": "tokens/s"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="v3_bf16")
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local_rank))
+        res = run_ours(args, rank, world, local_rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,170 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) library for single-token Multi-head
+ * Latent Attention (MLA) decode over the compressed latent KV cache.
+ *
+ * What the library computes (citations are to the pages that define MLA):
+ *   [MLA-とは]  "Multi-head Latent Attention（MLA）とは？KVキャッシュを圧縮する
+ *              DeepSeekの注意機構を完全解説" (disassemble-channel.com)
+ *
+ * One decode step for a batch of B sequences, each with L_b cached tokens:
+ *   1. mla_cache_append  writes the new token's latent row
+ *                        [RMSNorm(W^DKV h) * gamma || RoPE(W^KR h, pos = L_b)]
+ *                        at row L_b and increments L_b.
+ *   2. mla_absorb_q      q_cat = [W^UK_i^T q^C ; RoPE(q^R, q_pos)] per head
+ *                        (W^UK absorbed into the query).
+ *   3. mla_decode        split-KV attention of q_cat over the latent rows:
+ *                        the latent row is the one key shared by all heads,
+ *                        its first d_c entries the shared value (MQA with head
+ *                        dim d_c + d_r).  Writes partial results.
+ *   4. mla_combine       merges the partials by log-sum-exp into
+ *                        o_lat = sum_j softmax_j c_j and lse.
+ *   5. mla_out_proj      out = W^UV_i o_lat (W^UV applied once, after the sum).
+ * K and V are never materialised.
+ *
+ * Conventions for every entry point
+ *   - All tensor arguments are caller-owned DEVICE pointers (e.g. a torch
+ *     tensor's data_ptr()), row-major and contiguous, 16-byte aligned.  The
+ *     library never allocates, frees or retains memory.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work and return; nothing synchronises except
+ *     mla_get_device_status.
+ *   - Argument, shape, alignment and workspace errors return a non-zero
+ *     status BEFORE anything is launched.  A failed launch returns
+ *     MLA_ERR_CUDA.  Errors found on the device (a sequence already at
+ *     capacity, a wait that gave up) are recorded in a per-device status word
+ *     read by mla_get_device_status.  No exception crosses the ABI.
+ *   - dtype MLA_BF16: bf16 tensors, fp32 accumulation; decode requires
+ *     d_c = 512 and d_r = 64 (the tensor-core kernel's tile shape).
+ *     dtype MLA_F32: fp32 tensors throughout; d_c, d_nope, d_v multiples of 4,
+ *     d_r even, d_c <= 1024, d_r <= 256.
+ *   - o_lat and lse are fp32 in both dtypes.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MLA_BF16 = 0, MLA_F32 = 1 } mla_dtype;
+
+/* Problem shape.  Names follow [MLA-とは]: H = n_h, d_nope = d_h (content
+ * query/key width per head), d_r = d_h^R (decoupled RoPE width), d_c = latent
+ * width (kv_lora_rank), d_v = value width per head. */
+typedef struct {
+  int32_t B;              /* sequences; one query token each */
+  int32_t H;              /* attention heads */
+  int32_t d_c;            /* latent width */
+  int32_t d_r;            /* decoupled RoPE width */
+  int32_t d_nope;         /* per-head content width of q and k */
+  int32_t d_v;            /* per-head value width */
+  int64_t cache_capacity; /* rows allocated per sequence in the cache */
+  int32_t dtype;          /* mla_dtype */
+} mla_dims;
+
+enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive or inconsistent size */
+  MLA_ERR_UNSUPPORTED = 2,    /* shape/dtype this build has no kernel for */
+  MLA_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
+  MLA_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
+  MLA_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+  MLA_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait gave up */
+  MLA_ERR_BOUNDS = 7          /* device-side index check failed (e.g. cache full) */
+};
+
+/* Elements of one latent cache row per token per layer: d_c + d_r
+ * ([MLA-とは] "KVキャッシュ容量の比較": MLA caches (d_c + d_h^R) per layer). */
+MLA_API int64_t mla_cache_row_elems(int32_t d_c, int32_t d_r);
+
+/* --- 1. cache append ------------------------------------------------------
+ * [MLA-とは] "MLAの発想" (c^KV_t = W^DKV h_t), "Decoupled RoPE"
+ * (k^R_j = R_j W^KR h_j, cached already rotated), "実装上のトレードオフ"
+ * (the normalised latent is cached).  For each sequence b:
+ *   x = W_DKV h_b (fp32 accumulation);  c = x[0:d_c] / sqrt(mean(x[0:d_c]^2) + eps) * gamma
+ *   k = RoPE(x[d_c:d_c+d_r], pos = L_b) (half-split pairs, theta_k = pos * base^(-2k/d_r))
+ *   cache[b, L_b, :] = [c || k] rounded once to the cache dtype;  seqlens[b] = L_b + 1
+ * h       [B, hidden]                 dtype
+ * W_DKV   [d_c + d_r, hidden]         dtype; rows 0..d_c-1 = W^DKV, the rest = W^KR
+ * gamma   [d_c] fp32, or NULL for ones
+ * cache   [B, cache_capacity, d_c + d_r] dtype, written at row L_b only
+ * seqlens [B] int32, read then incremented on the device
+ * workspace  >= mla_cache_append_workspace_bytes(dims) bytes of device scratch
+ * A sequence already at capacity is left untouched and sets MLA_ERR_BOUNDS in
+ * the device status word. */
+MLA_API size_t mla_cache_append_workspace_bytes(const mla_dims* dims);
+MLA_API int mla_cache_append(const mla_dims* dims, int32_t hidden, const void* h,
+                     const void* W_DKV, const float* gamma, float eps,
+                     float rope_base, void* cache, int32_t* seqlens,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* --- 2. query absorption --------------------------------------------------
+ * [MLA-とは] "行列吸収": q~_{t,i} = W^UK_i^T q_{t,i} in R^{d_c};
+ * "Decoupled RoPE": q^R rotated at the query position.
+ *   q_cat[b,i,0:d_c]      = sum_r q_nope[b,i,r] W_UK[i,r,:]
+ *   q_cat[b,i,d_c:d_c+d_r] = RoPE(q_pe[b,i], q_pos[b])   (q_pos == NULL: copied as given)
+ * q_nope [B,H,d_nope], q_pe [B,H,d_r], W_UK [H,d_nope,d_c] (dtype);
+ * q_pos [B] int32 or NULL; q_cat [B,H,d_c+d_r] (dtype, rounded once). */
+MLA_API int mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q_pe,
+                 const void* W_UK, const int32_t* q_pos, float rope_base,
+                 void* q_cat, void* stream);
+
+/* --- 3. split-KV latent decode --------------------------------------------
+ * [MLA-とは] "実装上のトレードオフ" (absorbed form = MQA with head dim
+ * d_c + d_r), "Value側の吸収" (weighted sum in latent space), "Decoupled
+ * RoPE" (softmax scale 1/sqrt(d_h + d_h^R) in the pages' configs).
+ * For sequence b, head i and cached rows j < L_b:
+ *   s_j = softmax_scale * (q_cat[b,i] . cache[b,j,:])
+ * The key space of all sequences, cut into tiles of 64 rows, is dealt into
+ * `num_splits` contiguous ranges (worker w takes tiles [w*T/W, (w+1)*T/W) of
+ * the concatenated per-sequence tile lists, T = sum_b ceil(L_b/64)).  Worker w
+ * writes, for each sequence b it touches, partial slot (b + w):
+ *   o_part[b+w][i][:] = sum_{j in range} e^{s_j - lse_part} c_j,   lse_part[b+w][i] = log sum e^{s_j}
+ * Workspace layout (fp32): o_part [B + W - 1][H][d_c], then lse_part [B + W - 1][H].
+ * Rows j >= L_b never influence the result (they may hold anything).
+ * num_splits = 0 picks the default for the current device; the number used is
+ * returned through splits_used (may be NULL). */
+MLA_API int mla_decode_default_splits(const mla_dims* dims);
+MLA_API size_t mla_decode_workspace_bytes(const mla_dims* dims, int num_splits);
+MLA_API int mla_decode(const mla_dims* dims, const void* q_cat, const void* cache,
+               const int32_t* seqlens, float softmax_scale, int num_splits,
+               void* workspace, size_t workspace_bytes, int* splits_used,
+               void* stream);
+
+/* --- 4. log-sum-exp combine ------------------------------------------------
+ * Merges the partials of mla_decode (same dims, seqlens and splits_used):
+ *   lse[b,i] = log sum_s exp(lse_part_s),  o_lat[b,i] = sum_s exp(lse_part_s - lse[b,i]) o_part_s
+ * An empty sequence (L_b = 0) gives o_lat = 0 and lse = -inf.
+ * o_lat [B,H,d_c] fp32; lse [B,H] fp32 (may be NULL). */
+MLA_API int mla_combine(const mla_dims* dims, const int32_t* seqlens,
+                const void* workspace, size_t workspace_bytes, int splits_used,
+                float* o_lat, float* lse, void* stream);
+
+/* --- 5. value up-projection -------------------------------------------------
+ * [MLA-とは] "Value側の吸収": o_{t,i} = W^UV_i (sum_j a_{tj,i} c^KV_j).
+ *   out[b,i,v] = sum_c W_UV[i,v,c] o_lat[b,i,c]
+ * o_lat [B,H,d_c] fp32; W_UV [H,d_v,d_c] dtype; out [B,H,d_v] dtype. */
+MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W_UV,
+                 void* out, void* stream);
+
+/* --- status ------------------------------------------------------------------
+ * Synchronises `stream`, then returns and clears the current device's status
+ * word (MLA_OK if no device-side error was recorded since the last call).
+ * Returns MLA_ERR_CUDA if the synchronisation itself failed. */
+MLA_API int mla_get_device_status(void* stream);
+MLA_API const char* mla_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,10 @@
+"""B200-native (sm_100a) single-token MLA decode over the latent KV cache.
+
+The compute lives in ``libmla_b200.so`` (hand-written CUDA kernels behind the C
+ABI declared in ``include/mla.h``); ``binding`` marshals torch tensors to it.
+"""
+from .binding import (  # noqa: F401
+    Dims, DecodeStep, MLAError, absorb_q, cache_append, cache_append_workspace_bytes,
+    cache_row_elems, combine, decode, decode_default_splits, decode_workspace_bytes,
+    get_device_status, load_library, out_proj,
+)

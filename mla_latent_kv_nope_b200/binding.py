@@ -1,0 +1,265 @@
+"""Thin Python binding of the C ABI in ``include/mla.h`` (ctypes).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of ``libmla_b200.so``.  Tensors are torch CUDA tensors (device memory
+and streams only); each call enqueues on the current torch stream.  A missing
+library raises immediately -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
+
+MLA_BF16, MLA_F32 = 0, 1
+STATUS = {
+    0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
+    3: "MLA_ERR_ALIGNMENT", 4: "MLA_ERR_WORKSPACE", 5: "MLA_ERR_CUDA",
+    6: "MLA_ERR_DEVICE_TIMEOUT", 7: "MLA_ERR_BOUNDS",
+}
+EXPORTED = (
+    "mla_cache_row_elems", "mla_cache_append_workspace_bytes", "mla_cache_append",
+    "mla_absorb_q", "mla_decode_default_splits", "mla_decode_workspace_bytes",
+    "mla_decode", "mla_combine", "mla_out_proj", "mla_get_device_status",
+    "mla_status_string",
+)
+
+
+class MLAError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({msg})")
+        self.status = status
+
+
+class CDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d_c", ctypes.c_int32),
+                ("d_r", ctypes.c_int32), ("d_nope", ctypes.c_int32), ("d_v", ctypes.c_int32),
+                ("cache_capacity", ctypes.c_int64), ("dtype", ctypes.c_int32)]
+
+
+@dataclass(frozen=True)
+class Dims:
+    """Problem shape (names as in the header: H heads, d_c latent width,
+    d_r decoupled-RoPE width, d_nope / d_v per-head content / value widths)."""
+    B: int
+    H: int
+    d_c: int
+    d_r: int
+    d_nope: int
+    d_v: int
+    cache_capacity: int
+    dtype: str = "bf16"  # "bf16" | "f32"
+
+    def c(self) -> CDims:
+        return CDims(self.B, self.H, self.d_c, self.d_r, self.d_nope, self.d_v,
+                     self.cache_capacity, MLA_BF16 if self.dtype == "bf16" else MLA_F32)
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    @property
+    def R(self) -> int:
+        return self.d_c + self.d_r
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the sm_100a library.  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with mla_latent_kv_nope_b200.build.build(); "
+            "there is no non-CUDA implementation")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, SZ, F = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
+                          ctypes.c_float)
+    D = ctypes.POINTER(CDims)
+    sig = {
+        "mla_cache_row_elems": (I64, [I32, I32]),
+        "mla_cache_append_workspace_bytes": (SZ, [D]),
+        "mla_cache_append": (ctypes.c_int, [D, I32, P, P, P, F, F, P, P, P, SZ, P]),
+        "mla_absorb_q": (ctypes.c_int, [D, P, P, P, P, F, P, P]),
+        "mla_decode_default_splits": (ctypes.c_int, [D]),
+        "mla_decode_workspace_bytes": (SZ, [D, ctypes.c_int]),
+        "mla_decode": (ctypes.c_int, [D, P, P, P, F, ctypes.c_int, P, SZ,
+                                      ctypes.POINTER(ctypes.c_int), P]),
+        "mla_combine": (ctypes.c_int, [D, P, P, SZ, ctypes.c_int, P, P, P]),
+        "mla_out_proj": (ctypes.c_int, [D, P, P, P, P]),
+        "mla_get_device_status": (ctypes.c_int, [P]),
+        "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        msg = load_library().mla_status_string(status).decode()
+        raise MLAError(fn, status, msg)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_cuda:
+        raise ValueError(f"{name}: expected CUDA {dtype} {tuple(shape)}, got "
+                         f"{t.device} {t.dtype} {tuple(t.shape)}")
+
+
+# ---------------------------------------------------------------------------
+def cache_row_elems(d_c: int, d_r: int) -> int:
+    return int(load_library().mla_cache_row_elems(d_c, d_r))
+
+
+def cache_append_workspace_bytes(dims: Dims) -> int:
+    return int(load_library().mla_cache_append_workspace_bytes(ctypes.byref(dims.c())))
+
+
+def cache_append(dims: Dims, h, W_DKV, gamma, cache, seqlens, workspace, eps=1e-6,
+                 rope_base=10000.0, stream=None):
+    dt = dims.torch_dtype
+    hidden = h.shape[-1]
+    _need(h, dt, (dims.B, hidden), "h")
+    _need(W_DKV, dt, (dims.R, hidden), "W_DKV")
+    _need(cache, dt, (dims.B, dims.cache_capacity, dims.R), "cache")
+    _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    if gamma is not None:
+        _need(gamma, torch.float32, (dims.d_c,), "gamma")
+    st = load_library().mla_cache_append(
+        ctypes.byref(dims.c()), hidden, _ptr(h), _ptr(W_DKV), _ptr(gamma), eps, rope_base,
+        _ptr(cache), _ptr(seqlens), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("mla_cache_append", st)
+
+
+def absorb_q(dims: Dims, q_nope, q_pe, W_UK, q_pos, q_cat, rope_base=10000.0, stream=None):
+    dt = dims.torch_dtype
+    _need(q_nope, dt, (dims.B, dims.H, dims.d_nope), "q_nope")
+    _need(q_pe, dt, (dims.B, dims.H, dims.d_r), "q_pe")
+    _need(W_UK, dt, (dims.H, dims.d_nope, dims.d_c), "W_UK")
+    _need(q_cat, dt, (dims.B, dims.H, dims.R), "q_cat")
+    if q_pos is not None:
+        _need(q_pos, torch.int32, (dims.B,), "q_pos")
+    st = load_library().mla_absorb_q(ctypes.byref(dims.c()), _ptr(q_nope), _ptr(q_pe),
+                                     _ptr(W_UK), _ptr(q_pos), rope_base, _ptr(q_cat),
+                                     _stream(stream))
+    _check("mla_absorb_q", st)
+
+
+def decode_default_splits(dims: Dims) -> int:
+    return int(load_library().mla_decode_default_splits(ctypes.byref(dims.c())))
+
+
+def decode_workspace_bytes(dims: Dims, num_splits: int = 0) -> int:
+    return int(load_library().mla_decode_workspace_bytes(ctypes.byref(dims.c()), num_splits))
+
+
+def decode(dims: Dims, q_cat, cache, seqlens, softmax_scale, workspace, num_splits=0,
+           stream=None) -> int:
+    dt = dims.torch_dtype
+    _need(q_cat, dt, (dims.B, dims.H, dims.R), "q_cat")
+    _need(cache, dt, (dims.B, dims.cache_capacity, dims.R), "cache")
+    _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    used = ctypes.c_int(0)
+    st = load_library().mla_decode(ctypes.byref(dims.c()), _ptr(q_cat), _ptr(cache),
+                                   _ptr(seqlens), float(softmax_scale), num_splits,
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   ctypes.byref(used), _stream(stream))
+    _check("mla_decode", st)
+    return used.value
+
+
+def combine(dims: Dims, seqlens, workspace, splits_used, o_lat, lse=None, stream=None):
+    _need(o_lat, torch.float32, (dims.B, dims.H, dims.d_c), "o_lat")
+    if lse is not None:
+        _need(lse, torch.float32, (dims.B, dims.H), "lse")
+    st = load_library().mla_combine(ctypes.byref(dims.c()), _ptr(seqlens), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), splits_used,
+                                    _ptr(o_lat), _ptr(lse), _stream(stream))
+    _check("mla_combine", st)
+
+
+def out_proj(dims: Dims, o_lat, W_UV, out, stream=None):
+    dt = dims.torch_dtype
+    _need(o_lat, torch.float32, (dims.B, dims.H, dims.d_c), "o_lat")
+    _need(W_UV, dt, (dims.H, dims.d_v, dims.d_c), "W_UV")
+    _need(out, dt, (dims.B, dims.H, dims.d_v), "out")
+    st = load_library().mla_out_proj(ctypes.byref(dims.c()), _ptr(o_lat), _ptr(W_UV), _ptr(out),
+                                     _stream(stream))
+    _check("mla_out_proj", st)
+
+
+def get_device_status(stream=None) -> int:
+    return int(load_library().mla_get_device_status(_stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+class DecodeStep:
+    """One MLA decode layer on the device: owns its workspaces (allocated once
+    by the caller side through torch) and runs append -> absorb_q -> decode ->
+    combine -> out_proj on the current stream.  All arithmetic is in the CUDA
+    kernels; this class only keeps buffers and pointers."""
+
+    def __init__(self, dims: Dims, W_UK, W_UV, W_DKV=None, gamma=None, softmax_scale=None,
+                 rope_base=10000.0, eps=1e-6, num_splits=0, device="cuda"):
+        self.dims = dims
+        self.W_UK, self.W_UV, self.W_DKV, self.gamma = W_UK, W_UV, W_DKV, gamma
+        self.scale = (softmax_scale if softmax_scale is not None
+                      else (dims.d_nope + dims.d_r) ** -0.5)
+        self.rope_base, self.eps = rope_base, eps
+        self.num_splits = num_splits or decode_default_splits(dims)
+        ws = decode_workspace_bytes(dims, self.num_splits)
+        self.ws = torch.empty(ws // 4, dtype=torch.float32, device=device)
+        self.ws_append = torch.empty(max(cache_append_workspace_bytes(dims) // 4, 1),
+                                     dtype=torch.float32, device=device)
+        dt = dims.torch_dtype
+        self.q_cat = torch.empty(dims.B, dims.H, dims.R, dtype=dt, device=device)
+        self.o_lat = torch.empty(dims.B, dims.H, dims.d_c, dtype=torch.float32, device=device)
+        self.lse = torch.empty(dims.B, dims.H, dtype=torch.float32, device=device)
+        self.out = torch.empty(dims.B, dims.H, dims.d_v, dtype=dt, device=device)
+        self.splits_used = self.num_splits
+
+    def append(self, h, cache, seqlens):
+        cache_append(self.dims, h, self.W_DKV, self.gamma, cache, seqlens, self.ws_append,
+                     self.eps, self.rope_base)
+
+    def attend(self, q_nope, q_pe, q_pos, cache, seqlens):
+        absorb_q(self.dims, q_nope, q_pe, self.W_UK, q_pos, self.q_cat, self.rope_base)
+        self.splits_used = decode(self.dims, self.q_cat, cache, seqlens, self.scale, self.ws,
+                                  self.num_splits)
+        combine(self.dims, seqlens, self.ws, self.splits_used, self.o_lat, self.lse)
+        out_proj(self.dims, self.o_lat, self.W_UV, self.out)
+        return self.out
+
+    def __call__(self, q_nope, q_pe, q_pos, cache, seqlens, h=None):
+        if h is not None:
+            self.append(h, cache, seqlens)
+        return self.attend(q_nope, q_pe, q_pos, cache, seqlens)

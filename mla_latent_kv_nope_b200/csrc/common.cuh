@@ -1,0 +1,85 @@
+// Shared device helpers for the MLA decode library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+
+namespace mla {
+
+// Keys per work tile.  The split-KV work list, the combine and every decode
+// kernel agree on this unit.
+constexpr int kTileKeys = 64;
+
+// Device code records the first error it meets (bounds, timeout) in the
+// per-device status word whose address the host passes to the kernel;
+// mla_get_device_status reads and clears it.
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicCAS(status, MLA_OK, code);
+}
+
+template <typename T> struct Storage;
+template <> struct Storage<float> {
+  static __device__ __forceinline__ float load(const float* p) { return *p; }
+  static __device__ __forceinline__ float to_f(float v) { return v; }
+  static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <> struct Storage<__nv_bfloat16> {
+  static __device__ __forceinline__ float load(const __nv_bfloat16* p) {
+    return __bfloat162float(*p);
+  }
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 v) {
+    return __bfloat162float(v);
+  }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float v) {
+    return __float2bfloat16_rn(v);
+  }
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Usable length of a sequence: the stored length clamped to [0, capacity], so
+// that a corrupt length can never index past the cache.
+__device__ __forceinline__ int64_t clamp_len(int32_t L, int64_t cap) {
+  return L <= 0 ? 0 : (int64_t(L) > cap ? cap : int64_t(L));
+}
+
+// Number of 64-key tiles of a sequence of (clamped) length L.
+__device__ __forceinline__ int64_t tiles_of(int64_t L) {
+  return L > 0 ? (L + kTileKeys - 1) / kTileKeys : 0;
+}
+
+// First tile owned by worker w of W over T tiles: floor(w*T/W).
+__device__ __forceinline__ int64_t worker_tile_begin(int64_t w, int64_t T, int64_t W) {
+  return (w * T) / W;
+}
+// Worker owning tile t: the largest w with floor(w*T/W) <= t.
+__device__ __forceinline__ int64_t worker_of_tile(int64_t t, int64_t T, int64_t W) {
+  return ((t + 1) * W - 1) / T;
+}
+
+// RoPE angle pair for element pair k of a d-wide rotary block at position pos:
+// theta = pos * base^(-2k/d), evaluated in double so that long contexts keep
+// full fp32 accuracy after the reduction.
+__device__ __forceinline__ void rope_cos_sin(int64_t pos, int k, int d, float base,
+                                             float* c, float* s) {
+  double inv = pow(double(base), -2.0 * double(k) / double(d));
+  double th = double(pos) * inv;
+  double sd, cd;
+  sincos(th, &sd, &cd);
+  *c = float(cd);
+  *s = float(sd);
+}
+
+}  // namespace mla

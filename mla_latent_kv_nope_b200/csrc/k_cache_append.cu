@@ -1,0 +1,138 @@
+// Cache append: one new latent row per sequence.
+//   x = W_DKV h_b                                  ([MLA-とは] "MLAの発想", c^KV = W^DKV h;
+//                                                   "Decoupled RoPE", k^R = R_j W^KR h_j)
+//   c = x[0:d_c] / sqrt(mean(x[0:d_c]^2) + eps) * gamma   (latent RMSNorm, 正規化の扱い)
+//   k = RoPE(x[d_c:], pos = L_b)
+//   cache[b, L_b] = [c || k];  L_b += 1
+//
+// Two passes.  The projection pass reads W_DKV once: block = 4 rows of W_DKV,
+// all sequences (in chunks of 16), every thread striding over the hidden
+// dimension, then a block reduction; it writes x to the fp32 workspace.  The
+// finalize pass (block per sequence) applies the norm, the rotation and the
+// single rounding, checks the capacity, writes row L_b and bumps L_b.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mla {
+
+namespace {
+
+constexpr int kApRows = 4;
+constexpr int kApBatch = 16;
+constexpr int kApThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kApThreads)
+append_project_kernel(const T* __restrict__ h, const T* __restrict__ W, int B, int R,
+                      int hidden, float* __restrict__ x_out) {
+  __shared__ float s_red[kApThreads / 32][kApRows * kApBatch];
+  const int r0 = blockIdx.x * kApRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int b0 = 0; b0 < B; b0 += kApBatch) {
+    const int nb = min(kApBatch, B - b0);
+    float acc[kApRows][kApBatch];
+#pragma unroll
+    for (int r = 0; r < kApRows; ++r)
+#pragma unroll
+      for (int bb = 0; bb < kApBatch; ++bb) acc[r][bb] = 0.f;
+    for (int k = threadIdx.x; k < hidden; k += kApThreads) {
+      float wv[kApRows];
+#pragma unroll
+      for (int r = 0; r < kApRows; ++r)
+        wv[r] = (r0 + r < R) ? Storage<T>::to_f(W[int64_t(r0 + r) * hidden + k]) : 0.f;
+#pragma unroll
+      for (int bb = 0; bb < kApBatch; ++bb) {
+        if (bb < nb) {
+          const float hv = Storage<T>::to_f(h[int64_t(b0 + bb) * hidden + k]);
+#pragma unroll
+          for (int r = 0; r < kApRows; ++r) acc[r][bb] = fmaf(wv[r], hv, acc[r][bb]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kApRows; ++r)
+#pragma unroll
+      for (int bb = 0; bb < kApBatch; ++bb) {
+        const float v = warp_sum(acc[r][bb]);
+        if (lane == 0) s_red[warp][r * kApBatch + bb] = v;
+      }
+    __syncthreads();
+    if (threadIdx.x < kApRows * kApBatch) {
+      const int r = threadIdx.x / kApBatch, bb = threadIdx.x % kApBatch;
+      float v = 0.f;
+#pragma unroll
+      for (int wdx = 0; wdx < kApThreads / 32; ++wdx) v += s_red[wdx][threadIdx.x];
+      if (r0 + r < R && bb < nb) x_out[int64_t(b0 + bb) * R + r0 + r] = v;
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kApThreads)
+append_finalize_kernel(const float* __restrict__ x, const float* __restrict__ gamma,
+                       float eps, float rope_base, int d_c, int d_r, int64_t cap,
+                       T* __restrict__ cache, int32_t* __restrict__ seqlens,
+                       int* __restrict__ status) {
+  const int b = blockIdx.x;
+  const int R = d_c + d_r;
+  __shared__ float s_part[kApThreads / 32];
+  __shared__ int32_t s_L;
+  if (threadIdx.x == 0) s_L = seqlens[b];
+  const float* xb = x + int64_t(b) * R;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d_c; c += kApThreads) ss = fmaf(xb[c], xb[c], ss);
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  const int32_t L = s_L;
+  if (L < 0 || int64_t(L) >= cap) {
+    if (threadIdx.x == 0) record_status(status, MLA_ERR_BOUNDS);
+    return;
+  }
+  float tot = 0.f;
+#pragma unroll
+  for (int wdx = 0; wdx < kApThreads / 32; ++wdx) tot += s_part[wdx];
+  const float inv = 1.f / sqrtf(tot / float(d_c) + eps);
+  T* row = cache + (int64_t(b) * cap + L) * R;
+  for (int c = threadIdx.x; c < d_c; c += kApThreads) {
+    const float g = gamma ? gamma[c] : 1.f;
+    row[c] = Storage<T>::from_f(xb[c] * inv * g);
+  }
+  const int half = d_r / 2;
+  for (int k = threadIdx.x; k < half; k += kApThreads) {
+    float cs, sn;
+    rope_cos_sin(L, k, d_r, rope_base, &cs, &sn);
+    const float x1 = xb[d_c + k], x2 = xb[d_c + k + half];
+    row[d_c + k] = Storage<T>::from_f(x1 * cs - x2 * sn);
+    row[d_c + k + half] = Storage<T>::from_f(x1 * sn + x2 * cs);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) seqlens[b] = L + 1;
+}
+
+}  // namespace
+
+template <typename T>
+cudaError_t launch_cache_append(const T* h, const T* W_DKV, const float* gamma, float eps,
+                                float rope_base, int B, int d_c, int d_r, int hidden,
+                                int64_t cap, T* cache, int32_t* seqlens, float* x_ws,
+                                int* status, cudaStream_t stream) {
+  const int R = d_c + d_r;
+  append_project_kernel<T><<<(R + kApRows - 1) / kApRows, kApThreads, 0, stream>>>(
+      h, W_DKV, B, R, hidden, x_ws);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  append_finalize_kernel<T><<<B, kApThreads, 0, stream>>>(x_ws, gamma, eps, rope_base, d_c,
+                                                          d_r, cap, cache, seqlens, status);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_cache_append<float>(const float*, const float*, const float*,
+                                                float, float, int, int, int, int, int64_t,
+                                                float*, int32_t*, float*, int*, cudaStream_t);
+template cudaError_t launch_cache_append<__nv_bfloat16>(
+    const __nv_bfloat16*, const __nv_bfloat16*, const float*, float, float, int, int, int,
+    int, int64_t, __nv_bfloat16*, int32_t*, float*, int*, cudaStream_t);
+
+}  // namespace mla

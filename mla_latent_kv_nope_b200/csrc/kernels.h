@@ -1,0 +1,45 @@
+// Internal launch functions (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mla {
+
+template <typename T>
+cudaError_t launch_absorb_q(const T* q_nope, const T* q_pe, const T* W_UK,
+                            const int32_t* q_pos, float rope_base, int B, int H, int d_c,
+                            int d_r, int d_n, T* q_cat, cudaStream_t stream);
+
+template <typename T>
+cudaError_t launch_decode_simt(const T* q_cat, const T* cache, const int32_t* seqlens,
+                               int B, int H, int d_c, int d_r, int64_t cap, float scale,
+                               int W, float* o_part, float* lse_part, int* status,
+                               cudaStream_t stream);
+size_t decode_simt_smem_bytes(int d_c, int d_r);
+
+// Tensor-core decode (bf16, d_c = 512, d_r = 64).  Returns cudaErrorNotSupported
+// when the build has no sm_100a kernel.
+cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* cache,
+                             const int32_t* seqlens, int B, int H, int64_t cap, float scale,
+                             int W, float* o_part, float* lse_part, int* status,
+                             cudaStream_t stream);
+int decode_tc_head_groups(int H);
+
+cudaError_t launch_combine(const int32_t* seqlens, int64_t cap, int B, int H, int d_c, int W,
+                           const float* o_part, const float* lse_part, float* o_lat,
+                           float* lse, cudaStream_t stream);
+
+template <typename T>
+cudaError_t launch_out_proj(const float* o_lat, const T* W_UV, int B, int H, int d_c,
+                            int d_v, T* out, cudaStream_t stream);
+
+template <typename T>
+cudaError_t launch_cache_append(const T* h, const T* W_DKV, const float* gamma, float eps,
+                                float rope_base, int B, int d_c, int d_r, int hidden,
+                                int64_t cap, T* cache, int32_t* seqlens, float* x_ws,
+                                int* status, cudaStream_t stream);
+
+}  // namespace mla

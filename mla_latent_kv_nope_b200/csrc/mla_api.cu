@@ -1,0 +1,265 @@
+// C ABI of the MLA decode library: argument validation, workspace layout and
+// kernel launches.  Every check runs before anything is enqueued; no entry
+// point allocates, frees or synchronises (except mla_get_device_status).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/mla.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mla {
+
+// Per-device status word (one copy per device that loads the library).
+__device__ int g_status = MLA_OK;
+
+namespace {
+
+// Device address of g_status for the current device, looked up once per
+// device.  Host code may not take the address of a __device__ symbol
+// directly; the runtime lookup gives the real device pointer.
+int* status_ptr() {
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+constexpr int kMaxSplits = 1024;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int check_dims(const mla_dims* d) {
+  if (!d) return MLA_ERR_INVALID_ARG;
+  if (d->B <= 0 || d->H <= 0 || d->d_c <= 0 || d->d_r < 0 || d->d_nope <= 0 || d->d_v <= 0 ||
+      d->cache_capacity <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (d->B > 65535 || d->H > 65535) return MLA_ERR_UNSUPPORTED;
+  if (d->dtype == MLA_BF16) {
+    if (d->d_c % 8 || d->d_r % 8 || d->d_nope % 8 || d->d_v % 8) return MLA_ERR_UNSUPPORTED;
+  } else if (d->dtype == MLA_F32) {
+    if (d->d_c % 4 || d->d_r % 2 || d->d_nope % 4 || d->d_v % 4) return MLA_ERR_UNSUPPORTED;
+  } else {
+    return MLA_ERR_INVALID_ARG;
+  }
+  if (d->d_c > 1024 || d->d_r > 256 || d->d_nope > 1024 || d->d_v > 1024)
+    return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+inline bool decode_uses_tc(const mla_dims* d) { return d->dtype == MLA_BF16; }
+
+int decode_shape_supported(const mla_dims* d) {
+  if (d->dtype == MLA_BF16 && (d->d_c != 512 || d->d_r != 64)) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+struct WsLayout {
+  size_t o_off, lse_off, total;
+};
+
+WsLayout ws_layout(const mla_dims* d, int W) {
+  const size_t slots = size_t(d->B) + size_t(W) - 1;
+  WsLayout l;
+  l.o_off = 0;
+  l.lse_off = round_up(slots * size_t(d->H) * size_t(d->d_c) * sizeof(float), 256);
+  l.total = l.lse_off + round_up(slots * size_t(d->H) * sizeof(float), 256);
+  return l;
+}
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+}  // namespace
+}  // namespace mla
+
+using namespace mla;
+
+extern "C" {
+
+int64_t mla_cache_row_elems(int32_t d_c, int32_t d_r) { return int64_t(d_c) + int64_t(d_r); }
+
+const char* mla_status_string(int s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MLA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case MLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MLA_ERR_BOUNDS: return "device-side bounds check failed";
+    default: return "unknown status";
+  }
+}
+
+int mla_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  int v = MLA_OK;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  const int zero = MLA_OK;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+size_t mla_cache_append_workspace_bytes(const mla_dims* d) {
+  if (check_dims(d) != MLA_OK) return 0;
+  return round_up(size_t(d->B) * size_t(d->d_c + d->d_r) * sizeof(float), 256);
+}
+
+int mla_cache_append(const mla_dims* d, int32_t hidden, const void* h, const void* W_DKV,
+                     const float* gamma, float eps, float rope_base, void* cache,
+                     int32_t* seqlens, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if (hidden <= 0 || !h || !W_DKV || !cache || !seqlens) return MLA_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !(rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
+  if (d->dtype == MLA_BF16 ? (hidden % 8) : (hidden % 4)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(h) || !aligned16(W_DKV) || !aligned16(cache) || !aligned16(seqlens) ||
+      (gamma && !aligned16(gamma)) || (workspace && !aligned16(workspace)))
+    return MLA_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < mla_cache_append_workspace_bytes(d)) return MLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* x = static_cast<float*>(workspace);
+  if (d->dtype == MLA_BF16)
+    return cuda_status(launch_cache_append<__nv_bfloat16>(
+        static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(W_DKV), gamma,
+        eps, rope_base, d->B, d->d_c, d->d_r, hidden, d->cache_capacity,
+        static_cast<__nv_bfloat16*>(cache), seqlens, x, status_ptr(), s));
+  return cuda_status(launch_cache_append<float>(
+      static_cast<const float*>(h), static_cast<const float*>(W_DKV), gamma, eps, rope_base,
+      d->B, d->d_c, d->d_r, hidden, d->cache_capacity, static_cast<float*>(cache), seqlens, x,
+      status_ptr(), s));
+}
+
+// ---------------------------------------------------------------------------
+int mla_absorb_q(const mla_dims* d, const void* q_nope, const void* q_pe, const void* W_UK,
+                 const int32_t* q_pos, float rope_base, void* q_cat, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if (!q_nope || (d->d_r && !q_pe) || !W_UK || !q_cat) return MLA_ERR_INVALID_ARG;
+  if (q_pos && !(rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || (q_pe && !aligned16(q_pe)) || !aligned16(W_UK) ||
+      !aligned16(q_cat) || (q_pos && !aligned16(q_pos)))
+    return MLA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->dtype == MLA_BF16)
+    return cuda_status(launch_absorb_q<__nv_bfloat16>(
+        static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_pe),
+        static_cast<const __nv_bfloat16*>(W_UK), q_pos, rope_base, d->B, d->H, d->d_c, d->d_r,
+        d->d_nope, static_cast<__nv_bfloat16*>(q_cat), s));
+  return cuda_status(launch_absorb_q<float>(
+      static_cast<const float*>(q_nope), static_cast<const float*>(q_pe),
+      static_cast<const float*>(W_UK), q_pos, rope_base, d->B, d->H, d->d_c, d->d_r, d->d_nope,
+      static_cast<float*>(q_cat), s));
+}
+
+// ---------------------------------------------------------------------------
+int mla_decode_default_splits(const mla_dims* d) {
+  if (check_dims(d) != MLA_OK) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  int W;
+  if (decode_uses_tc(d)) {
+    W = sms / decode_tc_head_groups(d->H);
+  } else {
+    const int groups = (d->H + 7) / 8;
+    W = (2 * sms + groups - 1) / groups;
+  }
+  if (W < 1) W = 1;
+  if (W > kMaxSplits) W = kMaxSplits;
+  return W;
+}
+
+size_t mla_decode_workspace_bytes(const mla_dims* d, int num_splits) {
+  if (check_dims(d) != MLA_OK) return 0;
+  const int W = num_splits > 0 ? num_splits : mla_decode_default_splits(d);
+  if (W <= 0 || W > kMaxSplits) return 0;
+  return ws_layout(d, W).total;
+}
+
+int mla_decode(const mla_dims* d, const void* q_cat, const void* cache, const int32_t* seqlens,
+               float softmax_scale, int num_splits, void* workspace, size_t workspace_bytes,
+               int* splits_used, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if ((st = decode_shape_supported(d))) return st;
+  if (!q_cat || !cache || !seqlens || num_splits < 0 || num_splits > kMaxSplits ||
+      !(softmax_scale > 0.f) || softmax_scale == INFINITY)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_cat) || !aligned16(cache) || !aligned16(seqlens) ||
+      (workspace && !aligned16(workspace)))
+    return MLA_ERR_ALIGNMENT;
+  const int W = num_splits > 0 ? num_splits : mla_decode_default_splits(d);
+  if (W <= 0) return MLA_ERR_CUDA;
+  const WsLayout l = ws_layout(d, W);
+  if (!workspace || workspace_bytes < l.total) return MLA_ERR_WORKSPACE;
+  if (splits_used) *splits_used = W;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + l.o_off);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + l.lse_off);
+  if (d->dtype == MLA_BF16)
+    return cuda_status(launch_decode_tc(static_cast<const __nv_bfloat16*>(q_cat),
+                                        static_cast<const __nv_bfloat16*>(cache), seqlens, d->B,
+                                        d->H, d->cache_capacity, softmax_scale, W, o_part,
+                                        lse_part, status_ptr(), s));
+  return cuda_status(launch_decode_simt<float>(static_cast<const float*>(q_cat),
+                                               static_cast<const float*>(cache), seqlens, d->B,
+                                               d->H, d->d_c, d->d_r, d->cache_capacity,
+                                               softmax_scale, W, o_part, lse_part, status_ptr(),
+                                               s));
+}
+
+// ---------------------------------------------------------------------------
+int mla_combine(const mla_dims* d, const int32_t* seqlens, const void* workspace,
+                size_t workspace_bytes, int splits_used, float* o_lat, float* lse, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if (!seqlens || !workspace || !o_lat || splits_used <= 0 || splits_used > kMaxSplits)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(seqlens) || !aligned16(workspace) || !aligned16(o_lat) ||
+      (lse && !aligned16(lse)))
+    return MLA_ERR_ALIGNMENT;
+  const WsLayout l = ws_layout(d, splits_used);
+  if (workspace_bytes < l.total) return MLA_ERR_WORKSPACE;
+  const char* ws = static_cast<const char*>(workspace);
+  return cuda_status(launch_combine(seqlens, d->cache_capacity, d->B, d->H, d->d_c, splits_used,
+                                    reinterpret_cast<const float*>(ws + l.o_off),
+                                    reinterpret_cast<const float*>(ws + l.lse_off), o_lat, lse,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------------------
+int mla_out_proj(const mla_dims* d, const float* o_lat, const void* W_UV, void* out,
+                 void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if (!o_lat || !W_UV || !out) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_lat) || !aligned16(W_UV) || !aligned16(out)) return MLA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->dtype == MLA_BF16)
+    return cuda_status(launch_out_proj<__nv_bfloat16>(o_lat,
+                                                      static_cast<const __nv_bfloat16*>(W_UV),
+                                                      d->B, d->H, d->d_c, d->d_v,
+                                                      static_cast<__nv_bfloat16*>(out), s));
+  return cuda_status(launch_out_proj<float>(o_lat, static_cast<const float*>(W_UV), d->B, d->H,
+                                            d->d_c, d->d_v, static_cast<float*>(out), s));
+}
+
+}  // extern "C"

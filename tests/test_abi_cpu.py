@@ -1,0 +1,165 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+rejects bad arguments with the documented status before launching anything.
+No GPU is needed: validation runs first, and fake (never dereferenced)
+pointers are enough to exercise it."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_latent_kv_nope_b200 import binding as bd
+from mla_latent_kv_nope_b200 import build as bld
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, UNSUP, ALIGN, WS, CUDA = 0, 1, 2, 3, 4, 5
+
+
+@pytest.fixture(scope="module")
+def lib():
+    bld.build()
+    return bd.load_library()
+
+
+def _dims(**kw):
+    base = dict(B=4, H=16, d_c=512, d_r=64, d_nope=128, d_v=128, cache_capacity=4097,
+                dtype=bd.MLA_BF16)
+    base.update(kw)
+    return bd.CDims(**base)
+
+
+P = ctypes.c_void_p
+GOOD = P(0x10000)      # 16-byte aligned, never dereferenced
+GOOD2 = P(0x20000)
+BAD = P(0x10008)       # misaligned
+
+
+def test_header_symbols_all_exported(lib):
+    hdr = open(os.path.join(ROOT, "include", "mla.h")).read()
+    declared = set(re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", hdr))
+    assert declared == set(bd.EXPORTED)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(bd, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        bd.load_library(str(tmp_path / "nope.so"))
+
+
+def test_row_elems_and_status_strings(lib):
+    assert lib.mla_cache_row_elems(512, 64) == 576
+    assert lib.mla_cache_row_elems(32, 16) == 48
+    assert lib.mla_status_string(0) == b"ok"
+    assert lib.mla_status_string(4) == b"workspace missing or too small"
+    assert lib.mla_status_string(99) == b"unknown status"
+
+
+def test_workspace_layout_formula(lib):
+    for B, H, W in [(4, 16, 148), (32, 128, 74), (64, 64, 148), (1, 4, 3)]:
+        d = _dims(B=B, H=H)
+        slots = B + W - 1
+        r256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
+        expect = r256(slots * H * 512 * 4) + r256(slots * H * 4)
+        assert lib.mla_decode_workspace_bytes(ctypes.byref(d), W) == expect
+    d = _dims(B=64, d_c=512, d_r=64)
+    assert lib.mla_cache_append_workspace_bytes(ctypes.byref(d)) == 64 * 576 * 4
+    assert lib.mla_decode_workspace_bytes(ctypes.byref(d), 2000) == 0  # > 1024 splits
+
+
+def test_dims_validation(lib):
+    cases = [
+        (None, INVALID),
+        (_dims(B=0), INVALID), (_dims(H=-1), INVALID), (_dims(d_c=0), INVALID),
+        (_dims(cache_capacity=0), INVALID), (_dims(dtype=7), INVALID),
+        (_dims(d_c=500), UNSUP),                    # bf16 needs multiples of 8
+        (_dims(dtype=bd.MLA_F32, d_c=30), UNSUP),   # f32 needs multiples of 4
+        (_dims(dtype=bd.MLA_F32, d_c=2048), UNSUP),
+    ]
+    for d, want in cases:
+        ref = ctypes.byref(d) if d is not None else None
+        st = lib.mla_absorb_q(ref, GOOD, GOOD, GOOD, None, 10000.0, GOOD2, None)
+        assert st == want, (d and d.d_c, st, want)
+
+
+def test_decode_argument_errors(lib):
+    d = _dims()
+    ws_need = lib.mla_decode_workspace_bytes(ctypes.byref(d), 8)
+    used = ctypes.c_int(-1)
+    call = lambda dd, q=GOOD, c=GOOD, s=GOOD, scale=0.07, W=8, ws=GOOD2, wsb=ws_need: \
+        lib.mla_decode(ctypes.byref(dd), q, c, s, scale, W, ws, wsb, ctypes.byref(used), None)  # noqa: E731
+    assert call(_dims(d_c=256)) == UNSUP            # bf16 decode tile is 512 + 64
+    assert call(_dims(d_r=32)) == UNSUP
+    assert call(d, q=None) == INVALID
+    assert call(d, scale=0.0) == INVALID
+    assert call(d, scale=float("nan")) == INVALID
+    assert call(d, W=-1) == INVALID
+    assert call(d, W=5000) == INVALID
+    assert call(d, c=BAD) == ALIGN
+    assert call(d, ws=BAD) == ALIGN
+    assert call(d, wsb=ws_need - 1) == WS
+    assert call(d, ws=None) == WS
+    assert used.value == -1  # nothing reported before a successful launch
+
+
+def test_other_entry_point_errors(lib):
+    d = _dims()
+    # combine
+    need = lib.mla_decode_workspace_bytes(ctypes.byref(d), 8)
+    assert lib.mla_combine(ctypes.byref(d), GOOD, GOOD2, need, 0, GOOD, None, None) == INVALID
+    assert lib.mla_combine(ctypes.byref(d), GOOD, GOOD2, need - 4, 8, GOOD, None, None) == WS
+    assert lib.mla_combine(ctypes.byref(d), GOOD, BAD, need, 8, GOOD, None, None) == ALIGN
+    # out_proj
+    assert lib.mla_out_proj(ctypes.byref(d), None, GOOD, GOOD2, None) == INVALID
+    assert lib.mla_out_proj(ctypes.byref(d), GOOD, BAD, GOOD2, None) == ALIGN
+    # absorb_q
+    assert lib.mla_absorb_q(ctypes.byref(d), GOOD, None, GOOD, None, 1e4, GOOD2, None) == INVALID
+    assert lib.mla_absorb_q(ctypes.byref(d), GOOD, GOOD, GOOD, GOOD, -1.0, GOOD2, None) == INVALID
+    assert lib.mla_absorb_q(ctypes.byref(d), GOOD, GOOD, GOOD, BAD, 1e4, GOOD2, None) == ALIGN
+    # cache append
+    wsb = lib.mla_cache_append_workspace_bytes(ctypes.byref(d))
+    ap = lambda hidden=7168, h=GOOD, eps=1e-6, base=1e4, ws=GOOD2, n=wsb: lib.mla_cache_append(  # noqa: E731
+        ctypes.byref(d), hidden, h, GOOD, None, eps, base, GOOD, GOOD, ws, n, None)
+    assert ap(hidden=0) == INVALID
+    assert ap(h=None) == INVALID
+    assert ap(eps=-1.0) == INVALID
+    assert ap(base=0.0) == INVALID
+    assert ap(hidden=7161) == UNSUP
+    assert ap(h=BAD) == ALIGN
+    assert ap(n=wsb - 1) == WS
+    assert ap(ws=None) == WS
+
+
+def _deal(lens, W, tile=64):
+    """Host restatement of the documented split-KV dealing: worker w takes
+    tiles [w*T//W, (w+1)*T//W) of the concatenated per-sequence tiles."""
+    nt = [(L + tile - 1) // tile for L in lens]
+    T = sum(nt)
+    pre = [sum(nt[:b]) for b in range(len(lens))]
+    owner = {}
+    for w in range(W):
+        for t in range(w * T // W, (w + 1) * T // W):
+            owner[t] = w
+    pairs = set()
+    for b, (p, n) in enumerate(zip(pre, nt)):
+        for t in range(p, p + n):
+            pairs.add((owner[t], b))
+    return T, owner, pairs
+
+
+@pytest.mark.parametrize("lens,W", [([8192] * 32, 74), ([1, 2, 64, 65, 0, 300], 7),
+                                    ([5, 0, 0, 7], 16), ([131072] * 4, 148),
+                                    ([0, 0], 3)])
+def test_split_dealing_slots_unique(lens, W):
+    """Every tile has exactly one worker; the partial slots b + w of the
+    (worker, sequence) pairs are distinct and below B + W - 1; the owner of
+    tile t is ((t+1)*W - 1) // T, the closed form the kernels use."""
+    T, owner, pairs = _deal(lens, W)
+    assert len(owner) == T
+    slots = [b + w for (w, b) in pairs]
+    assert len(slots) == len(set(slots))
+    assert all(s < len(lens) + W - 1 for s in slots)
+    for t, w in owner.items():
+        assert ((t + 1) * W - 1) // T == w

@@ -1,0 +1,302 @@
+"""GPU parity: every entry point of the C ABI against the float64 CPU oracle on
+the same seeded inputs.  Tolerances (from the target statement): max over
+(sequence, head) of the relative L2 error <= 1e-2 for bf16 inputs with fp32
+accumulation and <= 1e-5 for the fp32 path; lse by absolute error with the
+same bounds; cache-append indexing bit-exact."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mla_latent_kv_nope_b200 as mla
+from mla_latent_kv_nope_b200 import inputs
+from oracle import mla_oracle as O
+
+from helpers import (dev, device_cache, dims_of, f64, host_cache, rel_l2, rounded, tol,
+                     torch_dtype)
+
+pytestmark = pytest.mark.gpu
+
+W = inputs.WORKLOADS
+SMALL_BF16 = W["v2lite_bf16"].scaled(B=3, N=200)
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _lib():
+    from mla_latent_kv_nope_b200 import build
+    build.build()
+    mla.load_library()
+    torch.cuda.set_device(0)
+
+
+def _lse_err(got, ref):
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isneginf(got), np.isneginf(ref))
+    return float(np.max(np.abs(got[fin] - ref[fin]))) if fin.any() else 0.0
+
+
+# ---------------------------------------------------------------------------
+# absorb_q
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [W["tiny_f32"], SMALL_BF16, W["v3_bf16"],
+                               W["ragged_append_bf16"].scaled(B=17)],
+                         ids=lambda w: f"{w.name}-B{w.B}-H{w.H}")
+def test_absorb_q(w):
+    qn, qp = inputs.query(w)
+    Wuk, _ = inputs.weights(w)
+    pos = np.arange(w.B, dtype=np.int32) * 977 + 5
+    d = dims_of(w)
+    q_cat = torch.empty(w.B, w.H, w.R, dtype=torch_dtype(w), device="cuda")
+    mla.absorb_q(d, dev(qn, w), dev(qp, w), dev(Wuk, w), torch.from_numpy(pos).cuda(), q_cat)
+    ref = O.absorb_q(rounded(qn, w), rounded(qp, w), rounded(Wuk, w), pos)
+    got = f64(q_cat)
+    assert rel_l2(got[..., :w.d_c], ref[..., :w.d_c]) < tol(w)
+    assert rel_l2(got[..., w.d_c:], ref[..., w.d_c:]) < tol(w)
+    # q_pos = NULL: the RoPE block is copied unchanged.
+    mla.absorb_q(d, dev(qn, w), dev(qp, w), dev(Wuk, w), None, q_cat)
+    np.testing.assert_array_equal(f64(q_cat)[..., w.d_c:], rounded(qp, w))
+
+
+# ---------------------------------------------------------------------------
+# out_proj
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [W["tiny_f32"], SMALL_BF16, W["v3_bf16"]],
+                         ids=lambda w: w.name)
+def test_out_proj(w):
+    _, Wuv = inputs.weights(w)
+    o_lat = inputs.normal((w.B, w.H, w.d_c), 0.05, 123, 1)
+    out = torch.empty(w.B, w.H, w.d_v, dtype=torch_dtype(w), device="cuda")
+    mla.out_proj(dims_of(w), dev(o_lat, w, torch.float32), dev(Wuv, w), out)
+    ref = O.out_proj(o_lat.astype(np.float64), rounded(Wuv, w))
+    assert rel_l2(f64(out), ref) < tol(w)
+
+
+# ---------------------------------------------------------------------------
+# cache append: values within tolerance, indexing bit-exact
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [W["tiny_f32"].scaled(B=3, hidden=64),
+                               W["ragged_append_bf16"].scaled(B=9, N=300),
+                               W["ragged_append_bf16"]],
+                         ids=lambda w: f"{w.name}-B{w.B}")
+def test_cache_append(w):
+    lens = inputs.seqlens(w) if w.ragged else np.array([0, 1, 63][:w.B] + [5] * max(0, w.B - 3),
+                                                       dtype=np.int32)
+    h, Wdkv = inputs.append_inputs(w)
+    gamma = 1.0 + inputs.normal((w.d_c,), 0.1, 77, 1)
+    d = dims_of(w)
+    dt = torch_dtype(w)
+    # Sentinel-filled cache: every element a fixed non-trivial pattern.
+    cache = torch.full((w.B, w.capacity, w.R), -3.25, dtype=dt, device="cuda")
+    before = cache.clone()
+    seq = torch.from_numpy(lens).cuda()
+    ws = torch.empty(mla.cache_append_workspace_bytes(d) // 4, dtype=torch.float32,
+                     device="cuda")
+    mla.cache_append(d, dev(h, w), dev(Wdkv, w), torch.from_numpy(gamma).cuda(), cache, seq, ws,
+                     eps=w.eps)
+    assert mla.get_device_status() == 0
+    np.testing.assert_array_equal(seq.cpu().numpy(), lens + 1)
+    # Bit-exact: only row L_b of each sequence changed.
+    mask = torch.zeros(w.B, w.capacity, dtype=torch.bool, device="cuda")
+    mask[torch.arange(w.B), torch.from_numpy(lens).long().cuda()] = True
+    raw = lambda t: t.view(torch.int16) if dt == torch.bfloat16 else t.view(torch.int32)  # noqa
+    assert torch.equal(raw(cache)[~mask], raw(before)[~mask])
+    rows_got = f64(cache[torch.arange(w.B), torch.from_numpy(lens).long().cuda()])
+    zero = np.zeros((w.B, w.capacity, w.R))
+    _, _, rows_ref = O.cache_append(zero, lens, rounded(h, w), rounded(Wdkv, w), w.d_c,
+                                    gamma=gamma.astype(np.float64), eps=w.eps)
+    assert rel_l2(rows_got[:, :w.d_c], rows_ref[:, :w.d_c]) < tol(w)
+    assert rel_l2(rows_got[:, w.d_c:], rows_ref[:, w.d_c:]) < tol(w)
+
+
+def test_cache_append_capacity_is_reported():
+    w = W["ragged_append_bf16"].scaled(B=3, N=10, hidden=64)
+    d = dims_of(w, capacity=10)
+    lens = np.array([3, 10, 9], dtype=np.int32)  # sequence 1 is full
+    h, Wdkv = inputs.append_inputs(w)
+    cache = torch.zeros(w.B, 10, w.R, dtype=torch.bfloat16, device="cuda")
+    seq = torch.from_numpy(lens).cuda()
+    ws = torch.empty(mla.cache_append_workspace_bytes(d) // 4, dtype=torch.float32, device="cuda")
+    mla.get_device_status()
+    mla.cache_append(d, dev(h, w), dev(Wdkv, w), None, cache, seq, ws)
+    assert mla.get_device_status() == 7  # MLA_ERR_BOUNDS
+    assert mla.get_device_status() == 0  # cleared by the read
+    np.testing.assert_array_equal(seq.cpu().numpy(), [4, 10, 10])
+    assert torch.count_nonzero(cache[1]) == 0
+    assert torch.count_nonzero(cache[0, 3]) > 0 and torch.count_nonzero(cache[2, 9]) > 0
+
+
+# ---------------------------------------------------------------------------
+# decode + combine against the latent-attention definition
+# ---------------------------------------------------------------------------
+def _run_decode(w, lens, q_cat_np, scale, num_splits=0, capacity=None, fill_rest=float("nan")):
+    cap = capacity if capacity is not None else max(int(lens.max()), 1)
+    d = dims_of(w, capacity=cap)
+    cache = device_cache(w, lens, capacity=cap, fill_rest=fill_rest)
+    seq = torch.from_numpy(lens.astype(np.int32)).cuda()
+    W_ = num_splits or mla.decode_default_splits(d)
+    ws = torch.empty(mla.decode_workspace_bytes(d, W_) // 4, dtype=torch.float32, device="cuda")
+    ws.fill_(float("nan"))  # nothing may depend on unwritten workspace
+    used = mla.decode(d, dev(q_cat_np, w), cache, seq, scale, ws, W_)
+    assert used == W_
+    o_lat = torch.empty(w.B, w.H, w.d_c, dtype=torch.float32, device="cuda")
+    lse = torch.empty(w.B, w.H, dtype=torch.float32, device="cuda")
+    mla.combine(d, seq, ws, used, o_lat, lse)
+    assert mla.get_device_status() == 0
+    return f64(o_lat), f64(lse)
+
+
+def _oracle_latent(w, lens, q_cat_np, scale):
+    rows = host_cache(w, lens)
+    cap = max(int(lens.max()), 1)
+    cache = np.zeros((w.B, cap, w.R))
+    for b, r in rows.items():
+        cache[b, :len(r)] = r
+    return O.latent_attention(rounded(q_cat_np, w), cache, lens, scale, w.d_c)
+
+
+DECODE_CASES = [
+    ("tiny_f32", W["tiny_f32"], [64], 0, 1.0),
+    ("tiny_f32-ragged", W["tiny_f32"].scaled(B=5), [64, 1, 0, 130, 65], 3, 1.0),
+    ("bf16-H16-edges", SMALL_BF16.scaled(B=8), [1, 63, 64, 65, 127, 128, 200, 0], 0, 1.0),
+    ("bf16-H16-W1", SMALL_BF16.scaled(B=4), [200, 5, 64, 1], 1, 1.0),
+    ("bf16-H16-Wbig", SMALL_BF16.scaled(B=4), [200, 5, 64, 1], 1000, 1.0),
+    ("bf16-H64", W["ragged_append_bf16"].scaled(B=5, N=700), [700, 1, 333, 64, 0], 0, 1.0),
+    ("bf16-H128", W["v3_bf16"].scaled(B=3, N=600), [600, 129, 1], 0, 1.0),
+    ("bf16-H128-W7", W["v3_bf16"].scaled(B=3, N=600), [600, 129, 1], 7, 1.0),
+    ("bf16-H128-peaked", W["v3_bf16"].scaled(B=2, N=400), [400, 77], 0, 10.0),
+    ("bf16-H16-peaked", SMALL_BF16.scaled(B=2), [190, 64], 0, 10.0),
+]
+
+
+@pytest.mark.parametrize("name,w,lens,nsplit,boost", DECODE_CASES, ids=[c[0] for c in DECODE_CASES])
+def test_decode_combine(name, w, lens, nsplit, boost):
+    lens = np.array(lens, dtype=np.int32)
+    q_cat = inputs.normal((w.B, w.H, w.R), 0.5, 31, len(lens))
+    scale = w.softmax_scale * boost
+    got_o, got_l = _run_decode(w, lens, q_cat, scale, nsplit)
+    ref_o, ref_l = _oracle_latent(w, lens, q_cat, scale)
+    nz = lens > 0
+    assert rel_l2(got_o[nz], ref_o[nz]) < tol(w)
+    assert np.all(got_o[~nz] == 0)
+    assert _lse_err(got_l, ref_l) < tol(w)
+
+
+def test_combine_alone():
+    """Synthetic partials placed in the documented workspace slots; the merge
+    must equal the log-sum-exp combination of exactly those partials."""
+    B, H, d_c, Wn = 5, 16, 512, 6
+    lens = np.array([300, 0, 64, 1000, 1], dtype=np.int32)
+    w = SMALL_BF16.scaled(B=B)
+    d = dims_of(w, capacity=1000)
+    nt = [(L + 63) // 64 for L in lens]
+    T = sum(nt)
+    pre = np.concatenate([[0], np.cumsum(nt)])
+    slots = B + Wn - 1
+    o_all, l_all = inputs.partials(1, H, slots, d_c, seed=3, empty_frac=0.0)
+    ws = torch.full((mla.decode_workspace_bytes(d, Wn) // 4,), float("nan"), device="cuda")
+    ws[:slots * H * d_c] = torch.from_numpy(o_all[0].transpose(1, 0, 2).reshape(-1)).cuda()
+    lse_off = ((slots * H * d_c * 4 + 255) // 256 * 256) // 4
+    ws[lse_off:lse_off + slots * H] = torch.from_numpy(l_all[0].T.reshape(-1)).cuda()
+    o_lat = torch.empty(B, H, d_c, device="cuda")
+    lse = torch.empty(B, H, device="cuda")
+    mla.combine(d, torch.from_numpy(lens).cuda(), ws, Wn, o_lat, lse)
+    torch.cuda.synchronize()
+    for b in range(B):
+        if nt[b] == 0:
+            assert torch.all(o_lat[b] == 0) and torch.all(torch.isneginf(lse[b]))
+            continue
+        ws_ = sorted({w_ for t in range(pre[b], pre[b + 1]) for w_ in range(Wn)
+                      if w_ * T // Wn <= t < (w_ + 1) * T // Wn})
+        sl = [b + w_ for w_ in ws_]
+        ref_o, ref_l = O.combine_partials(o_all[0][:, sl].astype(np.float64),
+                                          l_all[0][:, sl].astype(np.float64))
+        assert rel_l2(f64(o_lat[b]), ref_o) < 1e-5
+        assert np.max(np.abs(f64(lse[b]) - ref_l)) < 1e-5
+
+
+# ---------------------------------------------------------------------------
+# Whole step (append, absorb, decode, combine, out_proj) against the
+# materialised-MHA oracle.
+# ---------------------------------------------------------------------------
+def _full_step(w, sample_pairs=None, num_splits=0):
+    lens = inputs.seqlens(w)
+    d = dims_of(w)
+    cache = device_cache(w, lens)
+    seq = torch.from_numpy(lens).cuda()
+    qn, qp = inputs.query(w)
+    Wuk, Wuv = inputs.weights(w)
+    step_kw = {}
+    h = Wdkv = None
+    if w.append:
+        h, Wdkv = inputs.append_inputs(w)
+        step_kw["h"] = dev(h, w)
+        q_pos = lens.copy()              # the new token's position
+    else:
+        q_pos = lens - 1                 # the query is the newest cached token
+    step = mla.DecodeStep(d, dev(Wuk, w), dev(Wuv, w), dev(Wdkv, w) if w.append else None,
+                          num_splits=num_splits)
+    out = step(dev(qn, w), dev(qp, w), torch.from_numpy(q_pos.astype(np.int32)).cuda(), cache,
+               seq, **step_kw)
+    torch.cuda.synchronize()
+    assert mla.get_device_status() == 0
+    got, got_lat, got_lse = f64(out), f64(step.o_lat), f64(step.lse)
+
+    if sample_pairs is None:
+        sample_pairs = [(b, i) for b in range(w.B) for i in range(w.H)]
+    seqs = sorted({b for b, _ in sample_pairs})
+    rows = host_cache(w, lens, seqs)
+    rq_n, rq_p, rWuk, rWuv = (rounded(a, w) for a in (qn, qp, Wuk, Wuv))
+    worst = worst_lat = worst_lse = 0.0
+    for b in seqs:
+        L = int(lens[b])
+        cache_b = np.zeros((1, L + 1, w.R))
+        cache_b[0, :L] = rows[b]
+        Lb = np.array([L])
+        if w.append:
+            cache_b, Lb, _ = O.cache_append(cache_b, Lb, rounded(h, w)[b:b + 1],
+                                            rounded(Wdkv, w), w.d_c, eps=w.eps)
+        heads = [i for bb, i in sample_pairs if bb == b]
+        o, ol, ls = O.mla_decode_materialised(
+            rq_n[b:b + 1, heads], rq_p[b:b + 1, heads], q_pos[b:b + 1], rWuk[heads],
+            rWuv[heads], cache_b, Lb, w.softmax_scale)
+        worst = max(worst, rel_l2(got[b, heads], o[0]))
+        worst_lat = max(worst_lat, rel_l2(got_lat[b, heads], ol[0]))
+        worst_lse = max(worst_lse, float(np.max(np.abs(got_lse[b, heads] - ls[0]))))
+    if w.append:
+        np.testing.assert_array_equal(seq.cpu().numpy(), lens + 1)
+    return worst, worst_lat, worst_lse
+
+
+SMALL_STEPS = [
+    W["tiny_f32"],
+    W["v2lite_bf16"].scaled(B=2, N=300),
+    W["v3_bf16"].scaled(B=2, N=260),
+    W["ragged_append_bf16"].scaled(B=6, N=500, hidden=512),
+]
+
+
+@pytest.mark.parametrize("w", SMALL_STEPS, ids=lambda w: f"{w.name}-small")
+def test_full_step_small(w):
+    e, el, els = _full_step(w)
+    assert e < tol(w) and el < tol(w) and els < tol(w), (e, el, els)
+
+
+def _sample(w, n_seq, heads, seed=0):
+    r = np.random.default_rng(seed)
+    seqs = sorted(set([0, w.B - 1] + list(r.choice(w.B, size=min(n_seq, w.B), replace=False))))
+    return [(int(b), int(i)) for b in seqs for i in heads]
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "v2lite_bf16", "v3_bf16", "longctx_bf16",
+                                  "ragged_append_bf16"])
+def test_full_step_full_size(name):
+    """Each configuration at its full size in the launch configuration the
+    bench times (default splits), checked on sampled (sequence, head) pairs
+    that the oracle recomputes from scratch."""
+    w = W[name]
+    heads = sorted({0, w.H - 1, w.H // 2, 1 % w.H})
+    n_seq = {"tiny_f32": 1, "v2lite_bf16": 4, "v3_bf16": 6, "longctx_bf16": 2,
+             "ragged_append_bf16": 6}[name]
+    e, el, els = _full_step(w, _sample(w, n_seq, heads))
+    assert e < tol(w) and el < tol(w) and els < tol(w), (e, el, els)
