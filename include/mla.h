@@ -156,6 +156,31 @@ MLA_API int mla_combine(const mla_dims* dims, const int32_t* seqlens,
 MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W_UV,
                  void* out, void* stream);
 
+/* --- 3+4 without a workspace -------------------------------------------------
+ * No counterpart on the pages: this is a convenience of this library.
+ * For callers that cannot allocate device memory (code running while a stream
+ * is captured into a CUDA graph, where cudaMalloc is not allowed; plugins that
+ * only receive fixed buffers from a host framework), this runs mla_decode and
+ * mla_combine with the split-KV partials kept in a fixed array inside the
+ * library instead of a caller workspace.  Inputs and outputs are as for
+ * mla_decode + mla_combine (q_cat, cache, seqlens in; o_lat [B,H,d_c] fp32 and
+ * lse [B,H] fp32 (may be NULL) out); nothing is allocated or freed.
+ *   - The array holds MLA_DECODE_NOALLOC_SCRATCH_BYTES on every device that
+ *     loads the library, until the process exits.  The split count is the
+ *     device default, lowered until the partials, (B + W - 1) * H * (d_c + 1)
+ *     floats, fit; if even one split does not fit (B * H * (d_c + 1) * 4 bytes
+ *     above the limit) the call returns MLA_ERR_WORKSPACE and launches nothing.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents (every partial read in a call is written earlier in the same
+ *     call).  Calls that overlap on the GPU (different streams, or several
+ *     host threads) race on it: serialise them. */
+#define MLA_DECODE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+MLA_API int mla_decode_noalloc(const mla_dims* dims, const void* q_cat, const void* cache,
+                               const int32_t* seqlens, float softmax_scale, float* o_lat,
+                               float* lse, void* stream);
+
 /* --- status ------------------------------------------------------------------
  * Synchronises `stream`, then returns and clears the current device's status
  * word (MLA_OK if no device-side error was recorded since the last call).

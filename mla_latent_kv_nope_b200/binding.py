@@ -26,7 +26,7 @@ EXPORTED = (
     "mla_cache_row_elems", "mla_cache_append_workspace_bytes", "mla_cache_append",
     "mla_absorb_q", "mla_decode_default_splits", "mla_decode_workspace_bytes",
     "mla_decode", "mla_combine", "mla_out_proj", "mla_get_device_status",
-    "mla_status_string",
+    "mla_status_string", "mla_decode_noalloc",
 )
 
 
@@ -96,6 +96,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_combine": (ctypes.c_int, [D, P, P, SZ, ctypes.c_int, P, P, P]),
         "mla_out_proj": (ctypes.c_int, [D, P, P, P, P]),
         "mla_get_device_status": (ctypes.c_int, [P]),
+        "mla_decode_noalloc": (ctypes.c_int, [D, P, P, P, F, P, P, P]),
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():

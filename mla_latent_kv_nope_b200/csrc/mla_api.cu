@@ -263,3 +263,74 @@ int mla_out_proj(const mla_dims* d, const float* o_lat, const void* W_UV, void* 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode + combine for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at all: code running while a stream is
+// being captured into a CUDA graph (allocation is illegal there), plugins
+// handed a fixed set of buffers by a host framework, or runtimes whose memory
+// is owned by another allocator.  For them the split-KV partials live in the
+// file-scope array below instead of a caller-provided workspace.  It is sized
+// once (MLA_DECODE_NOALLOC_SCRATCH_BYTES) and every device that loads this
+// library holds it until the process exits.
+namespace mla {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+// In host code `g_noalloc_scratch` names a host-side stand-in, not device
+// memory, so the kernels get the real device address, looked up once per
+// device (with that device current) and cached.
+void* noalloc_scratch_ptr() {
+  static void* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    cache[dev] = p;
+  }
+  return cache[dev];
+}
+
+}  // namespace
+}  // namespace mla
+
+extern "C" int mla_decode_noalloc(const mla_dims* d, const void* q_cat, const void* cache,
+                                  const int32_t* seqlens, float softmax_scale, float* o_lat,
+                                  float* lse, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if ((st = decode_shape_supported(d))) return st;
+  if (!q_cat || !cache || !seqlens || !o_lat || !(softmax_scale > 0.f) ||
+      softmax_scale == INFINITY)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_cat) || !aligned16(cache) || !aligned16(seqlens) || !aligned16(o_lat) ||
+      (lse && !aligned16(lse)))
+    return MLA_ERR_ALIGNMENT;
+  // Largest split count (up to the default) whose partials fit the array.
+  int W = mla_decode_default_splits(d);
+  if (W <= 0) return MLA_ERR_CUDA;
+  while (W >= 1 && ws_layout(d, W).total > size_t(MLA_DECODE_NOALLOC_SCRATCH_BYTES)) --W;
+  if (W < 1) return MLA_ERR_WORKSPACE;  // B * H too large for the fixed scratch
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return MLA_ERR_CUDA;
+  const WsLayout l = ws_layout(d, W);
+  float* o_part = reinterpret_cast<float*>(static_cast<char*>(scratch) + l.o_off);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(scratch) + l.lse_off);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d->dtype == MLA_BF16)
+    e = launch_decode_tc(static_cast<const __nv_bfloat16*>(q_cat),
+                         static_cast<const __nv_bfloat16*>(cache), seqlens, d->B, d->H,
+                         d->cache_capacity, softmax_scale, W, o_part, lse_part, status_ptr(), s);
+  else
+    e = launch_decode_simt<float>(static_cast<const float*>(q_cat),
+                                  static_cast<const float*>(cache), seqlens, d->B, d->H, d->d_c,
+                                  d->d_r, d->cache_capacity, softmax_scale, W, o_part, lse_part,
+                                  status_ptr(), s);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  return cuda_status(launch_combine(seqlens, d->cache_capacity, d->B, d->H, d->d_c, W, o_part,
+                                    lse_part, o_lat, lse, s));
+}
