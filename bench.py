@@ -21,7 +21,6 @@ import hashlib
 import json
 import math
 import os
-import subprocess
 import sys
 import time
 
@@ -67,57 +66,82 @@ def _ncu_traffic(workload):
     return None
 
 
+_SAMPLER_SRC = r"""
+import sys, time, pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[1]))
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    t = time.time()
+    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+    print(f"{t:.4f} {sm} {rs}", flush=True)
+    time.sleep(0.005)
+"""
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled through NVML every ~5 ms by a
+    separate process; only samples inside the [start, stop] window of the
+    timed steps are kept."""
+    REASONS = {  # NVML clocks-event-reason bits
+        0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+        0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown",
+    }
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
+        self.t_start = self.t_stop = None
 
     def __enter__(self):
+        import subprocess
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_SRC, str(self.index)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            first = self.proc.stdout.readline().split()
+            self.max_mhz = int(first[1]) if first and first[0] == "max" else None
         except Exception:
             self.proc = None
         return self
 
+    def start(self):
+        self.t_start = time.time()
+
+    def stop(self):
+        self.t_stop = time.time()
+
     def __exit__(self, *a):
-        self.out = ""
+        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                out, _ = self.proc.communicate(timeout=5)
+                self.lines = out.splitlines()
             except Exception:
                 self.proc.kill()
 
     def summary(self):
         rows = []
-        for line in (getattr(self, "out", "") or "").splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+        for ln in getattr(self, "lines", []):
+            f = ln.split()
+            if len(f) != 3:
                 continue
-            try:
-                rows.append(dict(sm=float(f[1]), smax=float(f[2]), hw=f[5], hwt=f[6], swt=f[7],
-                                 pcap=f[8]))
-            except ValueError:
+            t, sm, rs = float(f[0]), int(f[1]), int(f[2])
+            if self.t_start is not None and not (self.t_start <= t <= self.t_stop):
                 continue
+            rows.append((sm, rs))
         if not rows:
             return None
-        sms = sorted(r["sm"] for r in rows)
+        sms = sorted(r[0] for r in rows)
         reasons = set()
-        for r in rows:
-            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
-                            ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
-                if r[k].lower() == "active":
+        for _, rs in rows:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
                     reasons.add(name)
-        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": rows[0]["smax"],
-                "samples": len(rows), "reasons": sorted(reasons)}
+        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": self.max_mhz,
+                "sm_min_mhz": sms[0], "samples": len(rows), "reasons": sorted(reasons),
+                "source": "NVML from a separate process, ~5 ms period, timed window only"}
 
 
 # ---------------------------------------------------------------------------
@@ -167,22 +191,14 @@ def run_ours(args, rank, world, local_rank):
     if cache_bytes < 2 * L2_BYTES:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
-    ev_dec = []
-
-    def one_step(record=False):
+    def one_step():
         if flush is not None:
             flush.zero_()
         step.append(hh, cache, seq)
         mla.absorb_q(dims, q_nope, q_pe, W_UK, q_pos, step.q_cat, step.rope_base)
-        if record:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
         step.splits_used = mla.decode(dims, step.q_cat, cache, seq, step.scale, step.ws,
                                       step.num_splits)
         mla.combine(dims, seq, step.ws, step.splits_used, step.o_lat, step.lse)
-        if record:
-            e1.record(stream)
-            ev_dec.append((e0, e1))
         mla.out_proj(dims, step.o_lat, W_UV, step.out)
         seq.copy_(seq0)
 
@@ -221,6 +237,7 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         barrier()
         torch.cuda.synchronize()
+        clk.start()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -228,6 +245,7 @@ def run_ours(args, rank, world, local_rank):
             one_step()
         t1.record(stream)
         torch.cuda.synchronize()
+        clk.stop()
         barrier()
         ms_total = t0.elapsed_time(t1)
         dec_ms, decomb_ms = decode_only(max(args.steps, 5))

@@ -12,22 +12,26 @@
 // Structure (one CTA = 64 heads of one work range; CTAs of the same range for
 // the other head groups are launched next to it so the tile is read from HBM
 // once and from L2 after that):
-//   warp 4      TMA producer: per tile, 9 boxes of [64 keys x 64 dims] bf16
-//               with 128-byte swizzle into a 2-stage ring; the 64-head query
-//               block is loaded the same way once per sequence.
-//   warp 5      MMA issuer: tcgen05.mma kind::f16 (bf16 in, fp32 in TMEM).
-//               QK^T of tile i+1 is issued while the softmax of tile i runs.
-//   warps 0-3   softmax + correction + epilogue, reading S from TMEM
-//               (tcgen05.ld), writing P as bf16 into the tile's dead RoPE
-//               chunk (the swizzled K-major A operand of P.C), rescaling the
-//               TMEM accumulator only when the running max grows by more
-//               than 2^8, and storing the partial (o, lse).
-// TMEM (M = 64 tiles occupy lanes 0-15 of each 32-lane quadrant, or lanes
-// 16-31 with a lane offset of 16):
-//   lanes +0 : cols [0,256)  O[:, 0:256]      cols [256,384) S double buffer
-//   lanes +16: cols [0,256)  O[:, 256:512]
+//   warp 4      TMA producer: per 64-key tile, 9 boxes of [64 keys x 64 dims]
+//               bf16 with 128-byte swizzle into a 3-stage ring, plus an L2
+//               prefetch a few tiles ahead.
+//   warp 5      MMA issuer (one thread): S = Q C^T with Q read from tensor
+//               memory (only the cache tile is fetched from shared memory),
+//               O += P C with P and C from shared memory.  QK^T of tile i+1 is
+//               issued while the softmax of tile i runs.
+//   warps 0-3   softmax, correction and epilogue.  At each sequence start
+//               they write the 64 x 576 query block into tensor memory.
+// Tensor memory (an M = 64 tile occupies 16 of the 32 lanes of each
+// quadrant; "lo" = lanes 0-15, "hi" = lanes 16-31):
+//   lo lanes: cols [0,64) and [64,128) S double buffer; cols [128,416) Q
+//             (576 bf16 packed in pairs)
+//   hi lanes: cols [0,256) O[:, 0:256]; cols [256,512) O[:, 256:512]
+// All tensor-memory traffic of the softmax warps uses 16-lane accesses, so
+// each row is shared by two threads (keys 0-31 / 32-63 of S; columns
+// 0-255 / 256-511 of O) and the other lane half is never touched.
 // Every wait is bounded (2 s); on give-up the CTA raises a shared abort flag,
-// records MLA_ERR_DEVICE_TIMEOUT, drains its own loads, frees TMEM and exits.
+// records MLA_ERR_DEVICE_TIMEOUT, drains its own loads and MMAs, frees TMEM
+// and exits.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -48,20 +52,23 @@ constexpr int kChunks = kR / kChunkElems;             // 9 (8 latent + 1 RoPE)
 constexpr int kRopeChunk = 8;
 constexpr int kChunkBytes = kTileKeys * 128;          // 8192
 constexpr int kStageBytes = kChunks * kChunkBytes;    // 73728
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 32 * (kSoftmaxWarps + 2);    // 192
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 256;
+constexpr uint32_t kColS = 0;                         // lo lanes, 2 x 64 columns
+constexpr uint32_t kColQ = 128;                       // lo lanes, 288 columns
+constexpr uint32_t kHiLanes = 16u << 16;              // lane offset of the hi half
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.f;  // log2 units: rescale when the max grows by > 2^8
+constexpr int kPrefetchTiles = 4;         // tiles brought into L2 ahead of their load
 
 struct Barriers {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t q_full, q_empty;
+  uint64_t q_ready;
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2];
   uint64_t o_free;
@@ -70,9 +77,8 @@ struct Barriers {
   int abort_flag;
 };
 
-constexpr size_t kOffQ = 0;
-constexpr size_t kOffStage = kStageBytes;
-constexpr size_t kOffBar = kOffStage + size_t(kStages) * kStageBytes;
+constexpr size_t kOffStage = 0;
+constexpr size_t kOffBar = size_t(kStages) * kStageBytes;
 constexpr size_t kSmemBytes = kOffBar + sizeof(Barriers) + 1024;  // + alignment slack
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
@@ -116,14 +122,13 @@ __device__ __forceinline__ void for_each_segment(const int32_t* seqlens, int B, 
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* __restrict__ q_cat,
                  const int32_t* __restrict__ seqlens, int B, int H, int64_t cap,
                  float scale_log2, int W, float* __restrict__ o_part,
                  float* __restrict__ lse_part, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + kOffQ;
   uint8_t* sStage = smem + kOffStage;
   Barriers* bars = reinterpret_cast<Barriers*>(smem + kOffBar);
 
@@ -143,8 +148,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->q_ready, 32 * kSoftmaxWarps);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
       mbar_init(&bars->s_free[s], 32 * kSoftmaxWarps);
@@ -160,10 +164,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_c);
-  }
+  if (warp == kProducerWarp && lane == 0) tma_prefetch_desc(&tm_c);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -174,24 +175,26 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t i = 0;
-      int seg = 0;
       bool ok = true;
       for_each_segment(seqlens, B, cap, t_begin, t_end,
                        [&](int b, int64_t lo, int64_t hi, int64_t) {
-        if (seg > 0 && !(ok = mbar_wait(&bars->q_empty, (seg - 1) & 1, abort_flag, kWaitLimitNs)))
-          return false;
-        ++seg;
-        mbar_arrive_expect_tx(&bars->q_full, kStageBytes);
-        const int32_t qrow = b * H + g * kHeadsPerCta;
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_2d(&tm_q, &bars->q_full, sQ + c * kChunkBytes, c * kChunkElems, qrow);
+        // One CTA per tile range (head group 0) pulls tiles into L2 a few
+        // tiles ahead; the shared-memory loads of every head group hit L2.
+        const int64_t row0 = int64_t(b) * cap;
+        auto prefetch = [&](int64_t t) {
+          for (int c = 0; c < kChunks; ++c)
+            tma_prefetch_2d(&tm_c, c * kChunkElems, int32_t(row0 + t * kTileKeys));
+        };
+        if (g == 0)
+          for (int64_t t = lo; t < min(lo + kPrefetchTiles, hi); ++t) prefetch(t);
         for (int64_t t = lo; t < hi; ++t, ++i) {
-          const int s = i & 1;
-          if (i >= 2 && !(ok = mbar_wait(&bars->empty[s], ((i >> 1) - 1) & 1, abort_flag,
-                                         kWaitLimitNs)))
+          const int s = i % kStages;
+          if (g == 0 && t + kPrefetchTiles < hi) prefetch(t + kPrefetchTiles);
+          if (i >= kStages && !(ok = mbar_wait(&bars->empty[s], ((i / kStages) - 1) & 1,
+                                               abort_flag, kWaitLimitNs)))
             return false;
           mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
-          const int32_t crow = int32_t(int64_t(b) * cap + t * kTileKeys);
+          const int32_t crow = int32_t(row0 + t * kTileKeys);
           uint8_t* dst = sStage + s * kStageBytes;
           for (int c = 0; c < kChunks; ++c)
             tma_load_2d(&tm_c, &bars->full[s], dst + c * kChunkBytes, c * kChunkElems, crow);
@@ -201,128 +204,173 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!ok) {
         raise_abort(bars, status);
         // Drain this CTA's own loads before it may exit: the last load into
-        // each stage and the last query block (bounded, ignoring the flag).
+        // each stage (bounded, ignoring the flag).
         volatile int no_abort = 0;
-        for (uint32_t k = (i > 2 ? i - 2 : 0); k < i; ++k)
-          mbar_wait(&bars->full[k & 1], (k >> 1) & 1, &no_abort, kWaitLimitNs);
-        if (seg > 0) mbar_wait(&bars->q_full, (seg - 1) & 1, &no_abort, kWaitLimitNs);
+        for (uint32_t k = (i > kStages ? i - kStages : 0); k < i; ++k)
+          mbar_wait(&bars->full[k % kStages], (k / kStages) & 1, &no_abort, kWaitLimitNs);
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t i_qk = 0, i_pv = 0;
-      int seg = 0;
-      bool ok = true;
-      const uint32_t q_base = smem_u32(sQ);
-      const uint32_t st_base = smem_u32(sStage);
-      for_each_segment(seqlens, B, cap, t_begin, t_end,
-                       [&](int, int64_t lo, int64_t hi, int64_t) {
-        const uint32_t base = i_pv, end = i_pv + uint32_t(hi - lo);
-        if (!(ok = mbar_wait(&bars->q_full, seg & 1, abort_flag, kWaitLimitNs))) return false;
-        tc_fence_after();
-        uint64_t t_last = global_timer_ns();
-        uint32_t spins = 0;
-        while (i_pv < end) {
-          bool progressed = false;
-          if (i_qk < end && i_qk <= i_pv + 1) {
-            const int s = i_qk & 1;
-            if (mbar_test(&bars->full[s], (i_qk >> 1) & 1) &&
-                (i_qk < 2 || mbar_test(&bars->s_free[s], ((i_qk >> 1) - 1) & 1))) {
-              tc_fence_after();
-              const uint32_t d = tmem + kColS + uint32_t(s) * 64u;
-              const uint32_t stage = st_base + uint32_t(s) * kStageBytes;
-#pragma unroll 1
-              for (int c = 0; c < kChunks; ++c) {
+    // The whole warp runs the scheduler (decisions are lane 0's, broadcast)
+    // and elect.sync issues each instruction from one lane.
+    uint32_t i_qk = 0, i_pv = 0;
+    int seg = 0;
+    bool ok = true;
+    const uint32_t st_base = smem_u32(sStage);
+    for_each_segment(seqlens, B, cap, t_begin, t_end,
+                     [&](int, int64_t lo, int64_t hi, int64_t) {
+      const uint32_t base = i_pv, end = i_pv + uint32_t(hi - lo);
+      // The softmax warps have written this sequence's query block.
+      if (!(ok = warp_wait(&bars->q_ready, seg & 1, abort_flag))) return false;
+      tc_fence_after();
+      uint64_t t_last = global_timer_ns();
+      uint32_t spins = 0;
+      while (i_pv < end) {
+        bool progressed = false;
+        if (i_qk < end && i_qk <= i_pv + 1) {
+          const int st = i_qk % kStages, sb = i_qk & 1;
+          int ready = 0;
+          if (lane == 0)
+            ready = mbar_test(&bars->full[st], (i_qk / kStages) & 1) &&
+                    (i_qk < 2 || mbar_test(&bars->s_free[sb], ((i_qk >> 1) - 1) & 1));
+          if (__shfl_sync(0xffffffffu, ready, 0)) {
+            tc_fence_after();
+            const uint32_t d = tmem + kColS + uint32_t(sb) * 64u;
+            // Descriptor and TMEM address bases are formed once; each of the
+            // 36 MMAs then only adds a compile-time offset (the start address
+            // field is the low 14 bits: shared-memory offsets >> 4).
+            const uint64_t b0 = smem_desc_sw128(st_base + uint32_t(st) * kStageBytes, 16, 1024);
+            const uint32_t a0 = tmem + kColQ;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const uint64_t a = smem_desc_sw128(q_base + c * kChunkBytes + k * 32, 16, 1024);
-                  const uint64_t bdesc =
-                      smem_desc_sw128(stage + c * kChunkBytes + k * 32, 16, 1024);
-                  mma_bf16_ss(d, a, bdesc, kIdescQK, (c | k) != 0);
-                }
-              }
-              mma_commit(&bars->s_full[s]);
-              ++i_qk;
-              if (i_qk == end) mma_commit(&bars->q_empty);
-              progressed = true;
-            }
-          }
-          if (!progressed && i_pv < i_qk) {
-            const int s = i_pv & 1;
-            const bool first = (i_pv == base);
-            if (mbar_test(&bars->p_full[s], (i_pv >> 1) & 1) &&
-                (!first || seg == 0 || mbar_test(&bars->o_free, (seg - 1) & 1))) {
-              tc_fence_after();
-              const uint32_t stage = st_base + uint32_t(s) * kStageBytes;
+            for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const uint32_t d = tmem + (h ? (16u << 16) : 0u);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const uint64_t a =
-                      smem_desc_sw128(stage + kRopeChunk * kChunkBytes + k * 32, 16, 1024);
-                  const uint64_t bdesc = smem_desc_sw128(
-                      stage + (4 * h) * kChunkBytes + k * 2048, kChunkBytes, 1024);
-                  mma_bf16_ss(d, a, bdesc, kIdescPV, !(first && k == 0));
-                }
-              }
-              mma_commit(&bars->empty[s]);
-              ++i_pv;
-              progressed = true;
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ts_w(d, a0 + uint32_t(c * 4 + k) * 8u,
+                              b0 + uint64_t((c * kChunkBytes + k * 32) >> 4), kIdescQK,
+                              (c | k) != 0);
             }
-          }
-          if (progressed) {
-            spins = 0;
-            t_last = global_timer_ns();
-          } else if ((++spins & 255) == 0) {
-            if (*abort_flag || global_timer_ns() - t_last > kWaitLimitNs) {
-              ok = false;
-              return false;
-            }
+            mma_commit_w(&bars->s_full[sb]);
+            ++i_qk;
+            progressed = true;
           }
         }
-        ++seg;
-        return true;
-      });
-      if (!ok) raise_abort(bars, status);
-      // Every MMA issued by this thread has completed before TMEM is freed.
-      mma_commit(&bars->mma_drain);
-      volatile int no_abort = 0;
-      mbar_wait(&bars->mma_drain, 0, &no_abort, kWaitLimitNs);
-    }
+        if (!progressed && i_pv < i_qk) {
+          const int st = i_pv % kStages, sb = i_pv & 1;
+          const bool first = (i_pv == base);
+          int ready = 0;
+          if (lane == 0)
+            ready = mbar_test(&bars->p_full[sb], (i_pv >> 1) & 1) &&
+                    (!first || seg == 0 || mbar_test(&bars->o_free, (seg - 1) & 1));
+          if (__shfl_sync(0xffffffffu, ready, 0)) {
+            tc_fence_after();
+            const uint32_t stage = st_base + uint32_t(st) * kStageBytes;
+            const uint64_t a0 = smem_desc_sw128(stage + kRopeChunk * kChunkBytes, 16, 1024);
+            const uint64_t b0 = smem_desc_sw128(stage, kChunkBytes, 1024);
+            // The two output halves are independent accumulators: alternate
+            // them so consecutive MMAs do not depend on each other.
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                mma_bf16_ss_w(tmem + kHiLanes + uint32_t(h) * 256u, a0 + uint64_t((k * 32) >> 4),
+                              b0 + uint64_t((4 * h * kChunkBytes + k * 2048) >> 4), kIdescPV,
+                              !(first && k == 0));
+            }
+            mma_commit_w(&bars->empty[st]);
+            ++i_pv;
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          spins = 0;
+          t_last = global_timer_ns();
+        } else if ((++spins & 255) == 0) {
+          int give_up = 0;
+          if (lane == 0) give_up = *abort_flag || global_timer_ns() - t_last > kWaitLimitNs;
+          if (__shfl_sync(0xffffffffu, give_up, 0)) {
+            ok = false;
+            return false;
+          }
+        }
+      }
+      ++seg;
+      return true;
+    });
+    if (!ok && lane == 0) raise_abort(bars, status);
+    // Every MMA issued by this warp has completed before TMEM is freed.
+    mma_commit_w(&bars->mma_drain);
+    volatile int no_abort = 0;
+    warp_wait(&bars->mma_drain, 0, &no_abort);
   } else {
     // ------------------------------------------------------------ softmax
     const int q = warp;                      // TMEM lane quadrant
     const bool lo_half = lane < 16;
     const int row = 16 * q + (lane & 15);    // head row within the CTA
     const int head = g * kHeadsPerCta + row;
-    const uint32_t lane_base = uint32_t(32 * q) << 16;
+    const uint32_t lo_base = tmem + (uint32_t(32 * q) << 16);
+    const uint32_t hi_base = lo_base + kHiLanes;
     const int tid = threadIdx.x;             // 0..127
     float m_ref = -INFINITY, l_sum = 0.f;
     uint32_t i = 0;
     bool ok = true;
+
+    // Query block of sequence b into tensor memory (lo lanes, K-major pairs of
+    // bf16 per 32-bit column).  The two half-warps write alternate 32-column
+    // groups of the same 16 rows.
+    auto write_query = [&](int b) {
+      const int64_t qrow = int64_t(b) * H + int64_t(g) * kHeadsPerCta + row;
+      const bool valid_row = qrow < int64_t(B) * H;
+      const uint4* src = reinterpret_cast<const uint4*>(q_cat + qrow * kR);
+#pragma unroll 1
+      for (int c = 0; c < 288; c += 64) {
+        // columns [c, c+32) for threads 0-15 and [c+32, c+64) for 16-31
+        if (c + 64 <= 288) {
+          uint32_t r[32];
+          const int w0 = c + (lo_half ? 0 : 32);  // first 32-bit word of this thread
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 x = valid_row ? src[(w0 >> 2) + v] : make_uint4(0, 0, 0, 0);
+            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          }
+          tmem_st16x2_32<32>(lo_base + kColQ + uint32_t(c), r);
+        } else {
+          uint32_t r[16];
+          const int w0 = c + (lo_half ? 0 : 16);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 x = valid_row ? src[(w0 >> 2) + v] : make_uint4(0, 0, 0, 0);
+            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+          }
+          tmem_st16x2_16<16>(lo_base + kColQ + uint32_t(c), r);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->q_ready);
+    };
+
+    bool first_seg = true;
     for_each_segment(seqlens, B, cap, t_begin, t_end,
                      [&](int b, int64_t lo, int64_t hi, int64_t L) {
+      // Q of this sequence: every QK of the previous sequence has completed
+      // (its last S was read), so the query columns are free.
+      write_query(b);
+      first_seg = false;
       const int slot = b + w;
       for (int64_t t = lo; t < hi; ++t, ++i) {
-        const int s = i & 1;
-        if (!(ok = warp_wait(&bars->s_full[s], (i >> 1) & 1, abort_flag))) return false;
+        const int st = i % kStages, sb = i & 1;
+        if (!(ok = warp_wait(&bars->s_full[sb], (i >> 1) & 1, abort_flag))) return false;
         tc_fence_after();
-        uint32_t sv[64];
-        {
-          uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
-          uint32_t (&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-          tmem_ld32(tmem + lane_base + kColS + uint32_t(s) * 64u, a);
-          tmem_ld32(tmem + lane_base + kColS + uint32_t(s) * 64u + 32u, c);
-        }
+        uint32_t xs[32];   // keys 0-31 (threads 0-15) or 32-63 (threads 16-31)
+        tmem_ld16x2_32<32>(lo_base + kColS + uint32_t(sb) * 64u, xs);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&bars->s_free[s]);
+        mbar_arrive(&bars->s_free[sb]);
 
         const int64_t key0 = t * kTileKeys;
         const int valid = int(min(int64_t(kTileKeys), L - key0));
-        uint8_t* stage = sStage + s * kStageBytes;
+        uint8_t* stage = sStage + st * kStageBytes;
         if (valid < kTileKeys) {
           // Rows past the sequence end may hold anything: zero them so the
           // P.C product (where their weight is exactly 0) stays finite.
@@ -335,76 +383,79 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           }
         }
         const bool first = (t == lo);
+        const int kofs = lo_half ? 0 : 32;
+        float mt = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float x = (kofs + j < valid) ? __uint_as_float(xs[j]) * scale_log2 : -INFINITY;
+          xs[j] = __float_as_uint(x);
+          mt = fmaxf(mt, x);
+        }
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
         float alpha = 1.f;
         int resc = 0;
-        if (lo_half) {
-          float mt = -INFINITY;
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const float x = (j < valid) ? __uint_as_float(sv[j]) * scale_log2 : -INFINITY;
-            sv[j] = __float_as_uint(x);
-            mt = fmaxf(mt, x);
-          }
-          if (first) {
-            m_ref = mt;
-            l_sum = 0.f;
-          } else if (mt > m_ref + kRescaleThreshold) {
-            alpha = exp2f(m_ref - mt);
-            m_ref = mt;
-            l_sum *= alpha;
-            resc = 1;
-          }
+        if (first) {
+          m_ref = mt;
+          l_sum = 0.f;
+        } else if (mt > m_ref + kRescaleThreshold) {
+          alpha = ex2_approx(m_ref - mt);
+          m_ref = mt;
+          l_sum *= alpha;
+          resc = 1;
+        }
+        {
           float sum = 0.f;
           uint8_t* prow = stage + kRopeChunk * kChunkBytes + row * 128;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
+          for (int uu = 0; uu < 4; ++uu) {
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float p0 = exp2f(__uint_as_float(sv[8 * u + 2 * e]) - m_ref);
-              const float p1 = exp2f(__uint_as_float(sv[8 * u + 2 * e + 1]) - m_ref);
+              const float p0 = ex2_approx(__uint_as_float(xs[8 * uu + 2 * e]) - m_ref);
+              const float p1 = ex2_approx(__uint_as_float(xs[8 * uu + 2 * e + 1]) - m_ref);
               const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
               sum += __low2float(pp) + __high2float(pp);
               pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
             }
+            const int u = (kofs >> 3) + uu;
             *reinterpret_cast<uint4*>(prow + ((u ^ (row & 7)) * 16)) =
                 make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
           l_sum += sum;
         }
-        alpha = __shfl_sync(0xffffffffu, alpha, lane & 15);
-        resc = __shfl_sync(0xffffffffu, resc, lane & 15);
         if (__any_sync(0xffffffffu, resc)) {
           // O holds tile i-1's product once PV(i-1) has completed.
           const uint32_t prev = i - 1;
-          if (!(ok = warp_wait(&bars->empty[prev & 1], (prev >> 1) & 1, abort_flag))) return false;
+          if (!(ok = warp_wait(&bars->empty[prev % kStages], (prev / kStages) & 1, abort_flag)))
+            return false;
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             uint32_t r[32];
-            tmem_ld32(tmem + lane_base + uint32_t(c), r);
+            tmem_ld16x2_32<256>(hi_base + uint32_t(c), r);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(tmem + lane_base + uint32_t(c), r);
+            tmem_st16x2_32<256>(hi_base + uint32_t(c), r);
           }
           tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[s]);
+        mbar_arrive(&bars->p_full[sb]);
       }
       // Segment epilogue: normalised partial output and log-sum-exp.
       const uint32_t last = i - 1;
-      if (!(ok = warp_wait(&bars->empty[last & 1], (last >> 1) & 1, abort_flag))) return false;
+      if (!(ok = warp_wait(&bars->empty[last % kStages], (last / kStages) & 1, abort_flag)))
+        return false;
       tc_fence_after();
-      const float l_row = __shfl_sync(0xffffffffu, l_sum, lane & 15);
+      const float l_row = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
       const float inv = 1.f / l_row;
       float* dst = o_part + (int64_t(slot) * H + head) * kDc + (lo_half ? 0 : 256);
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_base + uint32_t(c), r);
+        tmem_ld16x2_32<256>(hi_base + uint32_t(c), r);
         tmem_wait_ld();
         if (head < H) {
 #pragma unroll
@@ -415,11 +466,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       }
       if (lo_half && head < H)
-        lse_part[int64_t(slot) * H + head] = (m_ref + log2f(l_sum)) * 0.69314718055994531f;
+        lse_part[int64_t(slot) * H + head] = (m_ref + log2f(l_row)) * 0.69314718055994531f;
       tc_fence_before();
       mbar_arrive(&bars->o_free);
       return true;
     });
+    (void)first_seg;
     if (!ok && lane == 0) raise_abort(bars, status);
   }
 
@@ -473,10 +525,8 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
                              cudaStream_t stream) {
   if (int64_t(B) * cap >= (int64_t(1) << 31) || int64_t(B) * H >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
-  CUtensorMap tm_q, tm_c;
-  if (!make_rows_map(&tm_q, q_cat, uint64_t(B) * H) ||
-      !make_rows_map(&tm_c, cache, uint64_t(B) * uint64_t(cap)))
-    return cudaErrorInvalidValue;
+  CUtensorMap tm_c;
+  if (!make_rows_map(&tm_c, cache, uint64_t(B) * uint64_t(cap))) return cudaErrorInvalidValue;
   static bool attr_done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -489,7 +539,7 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
   }
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(decode_tc_head_groups(H), W);
-  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_q, tm_c, seqlens, B, H, cap,
+  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_c, q_cat, seqlens, B, H, cap,
                                                            scale_log2, W, o_part, lse_part,
                                                            status);
   return cudaGetLastError();
