@@ -98,10 +98,11 @@ MLA_API int64_t mla_cache_row_elems(int32_t d_c, int32_t d_r);
  * gamma   [d_c] fp32, or NULL for ones
  * cache   [B, cache_capacity, d_c + d_r] dtype, written at row L_b only
  * seqlens [B] int32, read then incremented on the device
- * workspace  >= mla_cache_append_workspace_bytes(dims) bytes of device scratch
+ * workspace  >= mla_cache_append_workspace_bytes(dims, hidden) bytes of device scratch
+ *             (partial sums of the projection; contents need not be initialised)
  * A sequence already at capacity is left untouched and sets MLA_ERR_BOUNDS in
  * the device status word. */
-MLA_API size_t mla_cache_append_workspace_bytes(const mla_dims* dims);
+MLA_API size_t mla_cache_append_workspace_bytes(const mla_dims* dims, int32_t hidden);
 MLA_API int mla_cache_append(const mla_dims* dims, int32_t hidden, const void* h,
                      const void* W_DKV, const float* gamma, float eps,
                      float rope_base, void* cache, int32_t* seqlens,

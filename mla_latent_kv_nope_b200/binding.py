@@ -86,7 +86,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     D = ctypes.POINTER(CDims)
     sig = {
         "mla_cache_row_elems": (I64, [I32, I32]),
-        "mla_cache_append_workspace_bytes": (SZ, [D]),
+        "mla_cache_append_workspace_bytes": (SZ, [D, I32]),
         "mla_cache_append": (ctypes.c_int, [D, I32, P, P, P, F, F, P, P, P, SZ, P]),
         "mla_absorb_q": (ctypes.c_int, [D, P, P, P, P, F, P, P]),
         "mla_decode_default_splits": (ctypes.c_int, [D]),
@@ -140,8 +140,8 @@ def cache_row_elems(d_c: int, d_r: int) -> int:
     return int(load_library().mla_cache_row_elems(d_c, d_r))
 
 
-def cache_append_workspace_bytes(dims: Dims) -> int:
-    return int(load_library().mla_cache_append_workspace_bytes(ctypes.byref(dims.c())))
+def cache_append_workspace_bytes(dims: Dims, hidden: int) -> int:
+    return int(load_library().mla_cache_append_workspace_bytes(ctypes.byref(dims.c()), hidden))
 
 
 def cache_append(dims: Dims, h, W_DKV, gamma, cache, seqlens, workspace, eps=1e-6,
@@ -239,7 +239,8 @@ class DecodeStep:
         self.num_splits = num_splits or decode_default_splits(dims)
         ws = decode_workspace_bytes(dims, self.num_splits)
         self.ws = torch.empty(ws // 4, dtype=torch.float32, device=device)
-        self.ws_append = torch.empty(max(cache_append_workspace_bytes(dims) // 4, 1),
+        hidden = W_DKV.shape[1] if W_DKV is not None else 1
+        self.ws_append = torch.empty(max(cache_append_workspace_bytes(dims, hidden) // 4, 1),
                                      dtype=torch.float32, device=device)
         dt = dims.torch_dtype
         self.q_cat = torch.empty(dims.B, dims.H, dims.R, dtype=dt, device=device)

@@ -70,16 +70,19 @@ __device__ __forceinline__ int64_t worker_of_tile(int64_t t, int64_t T, int64_t 
 }
 
 // RoPE angle pair for element pair k of a d-wide rotary block at position pos:
-// theta = pos * base^(-2k/d), evaluated in double so that long contexts keep
-// full fp32 accuracy after the reduction.
+// theta = pos * base^(-2k/d).  The frequency and the product are formed in
+// double and theta is reduced to [-pi, pi] in double (Cody-Waite style with a
+// two-part 2*pi), so the single-precision sincos only ever sees a small,
+// exact-enough argument even at positions ~1e5.
 __device__ __forceinline__ void rope_cos_sin(int64_t pos, int k, int d, float base,
                                              float* c, float* s) {
-  double inv = pow(double(base), -2.0 * double(k) / double(d));
-  double th = double(pos) * inv;
-  double sd, cd;
-  sincos(th, &sd, &cd);
-  *c = float(cd);
-  *s = float(sd);
+  const double inv = exp2(-2.0 * double(k) / double(d) * log2(double(base)));
+  const double th = double(pos) * inv;
+  const double kTwoPiHi = 6.283185307179586232;      // 2*pi rounded to double
+  const double kTwoPiLo = 2.4492935982947064e-16;    // 2*pi - kTwoPiHi
+  const double n = rint(th * 0.15915494309189535);   // th / (2*pi)
+  const double r = fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, th));
+  sincosf(float(r), s, c);
 }
 
 }  // namespace mla

@@ -70,16 +70,36 @@ append_project_kernel(const T* __restrict__ h, const T* __restrict__ W, int B, i
 
 template <typename T>
 __global__ void __launch_bounds__(kApThreads)
-append_finalize_kernel(const float* __restrict__ x, const float* __restrict__ gamma,
-                       float eps, float rope_base, int d_c, int d_r, int64_t cap,
-                       T* __restrict__ cache, int32_t* __restrict__ seqlens,
-                       int* __restrict__ status) {
+append_finalize_kernel(const float* __restrict__ part, int n_parts,
+                       const float* __restrict__ gamma, float eps, float rope_base, int d_c,
+                       int d_r, int64_t cap, T* __restrict__ cache,
+                       int32_t* __restrict__ seqlens, int* __restrict__ status) {
   const int b = blockIdx.x;
+  const int B = gridDim.x;
   const int R = d_c + d_r;
+  extern __shared__ float s_x[];  // [R]: the projection, summed over parts in order
   __shared__ float s_part[kApThreads / 32];
   __shared__ int32_t s_L;
   if (threadIdx.x == 0) s_L = seqlens[b];
-  const float* xb = x + int64_t(b) * R;
+  // Sum the partials in a fixed order (deterministic); 4 loads in flight.
+  for (int c = threadIdx.x; c < R; c += kApThreads) {
+    const float* src = part + int64_t(b) * R + c;
+    const int64_t stride = int64_t(B) * R;
+    float v = 0.f;
+    int p = 0;
+    for (; p + 4 <= n_parts; p += 4) {
+      const float a0 = src[(p + 0) * stride], a1 = src[(p + 1) * stride];
+      const float a2 = src[(p + 2) * stride], a3 = src[(p + 3) * stride];
+      v += a0;
+      v += a1;
+      v += a2;
+      v += a3;
+    }
+    for (; p < n_parts; ++p) v += src[p * stride];
+    s_x[c] = v;
+  }
+  __syncthreads();
+  const float* xb = s_x;
   float ss = 0.f;
   for (int c = threadIdx.x; c < d_c; c += kApThreads) ss = fmaf(xb[c], xb[c], ss);
   ss = warp_sum(ss);
@@ -123,10 +143,28 @@ cudaError_t launch_cache_append(const T* h, const T* W_DKV, const float* gamma, 
       h, W_DKV, B, R, hidden, x_ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  append_finalize_kernel<T><<<B, kApThreads, 0, stream>>>(x_ws, gamma, eps, rope_base, d_c,
-                                                          d_r, cap, cache, seqlens, status);
+  return launch_append_finalize<T>(x_ws, 1, gamma, eps, rope_base, B, d_c, d_r, cap, cache,
+                                   seqlens, status, stream);
+}
+
+template <typename T>
+cudaError_t launch_append_finalize(const float* part, int n_parts, const float* gamma, float eps,
+                                   float rope_base, int B, int d_c, int d_r, int64_t cap,
+                                   T* cache, int32_t* seqlens, int* status, cudaStream_t stream) {
+  const size_t smem = sizeof(float) * size_t(d_c + d_r);
+  append_finalize_kernel<T><<<B, kApThreads, smem, stream>>>(part, n_parts, gamma, eps, rope_base,
+                                                             d_c, d_r, cap, cache, seqlens,
+                                                             status);
   return cudaGetLastError();
 }
+
+template cudaError_t launch_append_finalize<float>(const float*, int, const float*, float, float,
+                                                   int, int, int, int64_t, float*, int32_t*, int*,
+                                                   cudaStream_t);
+template cudaError_t launch_append_finalize<__nv_bfloat16>(const float*, int, const float*, float,
+                                                           float, int, int, int, int64_t,
+                                                           __nv_bfloat16*, int32_t*, int*,
+                                                           cudaStream_t);
 
 template cudaError_t launch_cache_append<float>(const float*, const float*, const float*,
                                                 float, float, int, int, int, int, int64_t,

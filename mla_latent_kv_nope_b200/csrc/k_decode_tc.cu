@@ -77,9 +77,15 @@ struct Barriers {
   int abort_flag;
 };
 
+// Exclusive prefix of per-sequence tile counts, built once per CTA so that no
+// role walks the length array through global memory (a chain of dependent
+// loads).  Batches with more sequences fall back to walking global memory.
+constexpr int kMaxSeqSmem = 2048;
+
 constexpr size_t kOffStage = 0;
 constexpr size_t kOffBar = size_t(kStages) * kStageBytes;
-constexpr size_t kSmemBytes = kOffBar + sizeof(Barriers) + 1024;  // + alignment slack
+constexpr size_t kOffPrefix = kOffBar + ((sizeof(Barriers) + 15) / 16) * 16;
+constexpr size_t kSmemBytes = kOffPrefix + sizeof(int32_t) * (kMaxSeqSmem + 1) + 1024;
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256, false, true);
@@ -104,20 +110,52 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Sequences overlapping this worker's tile range are visited in order; the
-// callback gets (b, first tile, end tile (both local to b), length).
-template <typename F>
-__device__ __forceinline__ void for_each_segment(const int32_t* seqlens, int B, int64_t cap,
-                                                 int64_t t_begin, int64_t t_end, F&& f) {
-  int64_t prefix = 0;
-  for (int b = 0; b < B && prefix < t_end; ++b) {
-    const int64_t L = clamp_len(seqlens[b], cap);
-    const int64_t nt = tiles_of(L);
-    const int64_t lo = max(prefix, t_begin), hi = min(prefix + nt, t_end);
-    if (lo < hi) {
-      if (!f(b, lo - prefix, hi - prefix, L)) return;
+// Tile prefix of the batch: prefix(b) = sum of tiles of sequences < b, from
+// shared memory when the batch fits, else recomputed from the lengths.
+struct TilePrefix {
+  const int32_t* sp;       // shared prefix [B + 1] or nullptr
+  const int32_t* seqlens;
+  int B;
+  int64_t cap;
+  __device__ int64_t at(int b) const {
+    if (sp) return sp[b];
+    int64_t p = 0;
+    for (int k = 0; k < b; ++k) p += tiles_of(clamp_len(seqlens[k], cap));
+    return p;
+  }
+  __device__ int64_t len(int b) const { return clamp_len(seqlens[b], cap); }
+  // First sequence whose tiles end after tile t (binary search on the prefix).
+  __device__ int first_after(int64_t t) const {
+    if (!sp) {
+      int64_t p = 0;
+      for (int b = 0; b < B; ++b) {
+        p += tiles_of(len(b));
+        if (p > t) return b;
+      }
+      return B;
     }
-    prefix += nt;
+    int lo = 0, hi = B;  // smallest b with sp[b + 1] > t
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sp[mid + 1] > t) hi = mid; else lo = mid + 1;
+    }
+    return lo;
+  }
+};
+
+// Sequences overlapping this worker's tile range are visited in order; the
+// callback gets (b, first tile, end tile (both local to b), length) and
+// returns false to stop.
+template <typename F>
+__device__ __forceinline__ void for_each_segment(const TilePrefix& tp, int64_t t_begin,
+                                                 int64_t t_end, F&& f) {
+  for (int b = tp.first_after(t_begin); b < tp.B; ++b) {
+    const int64_t pre = tp.at(b);
+    if (pre >= t_end) return;
+    const int64_t L = tp.len(b);
+    const int64_t nt = tiles_of(L);
+    const int64_t lo = max(pre, t_begin), hi = min(pre + nt, t_end);
+    if (lo < hi && !f(b, lo - pre, hi - pre, L)) return;
   }
 }
 
@@ -136,8 +174,35 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
   const int w = blockIdx.y;   // worker
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // Tile prefix of the batch (all threads load lengths in parallel; warp 0
+  // scans 32 at a time with shuffles).
+  int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + kOffPrefix);
+  const bool prefix_in_smem = B <= kMaxSeqSmem;
   int64_t n_tiles = 0;
-  for (int b = 0; b < B; ++b) n_tiles += tiles_of(clamp_len(seqlens[b], cap));
+  if (prefix_in_smem) {
+    for (int b = threadIdx.x; b < B; b += kThreads)
+      s_prefix[b + 1] = int32_t(tiles_of(clamp_len(seqlens[b], cap)));
+    __syncthreads();
+    if (warp == 0) {
+      int32_t carry = 0;
+      for (int b0 = 0; b0 < B; b0 += 32) {
+        int32_t v = (b0 + lane < B) ? s_prefix[b0 + lane + 1] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        if (b0 + lane < B) s_prefix[b0 + lane + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) s_prefix[0] = 0;
+    }
+    __syncthreads();
+    n_tiles = s_prefix[B];
+  } else {
+    for (int b = 0; b < B; ++b) n_tiles += tiles_of(clamp_len(seqlens[b], cap));
+  }
+  const TilePrefix tp{prefix_in_smem ? s_prefix : nullptr, seqlens, B, cap};
   if (n_tiles == 0) return;
   const int64_t t_begin = worker_tile_begin(w, n_tiles, W);
   const int64_t t_end = worker_tile_begin(w + 1, n_tiles, W);
@@ -176,7 +241,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     if (lane == 0) {
       uint32_t i = 0;
       bool ok = true;
-      for_each_segment(seqlens, B, cap, t_begin, t_end,
+      for_each_segment(tp, t_begin, t_end,
                        [&](int b, int64_t lo, int64_t hi, int64_t) {
         // One CTA per tile range (head group 0) pulls tiles into L2 a few
         // tiles ahead; the shared-memory loads of every head group hit L2.
@@ -218,7 +283,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     int seg = 0;
     bool ok = true;
     const uint32_t st_base = smem_u32(sStage);
-    for_each_segment(seqlens, B, cap, t_begin, t_end,
+    for_each_segment(tp, t_begin, t_end,
                      [&](int, int64_t lo, int64_t hi, int64_t) {
       const uint32_t base = i_pv, end = i_pv + uint32_t(hi - lo);
       // The softmax warps have written this sequence's query block.
@@ -316,47 +381,66 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     bool ok = true;
 
     // Query block of sequence b into tensor memory (lo lanes, K-major pairs of
-    // bf16 per 32-bit column).  The two half-warps write alternate 32-column
-    // groups of the same 16 rows.
+    // bf16 per 32-bit column).  The two half-warps write alternate column
+    // groups of the same 16 rows.  All 36 16-byte loads of a thread are
+    // issued before the first store, so the block costs one memory round trip.
     auto write_query = [&](int b) {
       const int64_t qrow = int64_t(b) * H + int64_t(g) * kHeadsPerCta + row;
       const bool valid_row = qrow < int64_t(B) * H;
       const uint4* src = reinterpret_cast<const uint4*>(q_cat + qrow * kR);
-#pragma unroll 1
-      for (int c = 0; c < 288; c += 64) {
-        // columns [c, c+32) for threads 0-15 and [c+32, c+64) for 16-31
-        if (c + 64 <= 288) {
-          uint32_t r[32];
-          const int w0 = c + (lo_half ? 0 : 32);  // first 32-bit word of this thread
+      uint4 v[36];
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint4 x = valid_row ? src[(w0 >> 2) + v] : make_uint4(0, 0, 0, 0);
-            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
-          }
-          tmem_st16x2_32<32>(lo_base + kColQ + uint32_t(c), r);
-        } else {
-          uint32_t r[16];
-          const int w0 = c + (lo_half ? 0 : 16);
+      for (int j = 0; j < 32; ++j) {   // four 64-column groups: words [64c + half*32, +32)
+        const int word = (j / 8) * 64 + (lo_half ? 0 : 32) + (j % 8) * 4;
+        v[j] = valid_row ? src[word >> 2] : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 x = valid_row ? src[(w0 >> 2) + v] : make_uint4(0, 0, 0, 0);
-            r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
-          }
-          tmem_st16x2_16<16>(lo_base + kColQ + uint32_t(c), r);
+      for (int j = 0; j < 4; ++j) {    // last 32 columns: words [256 + half*16, +16)
+        const int word = 256 + (lo_half ? 0 : 16) + j * 4;
+        v[32 + j] = valid_row ? src[word >> 2] : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          r[4 * q4] = v[8 * c + q4].x; r[4 * q4 + 1] = v[8 * c + q4].y;
+          r[4 * q4 + 2] = v[8 * c + q4].z; r[4 * q4 + 3] = v[8 * c + q4].w;
         }
+        tmem_st16x2_32<32>(lo_base + kColQ + uint32_t(64 * c), r);
+      }
+      {
+        uint32_t r[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          r[4 * q4] = v[32 + q4].x; r[4 * q4 + 1] = v[32 + q4].y;
+          r[4 * q4 + 2] = v[32 + q4].z; r[4 * q4 + 3] = v[32 + q4].w;
+        }
+        tmem_st16x2_16<16>(lo_base + kColQ + 256u, r);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->q_ready);
     };
 
-    bool first_seg = true;
-    for_each_segment(seqlens, B, cap, t_begin, t_end,
+    // The sequence of the worker's range that follows sequence `after`
+    // (-1 for the first), or -1 if there is none.
+    auto next_sequence = [&](int after) {
+      for (int bb = (after < 0 ? tp.first_after(t_begin) : after + 1); bb < B; ++bb) {
+        const int64_t pre = tp.at(bb);
+        if (pre >= t_end) return -1;
+        if (tiles_of(tp.len(bb)) > 0 && pre + tiles_of(tp.len(bb)) > t_begin) return bb;
+      }
+      return -1;
+    };
+
+    // The first sequence's query block; each later one is written as soon as
+    // the previous sequence's last S has been read (all its QK^T are done),
+    // before that sequence's epilogue, so the next QK^T overlaps the stores.
+    const int first_b = next_sequence(-1);
+    if (first_b >= 0) write_query(first_b);
+    for_each_segment(tp, t_begin, t_end,
                      [&](int b, int64_t lo, int64_t hi, int64_t L) {
-      // Q of this sequence: every QK of the previous sequence has completed
-      // (its last S was read), so the query columns are free.
-      write_query(b);
-      first_seg = false;
       const int slot = b + w;
       for (int64_t t = lo; t < hi; ++t, ++i) {
         const int st = i % kStages, sb = i & 1;
@@ -444,6 +528,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
         tc_fence_before();
         mbar_arrive(&bars->p_full[sb]);
       }
+      // Every QK^T of this sequence has been read back: load the next query.
+      const int nb = next_sequence(b);
+      if (nb >= 0) write_query(nb);
       // Segment epilogue: normalised partial output and log-sum-exp.
       const uint32_t last = i - 1;
       if (!(ok = warp_wait(&bars->empty[last % kStages], (last / kStages) & 1, abort_flag)))
@@ -471,7 +558,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
       mbar_arrive(&bars->o_free);
       return true;
     });
-    (void)first_seg;
     if (!ok && lane == 0) raise_abort(bars, status);
   }
 

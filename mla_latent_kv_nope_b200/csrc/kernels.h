@@ -41,5 +41,24 @@ cudaError_t launch_cache_append(const T* h, const T* W_DKV, const float* gamma, 
                                 float rope_base, int B, int d_c, int d_r, int hidden,
                                 int64_t cap, T* cache, int32_t* seqlens, float* x_ws,
                                 int* status, cudaStream_t stream);
+// Finalize only (norm, rotation, store, length bump) over n_parts partial sums
+// part[p][b][r] of the projection.
+template <typename T>
+cudaError_t launch_append_finalize(const float* part, int n_parts, const float* gamma, float eps,
+                                   float rope_base, int B, int d_c, int d_r, int64_t cap,
+                                   T* cache, int32_t* seqlens, int* status, cudaStream_t stream);
+
+// Tensor-core kernels for the bf16 step (d_c = 512, d_r = 64, d_nope = d_v = 128).
+bool gemm_tc_supported(int d_c, int d_r, int d_n, int d_v);
+cudaError_t launch_out_proj_tc(const float* o_lat, const __nv_bfloat16* W_UV, int B, int H,
+                               __nv_bfloat16* out, int* status, cudaStream_t stream);
+cudaError_t launch_absorb_q_tc(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_pe,
+                               const __nv_bfloat16* W_UK, const int32_t* q_pos, float rope_base,
+                               int B, int H, __nv_bfloat16* q_cat, int* status,
+                               cudaStream_t stream);
+int append_tc_splits(int hidden);
+cudaError_t launch_append_proj_tc(const __nv_bfloat16* h, const __nv_bfloat16* W_DKV, int B,
+                                  int R, int hidden, float* part, int* status,
+                                  cudaStream_t stream);
 
 }  // namespace mla

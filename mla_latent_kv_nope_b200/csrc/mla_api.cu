@@ -118,9 +118,16 @@ int mla_get_device_status(void* stream) {
 }
 
 // ---------------------------------------------------------------------------
-size_t mla_cache_append_workspace_bytes(const mla_dims* d) {
-  if (check_dims(d) != MLA_OK) return 0;
-  return round_up(size_t(d->B) * size_t(d->d_c + d->d_r) * sizeof(float), 256);
+namespace {
+bool use_tc_gemm(const mla_dims* d) {
+  return d->dtype == MLA_BF16 && gemm_tc_supported(d->d_c, d->d_r, d->d_nope, d->d_v);
+}
+}  // namespace
+
+size_t mla_cache_append_workspace_bytes(const mla_dims* d, int32_t hidden) {
+  if (check_dims(d) != MLA_OK || hidden <= 0) return 0;
+  const size_t parts = use_tc_gemm(d) ? size_t(append_tc_splits(hidden)) : 1;
+  return round_up(parts * size_t(d->B) * size_t(d->d_c + d->d_r) * sizeof(float), 256);
 }
 
 int mla_cache_append(const mla_dims* d, int32_t hidden, const void* h, const void* W_DKV,
@@ -134,9 +141,19 @@ int mla_cache_append(const mla_dims* d, int32_t hidden, const void* h, const voi
   if (!aligned16(h) || !aligned16(W_DKV) || !aligned16(cache) || !aligned16(seqlens) ||
       (gamma && !aligned16(gamma)) || (workspace && !aligned16(workspace)))
     return MLA_ERR_ALIGNMENT;
-  if (!workspace || workspace_bytes < mla_cache_append_workspace_bytes(d)) return MLA_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < mla_cache_append_workspace_bytes(d, hidden))
+    return MLA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* x = static_cast<float*>(workspace);
+  if (use_tc_gemm(d)) {
+    cudaError_t e = launch_append_proj_tc(static_cast<const __nv_bfloat16*>(h),
+                                          static_cast<const __nv_bfloat16*>(W_DKV), d->B,
+                                          d->d_c + d->d_r, hidden, x, status_ptr(), s);
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    return cuda_status(launch_append_finalize<__nv_bfloat16>(
+        x, append_tc_splits(hidden), gamma, eps, rope_base, d->B, d->d_c, d->d_r,
+        d->cache_capacity, static_cast<__nv_bfloat16*>(cache), seqlens, status_ptr(), s));
+  }
   if (d->dtype == MLA_BF16)
     return cuda_status(launch_cache_append<__nv_bfloat16>(
         static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(W_DKV), gamma,
@@ -159,6 +176,11 @@ int mla_absorb_q(const mla_dims* d, const void* q_nope, const void* q_pe, const 
       !aligned16(q_cat) || (q_pos && !aligned16(q_pos)))
     return MLA_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_tc_gemm(d))
+    return cuda_status(launch_absorb_q_tc(
+        static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_pe),
+        static_cast<const __nv_bfloat16*>(W_UK), q_pos, rope_base, d->B, d->H,
+        static_cast<__nv_bfloat16*>(q_cat), status_ptr(), s));
   if (d->dtype == MLA_BF16)
     return cuda_status(launch_absorb_q<__nv_bfloat16>(
         static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_pe),
@@ -253,6 +275,9 @@ int mla_out_proj(const mla_dims* d, const float* o_lat, const void* W_UV, void* 
   if (!o_lat || !W_UV || !out) return MLA_ERR_INVALID_ARG;
   if (!aligned16(o_lat) || !aligned16(W_UV) || !aligned16(out)) return MLA_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (use_tc_gemm(d))
+    return cuda_status(launch_out_proj_tc(o_lat, static_cast<const __nv_bfloat16*>(W_UV), d->B,
+                                          d->H, static_cast<__nv_bfloat16*>(out), status_ptr(), s));
   if (d->dtype == MLA_BF16)
     return cuda_status(launch_out_proj<__nv_bfloat16>(o_lat,
                                                       static_cast<const __nv_bfloat16*>(W_UV),

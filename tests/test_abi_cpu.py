@@ -65,7 +65,10 @@ def test_workspace_layout_formula(lib):
         expect = r256(slots * H * 512 * 4) + r256(slots * H * 4)
         assert lib.mla_decode_workspace_bytes(ctypes.byref(d), W) == expect
     d = _dims(B=64, d_c=512, d_r=64)
-    assert lib.mla_cache_append_workspace_bytes(ctypes.byref(d)) == 64 * 576 * 4
+    # bf16 standard dims: one fp32 partial per 256-wide slice of the hidden dim
+    assert lib.mla_cache_append_workspace_bytes(ctypes.byref(d), 7168) == 28 * 64 * 576 * 4
+    f = _dims(B=3, d_c=32, d_r=16, d_nope=16, d_v=16, dtype=bd.MLA_F32)
+    assert lib.mla_cache_append_workspace_bytes(ctypes.byref(f), 64) == 256 * 3  # 3*48*4 -> 576, rounded to 768
     assert lib.mla_decode_workspace_bytes(ctypes.byref(d), 2000) == 0  # > 1024 splits
 
 
@@ -119,7 +122,7 @@ def test_other_entry_point_errors(lib):
     assert lib.mla_absorb_q(ctypes.byref(d), GOOD, GOOD, GOOD, GOOD, -1.0, GOOD2, None) == INVALID
     assert lib.mla_absorb_q(ctypes.byref(d), GOOD, GOOD, GOOD, BAD, 1e4, GOOD2, None) == ALIGN
     # cache append
-    wsb = lib.mla_cache_append_workspace_bytes(ctypes.byref(d))
+    wsb = lib.mla_cache_append_workspace_bytes(ctypes.byref(d), 7168)
     ap = lambda hidden=7168, h=GOOD, eps=1e-6, base=1e4, ws=GOOD2, n=wsb: lib.mla_cache_append(  # noqa: E731
         ctypes.byref(d), hidden, h, GOOD, None, eps, base, GOOD, GOOD, ws, n, None)
     assert ap(hidden=0) == INVALID

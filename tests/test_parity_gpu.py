@@ -90,7 +90,7 @@ def test_cache_append(w):
     cache = torch.full((w.B, w.capacity, w.R), -3.25, dtype=dt, device="cuda")
     before = cache.clone()
     seq = torch.from_numpy(lens).cuda()
-    ws = torch.empty(mla.cache_append_workspace_bytes(d) // 4, dtype=torch.float32,
+    ws = torch.empty(mla.cache_append_workspace_bytes(d, h.shape[1]) // 4, dtype=torch.float32,
                      device="cuda")
     mla.cache_append(d, dev(h, w), dev(Wdkv, w), torch.from_numpy(gamma).cuda(), cache, seq, ws,
                      eps=w.eps)
@@ -116,7 +116,7 @@ def test_cache_append_capacity_is_reported():
     h, Wdkv = inputs.append_inputs(w)
     cache = torch.zeros(w.B, 10, w.R, dtype=torch.bfloat16, device="cuda")
     seq = torch.from_numpy(lens).cuda()
-    ws = torch.empty(mla.cache_append_workspace_bytes(d) // 4, dtype=torch.float32, device="cuda")
+    ws = torch.empty(mla.cache_append_workspace_bytes(d, h.shape[1]) // 4, dtype=torch.float32, device="cuda")
     mla.get_device_status()
     mla.cache_append(d, dev(h, w), dev(Wdkv, w), None, cache, seq, ws)
     assert mla.get_device_status() == 7  # MLA_ERR_BOUNDS
