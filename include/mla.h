@@ -130,7 +130,9 @@ MLA_API int mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q
  * the concatenated per-sequence tile lists, T = sum_b ceil(L_b/64)).  Worker w
  * writes, for each sequence b it touches, partial slot (b + w):
  *   o_part[b+w][i][:] = sum_{j in range} e^{s_j - lse_part} c_j,   lse_part[b+w][i] = log sum e^{s_j}
- * Workspace layout (fp32): o_part [B + W - 1][H][d_c], then lse_part [B + W - 1][H].
+ * Workspace layout (fp32): o_part [B + W - 1][d_c / 4][H][4] (column c of
+ * head i at [slot][c / 4][i][c % 4], so 4-column groups of consecutive heads
+ * are contiguous), then, 256-byte aligned, lse_part [B + W - 1][H].
  * Rows j >= L_b never influence the result (they may hold anything).
  * num_splits = 0 picks the default for the current device; the number used is
  * returned through splits_used (may be NULL). */

@@ -6,7 +6,7 @@
 // The partials of sequence b live in slots (b + w) for every non-empty worker
 // w whose tile range meets b's tiles; the block recomputes that set from the
 // sequence lengths exactly as the decode kernels dealt the tiles.
-// (Kernel layout: see combine_kernel.)
+// Partials are stored as o_part[slot][d_c / 4][H][4] (see combine_kernel).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -14,23 +14,35 @@ namespace mla {
 
 namespace {
 
-constexpr int kCombineWarps = 8;   // heads per block (one warp each)
+constexpr int kCombineHeads = 32;    // heads per block, one per lane
+constexpr int kCombineWarps = 8;
 constexpr int kCombineThreads = 32 * kCombineWarps;
-constexpr int kMaxDcPerLane = 32;  // d_c <= 1024
+constexpr int kQuadsPerWarp = 4;     // 4-column groups per warp
+constexpr int kQuadsPerBlock = kCombineWarps * kQuadsPerWarp;   // 128 columns
 
-// Block = (sequence b, group of 8 heads).  The tile prefix of b and the total
-// are reduced by the whole block; then each warp merges one head: its lanes
-// read the partials' lse values, reduce max and sum with shuffles, and
-// accumulate d_c / 32 columns each over the partials (loads in flight
-// together rather than one after another).
+// Block = (sequence b, 32 heads, 128 columns).  The partials are stored as
+// o_part[slot][d_c / 4][H][4], so a warp load of one 4-column group for 32
+// consecutive heads is one contiguous 512-byte read.  Each thread owns one
+// head (its lane) and 4 column groups; it reduces the lse values of the
+// head's partials (max, then the sum of exponentials) and accumulates its
+// columns over the partials, two partials per step (8 loads in flight).  The
+// merged block goes through shared memory so o_lat rows are written with
+// coalesced stores.
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, int d_c, int W,
                const float* __restrict__ o_part, const float* __restrict__ lse_part,
                float* __restrict__ o_lat, float* __restrict__ lse_out) {
+  __shared__ float4 s_rows[kCombineHeads][kQuadsPerBlock + 1];
+  __shared__ int64_t s_red[2][kCombineWarps];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.y * kCombineWarps + warp;
-  __shared__ int64_t s_red[2][kCombineWarps];
+  const int h0 = blockIdx.y * kCombineHeads;
+  const int i = h0 + lane;
+  const bool head_ok = i < H;
+  const int nq = d_c / 4;
+  const int q_base = blockIdx.z * kQuadsPerBlock;
+  const int nqb = min(kQuadsPerBlock, nq - q_base);
+  const int nh = min(kCombineHeads, H - h0);
   int64_t pre = 0, tot = 0;
   for (int bb = threadIdx.x; bb < B; bb += kCombineThreads) {
     const int64_t nt = tiles_of(clamp_len(seqlens[bb], cap));
@@ -54,83 +66,62 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
     pre += s_red[0][k];
     tot += s_red[1][k];
   }
-  if (i >= H) return;
   const int64_t T = tot;
   const int64_t nt = tiles_of(clamp_len(seqlens[b], cap));
-  float* dst = o_lat + (int64_t(b) * H + i) * d_c;
   if (nt == 0) {
-    for (int c = lane * 4; c < d_c; c += 128)
-      *reinterpret_cast<float4*>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lane == 0 && lse_out) lse_out[int64_t(b) * H + i] = -INFINITY;
+    for (int idx = threadIdx.x; idx < nh * nqb; idx += kCombineThreads)
+      reinterpret_cast<float4*>(o_lat + (int64_t(b) * H + h0 + idx / nqb) * d_c)[q_base + idx % nqb] =
+          make_float4(0.f, 0.f, 0.f, 0.f);
+    if (blockIdx.z == 0 && warp == 0 && head_ok && lse_out) lse_out[int64_t(b) * H + i] = -INFINITY;
     return;
   }
   const int w_first = int(worker_of_tile(pre, T, W));
   const int w_last = int(worker_of_tile(pre + nt - 1, T, W));
-  // Weights of the partials: lane k holds partial k's lse (32 at a time).
-  const int nw = w_last - w_first + 1;
+  auto live = [&](int w) { return worker_tile_begin(w, T, W) != worker_tile_begin(w + 1, T, W); };
   float m = -INFINITY;
-  for (int k0 = 0; k0 < nw; k0 += 32) {
-    const int w = w_first + k0 + lane;
-    const bool live = (k0 + lane < nw) &&
-                      worker_tile_begin(w, T, W) != worker_tile_begin(w + 1, T, W);
-    if (live) m = fmaxf(m, lse_part[int64_t(b + w) * H + i]);
-  }
-  m = warp_max(m);
+  for (int w = w_first; w <= w_last; ++w)
+    if (live(w) && head_ok) m = fmaxf(m, lse_part[int64_t(b + w) * H + i]);
   float z = 0.f;
-  float my_e = 0.f;  // exp(lse - m) of this lane's partial in the first 32
-  for (int k0 = 0; k0 < nw; k0 += 32) {
-    const int w = w_first + k0 + lane;
-    const bool live = (k0 + lane < nw) &&
-                      worker_tile_begin(w, T, W) != worker_tile_begin(w + 1, T, W);
-    const float e = live ? expf(lse_part[int64_t(b + w) * H + i] - m) : 0.f;
-    if (k0 == 0) my_e = e;
-    z += e;
-  }
-  z = warp_sum(z);
-  const float inv_z = 1.f / z;
-  float acc[kMaxDcPerLane / 4][4];
+  for (int w = w_first; w <= w_last; ++w)
+    if (live(w) && head_ok) z += expf(lse_part[int64_t(b + w) * H + i] - m);
+  const float inv_z = head_ok ? 1.f / z : 0.f;
+  // Column groups of this thread: q_base + warp + 8 j, j < 4.
+  const float4* src0 = reinterpret_cast<const float4*>(o_part) + int64_t(q_base + warp) * H + i;
+  const int64_t slot_stride = int64_t(nq) * H;   // float4 units
+  float4 acc[kQuadsPerWarp];
 #pragma unroll
-  for (int q = 0; q < kMaxDcPerLane / 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
-  // Partials two at a time so their loads are in flight together.
-  for (int k = 0; k < nw; k += 2) {
-    const int wa = w_first + k, wb = w_first + k + 1;
-    float ea = k < 32 ? __shfl_sync(0xffffffffu, my_e, k) : 0.f;
-    float eb = k + 1 < 32 ? __shfl_sync(0xffffffffu, my_e, min(k + 1, 31)) : 0.f;
-    if (k >= 32) {
-      const bool la = worker_tile_begin(wa, T, W) != worker_tile_begin(wa + 1, T, W);
-      ea = la ? expf(lse_part[int64_t(b + wa) * H + i] - m) : 0.f;
-    }
-    if (k + 1 >= 32 && k + 1 < nw) {
-      const bool lb = worker_tile_begin(wb, T, W) != worker_tile_begin(wb + 1, T, W);
-      eb = lb ? expf(lse_part[int64_t(b + wb) * H + i] - m) : 0.f;
-    }
-    if (k + 1 >= nw) eb = 0.f;
-    ea *= inv_z;
-    eb *= inv_z;
-    const float* sa = o_part + (int64_t(b + wa) * H + i) * d_c;
-    const float* sb = o_part + (int64_t(b + min(wb, w_last)) * H + i) * d_c;
+  for (int j = 0; j < kQuadsPerWarp; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto weight = [&](int w) {
+    return (live(w) && head_ok) ? expf(lse_part[int64_t(b + w) * H + i] - m) * inv_z : 0.f;
+  };
+  for (int w = w_first; w <= w_last; w += 2) {
+    const bool two = w + 1 <= w_last;
+    const float ea = weight(w), eb = two ? weight(w + 1) : 0.f;
+    const float4* sa = src0 + int64_t(b + w) * slot_stride;
+    const float4* sb = src0 + int64_t(b + (two ? w + 1 : w)) * slot_stride;
+    float4 va[kQuadsPerWarp], vb[kQuadsPerWarp];
 #pragma unroll
-    for (int q = 0; q < kMaxDcPerLane / 4; ++q) {
-      const int c = (q * 32 + lane) * 4;
-      if (c < d_c) {
-        const float4 va = ea != 0.f ? *reinterpret_cast<const float4*>(sa + c)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 vb = eb != 0.f ? *reinterpret_cast<const float4*>(sb + c)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-        acc[q][0] = fmaf(ea, va.x, fmaf(eb, vb.x, acc[q][0]));
-        acc[q][1] = fmaf(ea, va.y, fmaf(eb, vb.y, acc[q][1]));
-        acc[q][2] = fmaf(ea, va.z, fmaf(eb, vb.z, acc[q][2]));
-        acc[q][3] = fmaf(ea, va.w, fmaf(eb, vb.w, acc[q][3]));
-      }
+    for (int j = 0; j < kQuadsPerWarp; ++j) {
+      const bool in = head_ok && warp + kCombineWarps * j < nqb;
+      va[j] = (in && ea != 0.f) ? sa[int64_t(kCombineWarps * j) * H] : make_float4(0.f, 0.f, 0.f, 0.f);
+      vb[j] = (in && eb != 0.f) ? sb[int64_t(kCombineWarps * j) * H] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < kQuadsPerWarp; ++j) {
+      acc[j].x = fmaf(ea, va[j].x, fmaf(eb, vb[j].x, acc[j].x));
+      acc[j].y = fmaf(ea, va[j].y, fmaf(eb, vb[j].y, acc[j].y));
+      acc[j].z = fmaf(ea, va[j].z, fmaf(eb, vb[j].z, acc[j].z));
+      acc[j].w = fmaf(ea, va[j].w, fmaf(eb, vb[j].w, acc[j].w));
     }
   }
 #pragma unroll
-  for (int q = 0; q < kMaxDcPerLane / 4; ++q) {
-    const int c = (q * 32 + lane) * 4;
-    if (c < d_c)
-      *reinterpret_cast<float4*>(dst + c) = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+  for (int j = 0; j < kQuadsPerWarp; ++j) s_rows[lane][warp + kCombineWarps * j] = acc[j];
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < nh * nqb; idx += kCombineThreads) {
+    const int hh = idx / nqb, q = idx % nqb;
+    reinterpret_cast<float4*>(o_lat + (int64_t(b) * H + h0 + hh) * d_c)[q_base + q] = s_rows[hh][q];
   }
-  if (lane == 0 && lse_out) lse_out[int64_t(b) * H + i] = m + logf(z);
+  if (blockIdx.z == 0 && warp == 0 && head_ok && lse_out) lse_out[int64_t(b) * H + i] = m + logf(z);
 }
 
 }  // namespace
@@ -138,7 +129,8 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
 cudaError_t launch_combine(const int32_t* seqlens, int64_t cap, int B, int H, int d_c, int W,
                            const float* o_part, const float* lse_part, float* o_lat,
                            float* lse, cudaStream_t stream) {
-  dim3 grid(B, (H + kCombineWarps - 1) / kCombineWarps);
+  const int nq = d_c / 4;
+  dim3 grid(B, (H + kCombineHeads - 1) / kCombineHeads, (nq + kQuadsPerBlock - 1) / kQuadsPerBlock);
   combine_kernel<<<grid, kCombineThreads, 0, stream>>>(seqlens, cap, B, H, d_c, W, o_part,
                                                        lse_part, o_lat, lse);
   return cudaGetLastError();

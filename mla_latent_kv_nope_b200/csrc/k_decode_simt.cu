@@ -109,11 +109,12 @@ decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache,
       if (head < H) {
         const int slot = b + w;
         const float inv_l = 1.f / l;
-        float* o = o_part + (int64_t(slot) * H + head) * d_c;
+        // Partials are o_part[slot][d_c / 4][H][4].
+        float* o = o_part + int64_t(slot) * d_c * H + int64_t(head) * 4;
 #pragma unroll
         for (int k = 0; k < kMaxAccPerLane; ++k) {
           const int c = lane + 32 * k;
-          if (c < d_c) o[c] = acc[k] * inv_l;
+          if (c < d_c) o[int64_t(c >> 2) * H * 4 + (c & 3)] = acc[k] * inv_l;
         }
         if (lane == 0) lse_part[int64_t(slot) * H + head] = m + logf(l);
       }

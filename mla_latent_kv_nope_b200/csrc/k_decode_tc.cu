@@ -29,9 +29,9 @@
 // All tensor-memory traffic of the softmax warps uses 16-lane accesses, so
 // each row is shared by two threads (keys 0-31 / 32-63 of S; columns
 // 0-255 / 256-511 of O) and the other lane half is never touched.
-// Every wait is bounded (2 s); on give-up the CTA raises a shared abort flag,
-// records MLA_ERR_DEVICE_TIMEOUT, drains its own loads and MMAs, frees TMEM
-// and exits.
+// Every wait is bounded (about 2 s of SM cycles); on give-up the CTA raises
+// a shared abort flag, records MLA_ERR_DEVICE_TIMEOUT, drains its own loads
+// and MMAs, frees TMEM and exits.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -61,7 +61,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;                         // lo lanes, 2 x 64 columns
 constexpr uint32_t kColQ = 128;                       // lo lanes, 288 columns
 constexpr uint32_t kHiLanes = 16u << 16;              // lane offset of the hi half
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.f;  // log2 units: rescale when the max grows by > 2^8
 constexpr int kPrefetchTiles = 4;         // tiles brought into L2 ahead of their load
 
@@ -86,6 +85,7 @@ constexpr size_t kOffStage = 0;
 constexpr size_t kOffBar = size_t(kStages) * kStageBytes;
 constexpr size_t kOffPrefix = kOffBar + ((sizeof(Barriers) + 15) / 16) * 16;
 constexpr size_t kSmemBytes = kOffPrefix + sizeof(int32_t) * (kMaxSeqSmem + 1) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA");
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256, false, true);
@@ -95,16 +95,17 @@ __device__ __forceinline__ void raise_abort(Barriers* bars, int* status) {
   record_status(status, MLA_ERR_DEVICE_TIMEOUT);
 }
 
-// Warp-uniform bounded wait (all 32 lanes poll; lane 0 owns the time limit).
+// Warp-uniform bounded wait (all 32 lanes poll; lane 0 owns the limit).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const uint64_t t0 = global_timer_ns();
+  if (__all_sync(0xffffffffu, mbar_try(bar, parity))) return true;
+  const uint64_t t0 = sm_cycles();
   for (uint32_t it = 0;; ++it) {
     const bool ok = mbar_try(bar, parity);
     if (__all_sync(0xffffffffu, ok)) return true;
     if ((it & 63) == 63) {
       int give_up = 0;
       if ((threadIdx.x & 31) == 0)
-        give_up = (*abort_flag != 0) || (global_timer_ns() - t0 > kWaitLimitNs);
+        give_up = (*abort_flag != 0) || (sm_cycles() - t0 > kWaitLimitCycles);
       if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
     }
   }
@@ -256,7 +257,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
           const int s = i % kStages;
           if (g == 0 && t + kPrefetchTiles < hi) prefetch(t + kPrefetchTiles);
           if (i >= kStages && !(ok = mbar_wait(&bars->empty[s], ((i / kStages) - 1) & 1,
-                                               abort_flag, kWaitLimitNs)))
+                                               abort_flag, kWaitLimitCycles)))
             return false;
           mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
           const int32_t crow = int32_t(row0 + t * kTileKeys);
@@ -272,7 +273,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
         // each stage (bounded, ignoring the flag).
         volatile int no_abort = 0;
         for (uint32_t k = (i > kStages ? i - kStages : 0); k < i; ++k)
-          mbar_wait(&bars->full[k % kStages], (k / kStages) & 1, &no_abort, kWaitLimitNs);
+          mbar_wait(&bars->full[k % kStages], (k / kStages) & 1, &no_abort, kWaitLimitCycles);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -289,38 +290,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
       // The softmax warps have written this sequence's query block.
       if (!(ok = warp_wait(&bars->q_ready, seg & 1, abort_flag))) return false;
       tc_fence_after();
-      uint64_t t_last = global_timer_ns();
+      uint64_t t_last = sm_cycles();
       uint32_t spins = 0;
       while (i_pv < end) {
         bool progressed = false;
-        if (i_qk < end && i_qk <= i_pv + 1) {
-          const int st = i_qk % kStages, sb = i_qk & 1;
-          int ready = 0;
-          if (lane == 0)
-            ready = mbar_test(&bars->full[st], (i_qk / kStages) & 1) &&
-                    (i_qk < 2 || mbar_test(&bars->s_free[sb], ((i_qk >> 1) - 1) & 1));
-          if (__shfl_sync(0xffffffffu, ready, 0)) {
-            tc_fence_after();
-            const uint32_t d = tmem + kColS + uint32_t(sb) * 64u;
-            // Descriptor and TMEM address bases are formed once; each of the
-            // 36 MMAs then only adds a compile-time offset (the start address
-            // field is the low 14 bits: shared-memory offsets >> 4).
-            const uint64_t b0 = smem_desc_sw128(st_base + uint32_t(st) * kStageBytes, 16, 1024);
-            const uint32_t a0 = tmem + kColQ;
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ts_w(d, a0 + uint32_t(c * 4 + k) * 8u,
-                              b0 + uint64_t((c * kChunkBytes + k * 32) >> 4), kIdescQK,
-                              (c | k) != 0);
-            }
-            mma_commit_w(&bars->s_full[sb]);
-            ++i_qk;
-            progressed = true;
-          }
-        }
-        if (!progressed && i_pv < i_qk) {
+        // P.C of a tile whose probabilities are ready goes first: it ends the
+        // tile's hold on its stage, so the next load can start.
+        if (i_pv < i_qk) {
           const int st = i_pv % kStages, sb = i_pv & 1;
           const bool first = (i_pv == base);
           int ready = 0;
@@ -347,12 +323,41 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
             progressed = true;
           }
         }
+        // QK^T of the next tile (all 36 MMAs) once its stage has landed and
+        // its S buffer has been read.
+        if (!progressed && i_qk < end && i_qk <= i_pv + 1) {
+          const int st = i_qk % kStages, sb = i_qk & 1;
+          int ready = 0;
+          if (lane == 0)
+            ready = mbar_test(&bars->full[st], (i_qk / kStages) & 1) &&
+                    (i_qk < 2 || mbar_test(&bars->s_free[sb], ((i_qk >> 1) - 1) & 1));
+          if (__shfl_sync(0xffffffffu, ready, 0)) {
+            tc_fence_after();
+            const uint32_t d = tmem + kColS + uint32_t(sb) * 64u;
+            // Descriptor and TMEM address bases are formed once; each of the
+            // 36 MMAs then only adds a compile-time offset (the start address
+            // field is the low 14 bits: shared-memory offsets >> 4).
+            const uint64_t b0 = smem_desc_sw128(st_base + uint32_t(st) * kStageBytes, 16, 1024);
+            const uint32_t a0 = tmem + kColQ;
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma_bf16_ts_w(d, a0 + uint32_t(c * 4 + k) * 8u,
+                              b0 + uint64_t((c * kChunkBytes + k * 32) >> 4), kIdescQK,
+                              (c | k) != 0);
+            }
+            mma_commit_w(&bars->s_full[sb]);
+            ++i_qk;
+            progressed = true;
+          }
+        }
         if (progressed) {
           spins = 0;
-          t_last = global_timer_ns();
+          t_last = sm_cycles();
         } else if ((++spins & 255) == 0) {
           int give_up = 0;
-          if (lane == 0) give_up = *abort_flag || global_timer_ns() - t_last > kWaitLimitNs;
+          if (lane == 0) give_up = *abort_flag || sm_cycles() - t_last > kWaitLimitCycles;
           if (__shfl_sync(0xffffffffu, give_up, 0)) {
             ok = false;
             return false;
@@ -538,7 +543,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
       tc_fence_after();
       const float l_row = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
       const float inv = 1.f / l_row;
-      float* dst = o_part + (int64_t(slot) * H + head) * kDc + (lo_half ? 0 : 256);
+      // Partials are o_part[slot][d_c / 4][H][4]: lanes 0-15 store 16
+      // consecutive heads of one 4-column group (256 contiguous bytes), lanes
+      // 16-31 the same heads 64 groups further on.
+      float* dst = o_part + ((int64_t(slot) * (kDc / 4) + (lo_half ? 0 : 64)) * H + head) * 4;
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
         uint32_t r[32];
@@ -546,10 +554,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
         tmem_wait_ld();
         if (head < H) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + c + e) =
-                make_float4(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv,
-                            __uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<float4*>(dst + int64_t(c / 4 + e) * H * 4) =
+                make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                            __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
         }
       }
       if (lo_half && head < H)
@@ -569,12 +577,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
   }
 }
 
+}  // namespace
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_tiled() {
+static EncodeTiledFn encode_tiled() {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -588,8 +598,7 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// 2D bf16 map over a row-major [rows, 576] matrix, 64 x 64 boxes, 128B swizzle.
-bool make_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
+bool make_cache_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cuuint64_t(kR), cuuint64_t(rows)};
@@ -601,8 +610,6 @@ bool make_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
 int decode_tc_head_groups(int H) { return (H + kHeadsPerCta - 1) / kHeadsPerCta; }
 
 cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* cache,
@@ -612,7 +619,7 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
   if (int64_t(B) * cap >= (int64_t(1) << 31) || int64_t(B) * H >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
   CUtensorMap tm_c;
-  if (!make_rows_map(&tm_c, cache, uint64_t(B) * uint64_t(cap))) return cudaErrorInvalidValue;
+  if (!make_cache_rows_map(&tm_c, cache, uint64_t(B) * uint64_t(cap))) return cudaErrorInvalidValue;
   static bool attr_done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;

@@ -30,7 +30,6 @@ using namespace sm100;
 
 constexpr int kThreadsG = 128;
 constexpr int kChunk = 64;                  // bf16 elements per 128-byte row
-constexpr uint64_t kLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -39,7 +38,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // Block-wide bounded wait on an mbarrier (every thread polls).
 __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity) {
   volatile int no_abort = 0;
-  return mbar_wait(bar, parity, &no_abort, kLimitNs);
+  return mbar_wait(bar, parity, &no_abort, kWaitLimitCycles);
 }
 
 // Store bf16 pairs of row `r` (64 elements = 8 16-byte units) into a K-major

@@ -1,6 +1,7 @@
 // Internal launch functions (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -27,6 +28,10 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
                              int W, float* o_part, float* lse_part, int* status,
                              cudaStream_t stream);
 int decode_tc_head_groups(int H);
+// 2D TMA map over the cache viewed as [rows, 576] bf16: 64 x 64 boxes, 128-byte
+// swizzle.  False if the driver entry point is missing or encoding fails.
+bool make_cache_rows_map(CUtensorMap* map, const void* base, uint64_t rows);
+
 
 cudaError_t launch_combine(const int32_t* seqlens, int64_t cap, int B, int H, int d_c, int W,
                            const float* o_part, const float* lse_part, float* o_lat,

@@ -58,6 +58,19 @@ int check_dims(const mla_dims* d) {
 
 inline bool decode_uses_tc(const mla_dims* d) { return d->dtype == MLA_BF16; }
 
+cudaError_t launch_decode_any(const mla_dims* d, const void* q_cat, const void* cache,
+                              const int32_t* seqlens, float scale, int W, float* o_part,
+                              float* lse_part, int* status, cudaStream_t s) {
+  if (decode_uses_tc(d))
+    return launch_decode_tc(static_cast<const __nv_bfloat16*>(q_cat),
+                            static_cast<const __nv_bfloat16*>(cache), seqlens, d->B, d->H,
+                            d->cache_capacity, scale, W, o_part, lse_part, status, s);
+  return launch_decode_simt<float>(static_cast<const float*>(q_cat),
+                                   static_cast<const float*>(cache), seqlens, d->B, d->H, d->d_c,
+                                   d->d_r, d->cache_capacity, scale, W, o_part, lse_part, status,
+                                   s);
+}
+
 int decode_shape_supported(const mla_dims* d) {
   if (d->dtype == MLA_BF16 && (d->d_c != 512 || d->d_r != 64)) return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
@@ -236,16 +249,8 @@ int mla_decode(const mla_dims* d, const void* q_cat, const void* cache, const in
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + l.o_off);
   float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + l.lse_off);
-  if (d->dtype == MLA_BF16)
-    return cuda_status(launch_decode_tc(static_cast<const __nv_bfloat16*>(q_cat),
-                                        static_cast<const __nv_bfloat16*>(cache), seqlens, d->B,
-                                        d->H, d->cache_capacity, softmax_scale, W, o_part,
-                                        lse_part, status_ptr(), s));
-  return cuda_status(launch_decode_simt<float>(static_cast<const float*>(q_cat),
-                                               static_cast<const float*>(cache), seqlens, d->B,
-                                               d->H, d->d_c, d->d_r, d->cache_capacity,
-                                               softmax_scale, W, o_part, lse_part, status_ptr(),
-                                               s));
+  return cuda_status(launch_decode_any(d, q_cat, cache, seqlens, softmax_scale, W, o_part,
+                                       lse_part, status_ptr(), s));
 }
 
 // ---------------------------------------------------------------------------
@@ -345,16 +350,8 @@ extern "C" int mla_decode_noalloc(const mla_dims* d, const void* q_cat, const vo
   float* o_part = reinterpret_cast<float*>(static_cast<char*>(scratch) + l.o_off);
   float* lse_part = reinterpret_cast<float*>(static_cast<char*>(scratch) + l.lse_off);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  if (d->dtype == MLA_BF16)
-    e = launch_decode_tc(static_cast<const __nv_bfloat16*>(q_cat),
-                         static_cast<const __nv_bfloat16*>(cache), seqlens, d->B, d->H,
-                         d->cache_capacity, softmax_scale, W, o_part, lse_part, status_ptr(), s);
-  else
-    e = launch_decode_simt<float>(static_cast<const float*>(q_cat),
-                                  static_cast<const float*>(cache), seqlens, d->B, d->H, d->d_c,
-                                  d->d_r, d->cache_capacity, softmax_scale, W, o_part, lse_part,
-                                  status_ptr(), s);
+  const cudaError_t e = launch_decode_any(d, q_cat, cache, seqlens, softmax_scale, W, o_part,
+                                          lse_part, status_ptr(), s);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   return cuda_status(launch_combine(seqlens, d->cache_capacity, d->B, d->H, d->d_c, W, o_part,
                                     lse_part, o_lat, lse, s));

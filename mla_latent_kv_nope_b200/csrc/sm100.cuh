@@ -59,17 +59,22 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after `limit_ns` of wall time, or as soon as the
+// SM cycle counter: cheap to read, unlike %globaltimer, so it bounds the
+// waits on hot paths.  2 s at the 1965 MHz boost clock is about 3.9e9 cycles.
+__device__ __forceinline__ uint64_t sm_cycles() { return clock64(); }
+constexpr uint64_t kWaitLimitCycles = 4000000000ull;
+
+// Bounded wait: gives up after `limit_cycles` SM cycles, or as soon as the
 // block-wide abort flag is raised by another role.  Returns false on give-up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag, uint64_t limit_ns) {
+                                          volatile int* abort_flag, uint64_t limit_cycles) {
   if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  const uint64_t t0 = sm_cycles();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > limit_ns) return false;
+      if (sm_cycles() - t0 > limit_cycles) return false;
     }
   }
 }

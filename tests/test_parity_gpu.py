@@ -166,6 +166,13 @@ DECODE_CASES = [
     ("bf16-H128-W7", W["v3_bf16"].scaled(B=3, N=600), [600, 129, 1], 7, 1.0),
     ("bf16-H128-peaked", W["v3_bf16"].scaled(B=2, N=400), [400, 77], 0, 10.0),
     ("bf16-H16-peaked", SMALL_BF16.scaled(B=2), [190, 64], 0, 10.0),
+    # more than 64 heads: CTA pairs, 128 heads per pair
+    ("bf16-H128-edges", W["v3_bf16"].scaled(B=8, N=200), [1, 63, 64, 65, 127, 128, 200, 0], 0, 1.0),
+    ("bf16-H128-W1", W["v3_bf16"].scaled(B=3, N=300), [300, 1, 100], 1, 1.0),
+    ("bf16-H128-Wbig", W["v3_bf16"].scaled(B=2, N=2000), [2000, 3], 300, 1.0),
+    ("bf16-H128-peaked-long", W["v3_bf16"].scaled(B=1, N=3000), [3000], 2, 10.0),
+    ("bf16-H100", W["v3_bf16"].scaled(B=3, H=100, N=300), [300, 65, 0], 0, 1.0),
+    ("bf16-H192", W["v3_bf16"].scaled(B=2, H=192, N=200), [200, 64], 0, 1.0),
 ]
 
 
@@ -195,7 +202,9 @@ def test_combine_alone():
     slots = B + Wn - 1
     o_all, l_all = inputs.partials(1, H, slots, d_c, seed=3, empty_frac=0.0)
     ws = torch.full((mla.decode_workspace_bytes(d, Wn) // 4,), float("nan"), device="cuda")
-    ws[:slots * H * d_c] = torch.from_numpy(o_all[0].transpose(1, 0, 2).reshape(-1)).cuda()
+    # documented partial layout: o_part[slot][d_c / 4][H][4]
+    o_ws = o_all[0].reshape(H, slots, d_c // 4, 4).transpose(1, 2, 0, 3)
+    ws[:slots * H * d_c] = torch.from_numpy(np.ascontiguousarray(o_ws).reshape(-1)).cuda()
     lse_off = ((slots * H * d_c * 4 + 255) // 256 * 256) // 4
     ws[lse_off:lse_off + slots * H] = torch.from_numpy(l_all[0].T.reshape(-1)).cuda()
     o_lat = torch.empty(B, H, d_c, device="cuda")
