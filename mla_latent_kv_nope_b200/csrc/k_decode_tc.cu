@@ -15,10 +15,13 @@
 //   warp 4      TMA producer: per 64-key tile, 9 boxes of [64 keys x 64 dims]
 //               bf16 with 128-byte swizzle into a 3-stage ring, plus an L2
 //               prefetch a few tiles ahead.
-//   warp 5      MMA issuer (one thread): S = Q C^T with Q read from tensor
-//               memory (only the cache tile is fetched from shared memory),
-//               O += P C with P and C from shared memory.  QK^T of tile i+1 is
-//               issued while the softmax of tile i runs.
+//   warp 5      QK^T issuer: S = Q C^T with Q read from tensor memory (only
+//               the cache tile is fetched from shared memory); it runs ahead
+//               as far as the stages and the two S buffers allow.
+//   warp 6      P.C issuer: O += P C with P and C from shared memory, as soon
+//               as a tile's probabilities are written.  Two issuing warps keep
+//               a ready P.C from waiting behind a queued QK^T (a warp's next
+//               barrier poll waits for its own MMAs to be taken up).
 //   warps 0-3   softmax, correction and epilogue.  At each sequence start
 //               they write the 64 x 576 query block into tensor memory.
 // Tensor memory (an M = 64 tile occupies 16 of the 32 lanes of each
@@ -55,8 +58,9 @@ constexpr int kStageBytes = kChunks * kChunkBytes;    // 73728
 constexpr int kStages = 3;
 constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);    // 192
+constexpr int kMmaWarp = 5;                           // QK^T; owns the TMEM allocation
+constexpr int kPvWarp = 6;                            // P.C
+constexpr int kThreads = 32 * (kSoftmaxWarps + 3);    // 224
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;                         // lo lanes, 2 x 64 columns
 constexpr uint32_t kColQ = 128;                       // lo lanes, 288 columns
@@ -71,7 +75,7 @@ struct Barriers {
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2];
   uint64_t o_free;
-  uint64_t mma_drain;
+  uint64_t mma_drain, pv_drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -222,6 +226,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     }
     mbar_init(&bars->o_free, 32 * kSoftmaxWarps);
     mbar_init(&bars->mma_drain, 1);
+    mbar_init(&bars->pv_drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -277,92 +282,37 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs the scheduler (decisions are lane 0's, broadcast)
-    // and elect.sync issues each instruction from one lane.
-    uint32_t i_qk = 0, i_pv = 0;
+    // ------------------------------------------------------------ QK^T issuer
+    // The whole warp waits (all lanes poll) and elect.sync issues each
+    // instruction from one lane.
+    uint32_t i = 0;
     int seg = 0;
     bool ok = true;
     const uint32_t st_base = smem_u32(sStage);
-    for_each_segment(tp, t_begin, t_end,
-                     [&](int, int64_t lo, int64_t hi, int64_t) {
-      const uint32_t base = i_pv, end = i_pv + uint32_t(hi - lo);
+    for_each_segment(tp, t_begin, t_end, [&](int, int64_t lo, int64_t hi, int64_t) {
       // The softmax warps have written this sequence's query block.
       if (!(ok = warp_wait(&bars->q_ready, seg & 1, abort_flag))) return false;
-      tc_fence_after();
-      uint64_t t_last = sm_cycles();
-      uint32_t spins = 0;
-      while (i_pv < end) {
-        bool progressed = false;
-        // P.C of a tile whose probabilities are ready goes first: it ends the
-        // tile's hold on its stage, so the next load can start.
-        if (i_pv < i_qk) {
-          const int st = i_pv % kStages, sb = i_pv & 1;
-          const bool first = (i_pv == base);
-          int ready = 0;
-          if (lane == 0)
-            ready = mbar_test(&bars->p_full[sb], (i_pv >> 1) & 1) &&
-                    (!first || seg == 0 || mbar_test(&bars->o_free, (seg - 1) & 1));
-          if (__shfl_sync(0xffffffffu, ready, 0)) {
-            tc_fence_after();
-            const uint32_t stage = st_base + uint32_t(st) * kStageBytes;
-            const uint64_t a0 = smem_desc_sw128(stage + kRopeChunk * kChunkBytes, 16, 1024);
-            const uint64_t b0 = smem_desc_sw128(stage, kChunkBytes, 1024);
-            // The two output halves are independent accumulators: alternate
-            // them so consecutive MMAs do not depend on each other.
+      for (int64_t t = lo; t < hi; ++t, ++i) {
+        const int st = i % kStages, sb = i & 1;
+        if (!(ok = warp_wait(&bars->full[st], (i / kStages) & 1, abort_flag))) return false;
+        if (i >= 2 && !(ok = warp_wait(&bars->s_free[sb], ((i >> 1) - 1) & 1, abort_flag)))
+          return false;
+        tc_fence_after();
+        const uint32_t d = tmem + kColS + uint32_t(sb) * 64u;
+        // Descriptor and TMEM address bases are formed once; each of the 36
+        // MMAs then only adds a compile-time offset (the start address field
+        // is the low 14 bits: shared-memory offsets >> 4).
+        const uint64_t b0 = smem_desc_sw128(st_base + uint32_t(st) * kStageBytes, 16, 1024);
+        const uint32_t a0 = tmem + kColQ;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+        for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
-              for (int h = 0; h < 2; ++h)
-                mma_bf16_ss_w(tmem + kHiLanes + uint32_t(h) * 256u, a0 + uint64_t((k * 32) >> 4),
-                              b0 + uint64_t((4 * h * kChunkBytes + k * 2048) >> 4), kIdescPV,
-                              !(first && k == 0));
-            }
-            mma_commit_w(&bars->empty[st]);
-            ++i_pv;
-            progressed = true;
-          }
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ts_w(d, a0 + uint32_t(c * 4 + k) * 8u,
+                          b0 + uint64_t((c * kChunkBytes + k * 32) >> 4), kIdescQK,
+                          (c | k) != 0);
         }
-        // QK^T of the next tile (all 36 MMAs) once its stage has landed and
-        // its S buffer has been read.
-        if (!progressed && i_qk < end && i_qk <= i_pv + 1) {
-          const int st = i_qk % kStages, sb = i_qk & 1;
-          int ready = 0;
-          if (lane == 0)
-            ready = mbar_test(&bars->full[st], (i_qk / kStages) & 1) &&
-                    (i_qk < 2 || mbar_test(&bars->s_free[sb], ((i_qk >> 1) - 1) & 1));
-          if (__shfl_sync(0xffffffffu, ready, 0)) {
-            tc_fence_after();
-            const uint32_t d = tmem + kColS + uint32_t(sb) * 64u;
-            // Descriptor and TMEM address bases are formed once; each of the
-            // 36 MMAs then only adds a compile-time offset (the start address
-            // field is the low 14 bits: shared-memory offsets >> 4).
-            const uint64_t b0 = smem_desc_sw128(st_base + uint32_t(st) * kStageBytes, 16, 1024);
-            const uint32_t a0 = tmem + kColQ;
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_bf16_ts_w(d, a0 + uint32_t(c * 4 + k) * 8u,
-                              b0 + uint64_t((c * kChunkBytes + k * 32) >> 4), kIdescQK,
-                              (c | k) != 0);
-            }
-            mma_commit_w(&bars->s_full[sb]);
-            ++i_qk;
-            progressed = true;
-          }
-        }
-        if (progressed) {
-          spins = 0;
-          t_last = sm_cycles();
-        } else if ((++spins & 255) == 0) {
-          int give_up = 0;
-          if (lane == 0) give_up = *abort_flag || sm_cycles() - t_last > kWaitLimitCycles;
-          if (__shfl_sync(0xffffffffu, give_up, 0)) {
-            ok = false;
-            return false;
-          }
-        }
+        mma_commit_w(&bars->s_full[sb]);
       }
       ++seg;
       return true;
@@ -372,6 +322,43 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     mma_commit_w(&bars->mma_drain);
     volatile int no_abort = 0;
     warp_wait(&bars->mma_drain, 0, &no_abort);
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ P.C issuer
+    uint32_t i = 0;
+    int seg = 0;
+    bool ok = true;
+    const uint32_t st_base = smem_u32(sStage);
+    for_each_segment(tp, t_begin, t_end, [&](int, int64_t lo, int64_t hi, int64_t) {
+      for (int64_t t = lo; t < hi; ++t, ++i) {
+        const int st = i % kStages, sb = i & 1;
+        const bool first = (t == lo);
+        if (!(ok = warp_wait(&bars->p_full[sb], (i >> 1) & 1, abort_flag))) return false;
+        // The previous sequence's epilogue has read O before it is overwritten.
+        if (first && seg > 0 && !(ok = warp_wait(&bars->o_free, (seg - 1) & 1, abort_flag)))
+          return false;
+        tc_fence_after();
+        const uint32_t stage = st_base + uint32_t(st) * kStageBytes;
+        const uint64_t a0 = smem_desc_sw128(stage + kRopeChunk * kChunkBytes, 16, 1024);
+        const uint64_t b0 = smem_desc_sw128(stage, kChunkBytes, 1024);
+        // The two output halves are independent accumulators: alternate them
+        // so consecutive MMAs do not depend on each other.
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            mma_bf16_ss_w(tmem + kHiLanes + uint32_t(h) * 256u, a0 + uint64_t((k * 32) >> 4),
+                          b0 + uint64_t((4 * h * kChunkBytes + k * 2048) >> 4), kIdescPV,
+                          !(first && k == 0));
+        }
+        mma_commit_w(&bars->empty[st]);
+      }
+      ++seg;
+      return true;
+    });
+    if (!ok && lane == 0) raise_abort(bars, status);
+    mma_commit_w(&bars->pv_drain);
+    volatile int no_abort = 0;
+    warp_wait(&bars->pv_drain, 0, &no_abort);
   } else {
     // ------------------------------------------------------------ softmax
     const int q = warp;                      // TMEM lane quadrant
