@@ -83,12 +83,13 @@ struct Barriers {
 // Exclusive prefix of per-sequence tile counts, built once per CTA so that no
 // role walks the length array through global memory (a chain of dependent
 // loads).  Batches with more sequences fall back to walking global memory.
-constexpr int kMaxSeqSmem = 2048;
+constexpr int kMaxSeqSmem = 1024;
 
 constexpr size_t kOffStage = 0;
 constexpr size_t kOffBar = size_t(kStages) * kStageBytes;
 constexpr size_t kOffPrefix = kOffBar + ((sizeof(Barriers) + 15) / 16) * 16;
-constexpr size_t kSmemBytes = kOffPrefix + sizeof(int32_t) * (kMaxSeqSmem + 1) + 1024;
+constexpr size_t kOffLens = kOffPrefix + sizeof(int32_t) * (kMaxSeqSmem + 1);
+constexpr size_t kSmemBytes = kOffLens + sizeof(int32_t) * kMaxSeqSmem + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA");
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
@@ -119,6 +120,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // shared memory when the batch fits, else recomputed from the lengths.
 struct TilePrefix {
   const int32_t* sp;       // shared prefix [B + 1] or nullptr
+  const int32_t* sl;       // shared clamped lengths [B] or nullptr
   const int32_t* seqlens;
   int B;
   int64_t cap;
@@ -128,7 +130,7 @@ struct TilePrefix {
     for (int k = 0; k < b; ++k) p += tiles_of(clamp_len(seqlens[k], cap));
     return p;
   }
-  __device__ int64_t len(int b) const { return clamp_len(seqlens[b], cap); }
+  __device__ int64_t len(int b) const { return sl ? sl[b] : clamp_len(seqlens[b], cap); }
   // First sequence whose tiles end after tile t (binary search on the prefix).
   __device__ int first_after(int64_t t) const {
     if (!sp) {
@@ -165,7 +167,8 @@ __device__ __forceinline__ void for_each_segment(const TilePrefix& tp, int64_t t
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* __restrict__ q_cat,
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* __restrict__ cache,
+                 const __nv_bfloat16* __restrict__ q_cat,
                  const int32_t* __restrict__ seqlens, int B, int H, int64_t cap,
                  float scale_log2, int W, float* __restrict__ o_part,
                  float* __restrict__ lse_part, int* __restrict__ status) {
@@ -182,11 +185,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
   // Tile prefix of the batch (all threads load lengths in parallel; warp 0
   // scans 32 at a time with shuffles).
   int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + kOffPrefix);
+  int32_t* s_lens = reinterpret_cast<int32_t*>(smem + kOffLens);
   const bool prefix_in_smem = B <= kMaxSeqSmem;
   int64_t n_tiles = 0;
   if (prefix_in_smem) {
-    for (int b = threadIdx.x; b < B; b += kThreads)
-      s_prefix[b + 1] = int32_t(tiles_of(clamp_len(seqlens[b], cap)));
+    for (int b = threadIdx.x; b < B; b += kThreads) {
+      const int64_t L = clamp_len(seqlens[b], cap);
+      s_lens[b] = int32_t(L);
+      s_prefix[b + 1] = int32_t(tiles_of(L));
+    }
     __syncthreads();
     if (warp == 0) {
       int32_t carry = 0;
@@ -207,7 +214,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
   } else {
     for (int b = 0; b < B; ++b) n_tiles += tiles_of(clamp_len(seqlens[b], cap));
   }
-  const TilePrefix tp{prefix_in_smem ? s_prefix : nullptr, seqlens, B, cap};
+  const TilePrefix tp{prefix_in_smem ? s_prefix : nullptr, prefix_in_smem ? s_lens : nullptr,
+                      seqlens, B, cap};
   if (n_tiles == 0) return;
   const int64_t t_begin = worker_tile_begin(w, n_tiles, W);
   const int64_t t_end = worker_tile_begin(w + 1, n_tiles, W);
@@ -249,18 +257,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
       bool ok = true;
       for_each_segment(tp, t_begin, t_end,
                        [&](int b, int64_t lo, int64_t hi, int64_t) {
-        // One CTA per tile range (head group 0) pulls tiles into L2 a few
-        // tiles ahead; the shared-memory loads of every head group hit L2.
+        // One CTA per tile range (head group 0) pulls tiles into L2 ahead of
+        // their loads: a tile's rows are one contiguous range of the cache,
+        // so one bulk prefetch covers it (clamped to this sequence's rows).
         const int64_t row0 = int64_t(b) * cap;
         auto prefetch = [&](int64_t t) {
-          for (int c = 0; c < kChunks; ++c)
-            tma_prefetch_2d(&tm_c, c * kChunkElems, int32_t(row0 + t * kTileKeys));
+          if (g != 0 || t >= hi) return;
+          const int64_t rows = min(int64_t(kTileKeys), cap - t * kTileKeys);
+          bulk_prefetch_l2(cache + (row0 + t * kTileKeys) * kR, uint32_t(rows * kR * 2));
         };
-        if (g == 0)
-          for (int64_t t = lo; t < min(lo + kPrefetchTiles, hi); ++t) prefetch(t);
         for (int64_t t = lo; t < hi; ++t, ++i) {
           const int s = i % kStages;
-          if (g == 0 && t + kPrefetchTiles < hi) prefetch(t + kPrefetchTiles);
           if (i >= kStages && !(ok = mbar_wait(&bars->empty[s], ((i / kStages) - 1) & 1,
                                                abort_flag, kWaitLimitCycles)))
             return false;
@@ -269,6 +276,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
           uint8_t* dst = sStage + s * kStageBytes;
           for (int c = 0; c < kChunks; ++c)
             tma_load_2d(&tm_c, &bars->full[s], dst + c * kChunkBytes, c * kChunkElems, crow);
+          // Loads of the first tiles go out before any prefetch.
+          if (t == lo)
+            for (int64_t u = t + kStages; u < t + kPrefetchTiles; ++u) prefetch(u);
+          prefetch(t + kPrefetchTiles);
         }
         return true;
       });
@@ -379,17 +390,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     auto write_query = [&](int b) {
       const int64_t qrow = int64_t(b) * H + int64_t(g) * kHeadsPerCta + row;
       const bool valid_row = qrow < int64_t(B) * H;
-      const uint4* src = reinterpret_cast<const uint4*>(q_cat + qrow * kR);
+      // All 36 loads are unconditional (a padding row reads row 0 and is
+      // zeroed afterwards) so they are in flight together.
+      const uint4* src = reinterpret_cast<const uint4*>(q_cat + (valid_row ? qrow : 0) * kR);
       uint4 v[36];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {   // four 64-column groups: words [64c + half*32, +32)
-        const int word = (j / 8) * 64 + (lo_half ? 0 : 32) + (j % 8) * 4;
-        v[j] = valid_row ? src[word >> 2] : make_uint4(0, 0, 0, 0);
-      }
+      for (int j = 0; j < 32; ++j)   // four 64-column groups: words [64c + half*32, +32)
+        v[j] = src[((j / 8) * 64 + (lo_half ? 0 : 32) + (j % 8) * 4) >> 2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {    // last 32 columns: words [256 + half*16, +16)
-        const int word = 256 + (lo_half ? 0 : 16) + j * 4;
-        v[32 + j] = valid_row ? src[word >> 2] : make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < 4; ++j)    // last 32 columns: words [256 + half*16, +16)
+        v[32 + j] = src[(256 + (lo_half ? 0 : 16) + j * 4) >> 2];
+      if (!valid_row) {
+#pragma unroll
+        for (int j = 0; j < 36; ++j) v[j] = make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -619,7 +632,7 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
   }
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(decode_tc_head_groups(H), W);
-  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_c, q_cat, seqlens, B, H, cap,
+  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_c, cache, q_cat, seqlens, B, H, cap,
                                                            scale_log2, W, o_part, lse_part,
                                                            status);
   return cudaGetLastError();

@@ -105,12 +105,13 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
       : "memory");
 }
 
-// Hint: bring a 2D tile into L2 ahead of its shared-memory load (no data
-// lands in shared memory and no barrier is signalled).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
+// Hint: bring `bytes` (a multiple of 16) of contiguous global memory into L2
+// ahead of its shared-memory load (no data lands in shared memory and no
+// barrier is signalled).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
                : "memory");
 }
 
