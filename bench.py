@@ -191,16 +191,24 @@ def run_ours(args, rank, world, local_rank):
     if cache_bytes < 2 * L2_BYTES:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
-    def one_step():
+    def eager_step():
         if flush is not None:
             flush.zero_()
-        step.append(hh, cache, seq)
-        mla.absorb_q(dims, q_nope, q_pe, W_UK, q_pos, step.q_cat, step.rope_base)
-        step.splits_used = mla.decode(dims, step.q_cat, cache, seq, step.scale, step.ws,
-                                      step.num_splits)
-        mla.combine(dims, seq, step.ws, step.splits_used, step.o_lat, step.lse)
-        mla.out_proj(dims, step.o_lat, W_UV, step.out)
+        step(q_nope, q_pe, q_pos, cache, seq, h=hh)
         seq.copy_(seq0)
+
+    # A step is replayed from a CUDA graph (one host launch per step) unless
+    # --eager; the graph holds every kernel of the step, each run every replay.
+    for _ in range(2):
+        eager_step()
+    torch.cuda.synchronize()
+    if args.eager:
+        one_step = eager_step
+    else:
+        graph = step.capture(q_nope, q_pe, q_pos, cache, seq, h=hh,
+                             before=(flush.zero_ if flush is not None else None),
+                             after=lambda: seq.copy_(seq0))
+        one_step = graph.replay
 
     # Decode-kernel-only events (for the roofline): separate pass so that
     # the step timing has no extra event records inside it.
@@ -264,16 +272,26 @@ def run_ours(args, rank, world, local_rank):
     bi = sum(t.numel() * t.element_size() for t in (h_qn, h_qp, h_pos, h_h))
     bo = h_out.numel() * h_out.element_size()
 
-    def e2e_step():
+    def e2e_in():
         q_nope.copy_(h_qn, non_blocking=True)
         q_pe.copy_(h_qp, non_blocking=True)
         q_pos.copy_(h_pos, non_blocking=True)
         hh.copy_(h_h, non_blocking=True)
         if flush is not None:
             flush.zero_()
-        step(q_nope, q_pe, q_pos, cache, seq, h=hh)
+
+    def e2e_out():
         h_out.copy_(step.out, non_blocking=True)
         seq.copy_(seq0)
+
+    def e2e_eager():
+        e2e_in()
+        step(q_nope, q_pe, q_pos, cache, seq, h=hh)
+        e2e_out()
+
+    # Host-buffer steps are issued eagerly: with the copies inside a graph
+    # they measured slower on B200 (the copies dominate this path).
+    e2e_step = e2e_eager
 
     for _ in range(3):
         e2e_step()
@@ -330,6 +348,7 @@ def run_ours(args, rank, world, local_rank):
             "l2": ("inputs exceed L2 (cache %.0f MB)" % (cache_bytes / 1e6)) if flush is None
                   else "L2 flushed between steps",
             "num_splits": step.splits_used,
+            "launch": "eager" if args.eager else "cuda_graph (absorb_q on a forked stream)",
         },
         "decode_only": {
             "ms": dec_avg, "ms_with_combine": decomb_avg,
@@ -453,6 +472,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch each kernel from the host every step instead of a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -226,11 +226,16 @@ def get_device_status(stream=None) -> int:
 class DecodeStep:
     """One MLA decode layer on the device: owns its workspaces (allocated once
     by the caller side through torch) and runs append -> absorb_q -> decode ->
-    combine -> out_proj on the current stream.  All arithmetic is in the CUDA
-    kernels; this class only keeps buffers and pointers."""
+    combine -> out_proj.  All arithmetic is in the CUDA kernels; this class
+    only keeps buffers, pointers and the stream order.
+
+    absorb_q does not depend on the cache append, so with ``overlap`` it runs
+    on a second stream forked from the current one and joined before decode.
+    ``capture`` records one step (plus any caller work) into a CUDA graph so a
+    step is replayed with one launch from the host."""
 
     def __init__(self, dims: Dims, W_UK, W_UV, W_DKV=None, gamma=None, softmax_scale=None,
-                 rope_base=10000.0, eps=1e-6, num_splits=0, device="cuda"):
+                 rope_base=10000.0, eps=1e-6, num_splits=0, device="cuda", overlap=True):
         self.dims = dims
         self.W_UK, self.W_UV, self.W_DKV, self.gamma = W_UK, W_UV, W_DKV, gamma
         self.scale = (softmax_scale if softmax_scale is not None
@@ -248,20 +253,51 @@ class DecodeStep:
         self.lse = torch.empty(dims.B, dims.H, dtype=torch.float32, device=device)
         self.out = torch.empty(dims.B, dims.H, dims.d_v, dtype=dt, device=device)
         self.splits_used = self.num_splits
+        self._side = torch.cuda.Stream(device=device) if overlap else None
 
     def append(self, h, cache, seqlens):
         cache_append(self.dims, h, self.W_DKV, self.gamma, cache, seqlens, self.ws_append,
                      self.eps, self.rope_base)
 
-    def attend(self, q_nope, q_pe, q_pos, cache, seqlens):
+    def _absorb(self, q_nope, q_pe, q_pos):
         absorb_q(self.dims, q_nope, q_pe, self.W_UK, q_pos, self.q_cat, self.rope_base)
+
+    def _attend_latent(self, cache, seqlens):
         self.splits_used = decode(self.dims, self.q_cat, cache, seqlens, self.scale, self.ws,
                                   self.num_splits)
         combine(self.dims, seqlens, self.ws, self.splits_used, self.o_lat, self.lse)
         out_proj(self.dims, self.o_lat, self.W_UV, self.out)
         return self.out
 
+    def attend(self, q_nope, q_pe, q_pos, cache, seqlens):
+        self._absorb(q_nope, q_pe, q_pos)
+        return self._attend_latent(cache, seqlens)
+
     def __call__(self, q_nope, q_pe, q_pos, cache, seqlens, h=None):
+        if self._side is None:
+            if h is not None:
+                self.append(h, cache, seqlens)
+            return self.attend(q_nope, q_pe, q_pos, cache, seqlens)
+        main = torch.cuda.current_stream()
+        # Fork: the side stream starts after everything issued so far (the
+        # previous step's decode has finished reading q_cat).
+        self._side.wait_stream(main)
+        with torch.cuda.stream(self._side):
+            self._absorb(q_nope, q_pe, q_pos)
         if h is not None:
             self.append(h, cache, seqlens)
-        return self.attend(q_nope, q_pe, q_pos, cache, seqlens)
+        main.wait_stream(self._side)
+        return self._attend_latent(cache, seqlens)
+
+    def capture(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, before=None, after=None):
+        """Record one step into a CUDA graph; ``before``/``after`` are optional
+        callables whose device work is recorded around it.  Replay with
+        ``graph.replay()``; inputs are read from the same tensors each time."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if before is not None:
+                before()
+            self(q_nope, q_pe, q_pos, cache, seqlens, h=h)
+            if after is not None:
+                after()
+        return g

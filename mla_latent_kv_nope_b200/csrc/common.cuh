@@ -74,15 +74,20 @@ __device__ __forceinline__ int64_t worker_of_tile(int64_t t, int64_t T, int64_t 
 // double and theta is reduced to [-pi, pi] in double (Cody-Waite style with a
 // two-part 2*pi), so the single-precision sincos only ever sees a small,
 // exact-enough argument even at positions ~1e5.
-__device__ __forceinline__ void rope_cos_sin(int64_t pos, int k, int d, float base,
-                                             float* c, float* s) {
-  const double inv = exp2(-2.0 * double(k) / double(d) * log2(double(base)));
+__device__ __forceinline__ double rope_inv_freq(int k, int d, float base) {
+  return exp2(-2.0 * double(k) / double(d) * log2(double(base)));
+}
+__device__ __forceinline__ void rope_cos_sin_at(int64_t pos, double inv, float* c, float* s) {
   const double th = double(pos) * inv;
   const double kTwoPiHi = 6.283185307179586232;      // 2*pi rounded to double
   const double kTwoPiLo = 2.4492935982947064e-16;    // 2*pi - kTwoPiHi
   const double n = rint(th * 0.15915494309189535);   // th / (2*pi)
   const double r = fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, th));
   sincosf(float(r), s, c);
+}
+__device__ __forceinline__ void rope_cos_sin(int64_t pos, int k, int d, float base,
+                                             float* c, float* s) {
+  rope_cos_sin_at(pos, rope_inv_freq(k, d, base), c, s);
 }
 
 }  // namespace mla

@@ -20,6 +20,7 @@ namespace {
 constexpr int kApRows = 4;
 constexpr int kApBatch = 16;
 constexpr int kApThreads = 256;
+constexpr int kFinBatch = 16;       // partial sums loaded together in the finalize
 
 template <typename T>
 __global__ void __launch_bounds__(kApThreads)
@@ -69,7 +70,7 @@ append_project_kernel(const T* __restrict__ h, const T* __restrict__ W, int B, i
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kApThreads)
+__global__ void __launch_bounds__(1024)
 append_finalize_kernel(const float* __restrict__ part, int n_parts,
                        const float* __restrict__ gamma, float eps, float rope_base, int d_c,
                        int d_r, int64_t cap, T* __restrict__ cache,
@@ -78,30 +79,29 @@ append_finalize_kernel(const float* __restrict__ part, int n_parts,
   const int B = gridDim.x;
   const int R = d_c + d_r;
   extern __shared__ float s_x[];  // [R]: the projection, summed over parts in order
-  __shared__ float s_part[kApThreads / 32];
+  __shared__ float s_part[32];
   __shared__ int32_t s_L;
   if (threadIdx.x == 0) s_L = seqlens[b];
-  // Sum the partials in a fixed order (deterministic); 4 loads in flight.
-  for (int c = threadIdx.x; c < R; c += kApThreads) {
+  // Sum the partials in a fixed order (deterministic) with up to
+  // kFinBatch loads in flight per thread; one column per thread when the
+  // block covers the row.
+  for (int c = threadIdx.x; c < R; c += blockDim.x) {
     const float* src = part + int64_t(b) * R + c;
     const int64_t stride = int64_t(B) * R;
     float v = 0.f;
-    int p = 0;
-    for (; p + 4 <= n_parts; p += 4) {
-      const float a0 = src[(p + 0) * stride], a1 = src[(p + 1) * stride];
-      const float a2 = src[(p + 2) * stride], a3 = src[(p + 3) * stride];
-      v += a0;
-      v += a1;
-      v += a2;
-      v += a3;
+    for (int p0 = 0; p0 < n_parts; p0 += kFinBatch) {
+      float x[kFinBatch];
+#pragma unroll
+      for (int j = 0; j < kFinBatch; ++j) x[j] = p0 + j < n_parts ? src[(p0 + j) * stride] : 0.f;
+#pragma unroll
+      for (int j = 0; j < kFinBatch; ++j) v += x[j];
     }
-    for (; p < n_parts; ++p) v += src[p * stride];
     s_x[c] = v;
   }
   __syncthreads();
   const float* xb = s_x;
   float ss = 0.f;
-  for (int c = threadIdx.x; c < d_c; c += kApThreads) ss = fmaf(xb[c], xb[c], ss);
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) ss = fmaf(xb[c], xb[c], ss);
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
   __syncthreads();
@@ -112,15 +112,15 @@ append_finalize_kernel(const float* __restrict__ part, int n_parts,
   }
   float tot = 0.f;
 #pragma unroll
-  for (int wdx = 0; wdx < kApThreads / 32; ++wdx) tot += s_part[wdx];
+  for (int wdx = 0; wdx < int(blockDim.x / 32); ++wdx) tot += s_part[wdx];
   const float inv = 1.f / sqrtf(tot / float(d_c) + eps);
   T* row = cache + (int64_t(b) * cap + L) * R;
-  for (int c = threadIdx.x; c < d_c; c += kApThreads) {
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
     const float g = gamma ? gamma[c] : 1.f;
     row[c] = Storage<T>::from_f(xb[c] * inv * g);
   }
   const int half = d_r / 2;
-  for (int k = threadIdx.x; k < half; k += kApThreads) {
+  for (int k = threadIdx.x; k < half; k += blockDim.x) {
     float cs, sn;
     rope_cos_sin(L, k, d_r, rope_base, &cs, &sn);
     const float x1 = xb[d_c + k], x2 = xb[d_c + k + half];
@@ -152,7 +152,8 @@ cudaError_t launch_append_finalize(const float* part, int n_parts, const float* 
                                    float rope_base, int B, int d_c, int d_r, int64_t cap,
                                    T* cache, int32_t* seqlens, int* status, cudaStream_t stream) {
   const size_t smem = sizeof(float) * size_t(d_c + d_r);
-  append_finalize_kernel<T><<<B, kApThreads, smem, stream>>>(part, n_parts, gamma, eps, rope_base,
+  const int threads = min(1024, (d_c + d_r + 31) / 32 * 32);
+  append_finalize_kernel<T><<<B, threads, smem, stream>>>(part, n_parts, gamma, eps, rope_base,
                                                              d_c, d_r, cap, cache, seqlens,
                                                              status);
   return cudaGetLastError();

@@ -182,6 +182,10 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
   const int i = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kR = 576;
+  // Rotation frequencies of the 32 RoPE pairs, computed once per CTA while
+  // the weight block loads.
+  __shared__ double s_inv[32];
+  if (threadIdx.x < 32) s_inv[threadIdx.x] = rope_inv_freq(threadIdx.x, 64, rope_base);
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
@@ -267,7 +271,7 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
     float y1 = x1, y2 = x2;
     if (q_pos) {
       float c, s;
-      rope_cos_sin(q_pos[b], k, 64, rope_base, &c, &s);
+      rope_cos_sin_at(q_pos[b], s_inv[k], &c, &s);
       y1 = x1 * c - x2 * s;
       y2 = x1 * s + x2 * c;
     }
