@@ -76,12 +76,12 @@ while True:
     sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
     rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
     print(f"{t:.4f} {sm} {rs}", flush=True)
-    time.sleep(0.005)
+    time.sleep(0.002)
 """
 
 
 class ClockSampler:
-    """SM clock and throttle reasons sampled through NVML every ~5 ms by a
+    """SM clock and throttle reasons sampled through NVML every ~2 ms by a
     separate process; only samples inside the [start, stop] window of the
     timed steps are kept."""
     REASONS = {  # NVML clocks-event-reason bits
@@ -141,7 +141,7 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": self.max_mhz,
                 "sm_min_mhz": sms[0], "samples": len(rows), "reasons": sorted(reasons),
-                "source": "NVML from a separate process, ~5 ms period, timed window only"}
+                "source": "NVML from a separate process, ~2 ms period, timed window only"}
 
 
 # ---------------------------------------------------------------------------

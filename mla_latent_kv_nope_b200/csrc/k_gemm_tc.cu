@@ -263,20 +263,38 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
     tc_fence_after();
   }
   // Decoupled RoPE block: rotate q_pe at q_pos (or copy when q_pos is NULL).
-  for (int u = threadIdx.x; u < B * 32; u += kThreadsG) {
-    const int b = u / 32, k = u % 32;
-    const int64_t row = int64_t(b) * H + i;
-    const float x1 = __bfloat162float(q_pe[row * 64 + k]);
-    const float x2 = __bfloat162float(q_pe[row * 64 + k + 32]);
-    float y1 = x1, y2 = x2;
-    if (q_pos) {
-      float c, s;
-      rope_cos_sin_at(q_pos[b], s_inv[k], &c, &s);
-      y1 = x1 * c - x2 * s;
-      y2 = x1 * s + x2 * c;
+  // Pairs (b, k) are taken 8 per thread with every load issued before the
+  // first rotation, so the pass costs one memory round trip per 8 pairs.
+  constexpr int kRopeBatch = 8;
+  for (int u0 = 0; u0 < B * 32; u0 += kRopeBatch * kThreadsG) {
+    float x1[kRopeBatch], x2[kRopeBatch];
+    int32_t pos[kRopeBatch];
+#pragma unroll
+    for (int j = 0; j < kRopeBatch; ++j) {
+      const int u = u0 + j * kThreadsG + threadIdx.x;
+      const bool in = u < B * 32;
+      const int b = in ? u / 32 : 0, k = u % 32;
+      const int64_t row = int64_t(b) * H + i;
+      x1[j] = __bfloat162float(q_pe[row * 64 + k]);
+      x2[j] = __bfloat162float(q_pe[row * 64 + k + 32]);
+      pos[j] = q_pos ? q_pos[b] : 0;
     }
-    q_cat[row * kR + 512 + k] = __float2bfloat16_rn(y1);
-    q_cat[row * kR + 512 + k + 32] = __float2bfloat16_rn(y2);
+#pragma unroll
+    for (int j = 0; j < kRopeBatch; ++j) {
+      const int u = u0 + j * kThreadsG + threadIdx.x;
+      if (u >= B * 32) continue;
+      const int b = u / 32, k = u % 32;
+      const int64_t row = int64_t(b) * H + i;
+      float y1 = x1[j], y2 = x2[j];
+      if (q_pos) {
+        float c, sn;
+        rope_cos_sin_at(pos[j], s_inv[k], &c, &sn);
+        y1 = x1[j] * c - x2[j] * sn;
+        y2 = x1[j] * sn + x2[j] * c;
+      }
+      q_cat[row * kR + 512 + k] = __float2bfloat16_rn(y1);
+      q_cat[row * kR + 512 + k + 32] = __float2bfloat16_rn(y2);
+    }
   }
   if (!ok && threadIdx.x == 0) record_status(status, MLA_ERR_DEVICE_TIMEOUT);
   tc_fence_before();
