@@ -19,6 +19,7 @@ constexpr int kCombineWarps = 8;
 constexpr int kCombineThreads = 32 * kCombineWarps;
 constexpr int kQuadsPerWarp = 4;     // 4-column groups per warp
 constexpr int kQuadsPerBlock = kCombineWarps * kQuadsPerWarp;   // 128 columns
+constexpr int kFastParts = 4;        // partials merged with all loads in one round
 
 // Block = (sequence b, 32 heads, 128 columns).  The partials are stored as
 // o_part[slot][d_c / 4][H][4], so a warp load of one 4-column group for 32
@@ -28,7 +29,7 @@ constexpr int kQuadsPerBlock = kCombineWarps * kQuadsPerWarp;   // 128 columns
 // columns over the partials, two partials per step (8 loads in flight).  The
 // merged block goes through shared memory so o_lat rows are written with
 // coalesced stores.
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineThreads, 4)
 combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, int d_c, int W,
                const float* __restrict__ o_part, const float* __restrict__ lse_part,
                float* __restrict__ o_lat, float* __restrict__ lse_out) {
@@ -78,40 +79,88 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
   const int w_first = int(worker_of_tile(pre, T, W));
   const int w_last = int(worker_of_tile(pre + nt - 1, T, W));
   auto live = [&](int w) { return worker_tile_begin(w, T, W) != worker_tile_begin(w + 1, T, W); };
-  float m = -INFINITY;
-  for (int w = w_first; w <= w_last; ++w)
-    if (live(w) && head_ok) m = fmaxf(m, lse_part[int64_t(b + w) * H + i]);
-  float z = 0.f;
-  for (int w = w_first; w <= w_last; ++w)
-    if (live(w) && head_ok) z += expf(lse_part[int64_t(b + w) * H + i] - m);
-  const float inv_z = head_ok ? 1.f / z : 0.f;
   // Column groups of this thread: q_base + warp + 8 j, j < 4.
   const float4* src0 = reinterpret_cast<const float4*>(o_part) + int64_t(q_base + warp) * H + i;
   const int64_t slot_stride = int64_t(nq) * H;   // float4 units
   float4 acc[kQuadsPerWarp];
 #pragma unroll
   for (int j = 0; j < kQuadsPerWarp; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-  auto weight = [&](int w) {
-    return (live(w) && head_ok) ? expf(lse_part[int64_t(b + w) * H + i] - m) * inv_z : 0.f;
-  };
-  for (int w = w_first; w <= w_last; w += 2) {
-    const bool two = w + 1 <= w_last;
-    const float ea = weight(w), eb = two ? weight(w + 1) : 0.f;
-    const float4* sa = src0 + int64_t(b + w) * slot_stride;
-    const float4* sb = src0 + int64_t(b + (two ? w + 1 : w)) * slot_stride;
-    float4 va[kQuadsPerWarp], vb[kQuadsPerWarp];
+  const int np = w_last - w_first + 1;
+  float m = -INFINITY, z = 0.f;
+  if (np <= kFastParts) {
+    // Common case (up to 4 partials): their lse values in one round of
+    // loads, then their column groups in two rounds.
+    float lv[kFastParts];
 #pragma unroll
-    for (int j = 0; j < kQuadsPerWarp; ++j) {
-      const bool in = head_ok && warp + kCombineWarps * j < nqb;
-      va[j] = (in && ea != 0.f) ? sa[int64_t(kCombineWarps * j) * H] : make_float4(0.f, 0.f, 0.f, 0.f);
-      vb[j] = (in && eb != 0.f) ? sb[int64_t(kCombineWarps * j) * H] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < kFastParts; ++k) {
+      const int w = w_first + k;
+      lv[k] = (k < np && head_ok && live(w)) ? lse_part[int64_t(b + w) * H + i] : -INFINITY;
     }
 #pragma unroll
-    for (int j = 0; j < kQuadsPerWarp; ++j) {
-      acc[j].x = fmaf(ea, va[j].x, fmaf(eb, vb[j].x, acc[j].x));
-      acc[j].y = fmaf(ea, va[j].y, fmaf(eb, vb[j].y, acc[j].y));
-      acc[j].z = fmaf(ea, va[j].z, fmaf(eb, vb[j].z, acc[j].z));
-      acc[j].w = fmaf(ea, va[j].w, fmaf(eb, vb[j].w, acc[j].w));
+    for (int k = 0; k < kFastParts; ++k) m = fmaxf(m, lv[k]);
+    float e[kFastParts];
+#pragma unroll
+    for (int k = 0; k < kFastParts; ++k) {
+      e[k] = lv[k] == -INFINITY ? 0.f : expf(lv[k] - m);
+      z += e[k];
+    }
+    const float inv_z = head_ok ? 1.f / z : 0.f;
+#pragma unroll
+    for (int k = 0; k < kFastParts; ++k) e[k] *= inv_z;
+    // Two column groups per round keep the live registers low enough for four
+    // blocks per SM.
+#pragma unroll
+    for (int j0 = 0; j0 < kQuadsPerWarp; j0 += 2) {
+      float4 v[kFastParts][2];
+#pragma unroll
+      for (int k = 0; k < kFastParts; ++k) {
+        const float4* sk = src0 + int64_t(b + w_first + (k < np ? k : 0)) * slot_stride;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = j0 + jj;
+          const bool in = e[k] != 0.f && warp + kCombineWarps * j < nqb;
+          v[k][jj] = in ? sk[int64_t(kCombineWarps * j) * H] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kFastParts; ++k)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = j0 + jj;
+          acc[j].x = fmaf(e[k], v[k][jj].x, acc[j].x);
+          acc[j].y = fmaf(e[k], v[k][jj].y, acc[j].y);
+          acc[j].z = fmaf(e[k], v[k][jj].z, acc[j].z);
+          acc[j].w = fmaf(e[k], v[k][jj].w, acc[j].w);
+        }
+    }
+  } else {
+    for (int w = w_first; w <= w_last; ++w)
+      if (live(w) && head_ok) m = fmaxf(m, lse_part[int64_t(b + w) * H + i]);
+    for (int w = w_first; w <= w_last; ++w)
+      if (live(w) && head_ok) z += expf(lse_part[int64_t(b + w) * H + i] - m);
+    const float inv_z = head_ok ? 1.f / z : 0.f;
+    auto weight = [&](int w) {
+      return (live(w) && head_ok) ? expf(lse_part[int64_t(b + w) * H + i] - m) * inv_z : 0.f;
+    };
+    for (int w = w_first; w <= w_last; w += 2) {
+      const bool two = w + 1 <= w_last;
+      const float ea = weight(w), eb = two ? weight(w + 1) : 0.f;
+      const float4* sa = src0 + int64_t(b + w) * slot_stride;
+      const float4* sb = src0 + int64_t(b + (two ? w + 1 : w)) * slot_stride;
+      float4 va[kQuadsPerWarp], vb[kQuadsPerWarp];
+#pragma unroll
+      for (int j = 0; j < kQuadsPerWarp; ++j) {
+        const bool in = head_ok && warp + kCombineWarps * j < nqb;
+        va[j] = (in && ea != 0.f) ? sa[int64_t(kCombineWarps * j) * H] : make_float4(0.f, 0.f, 0.f, 0.f);
+        vb[j] = (in && eb != 0.f) ? sb[int64_t(kCombineWarps * j) * H] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < kQuadsPerWarp; ++j) {
+        acc[j].x = fmaf(ea, va[j].x, fmaf(eb, vb[j].x, acc[j].x));
+        acc[j].y = fmaf(ea, va[j].y, fmaf(eb, vb[j].y, acc[j].y));
+        acc[j].z = fmaf(ea, va[j].z, fmaf(eb, vb[j].z, acc[j].z));
+        acc[j].w = fmaf(ea, va[j].w, fmaf(eb, vb[j].w, acc[j].w));
+      }
     }
   }
 #pragma unroll
