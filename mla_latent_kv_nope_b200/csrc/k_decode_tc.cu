@@ -384,48 +384,35 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     bool ok = true;
 
     // Query block of sequence b into tensor memory (lo lanes, K-major pairs of
-    // bf16 per 32-bit column).  The two half-warps write alternate column
-    // groups of the same 16 rows.  All 36 16-byte loads of a thread are
-    // issued before the first store, so the block costs one memory round trip.
+    // bf16 per 32-bit column).  A row is 72 16-byte units; the two half-warps
+    // take alternate units of the same 16 rows, so each warp load reads one
+    // 32-byte sector per row, and a 16x32bx2 store with a 4-column split puts
+    // unit 2j at columns [8j, 8j+4) and unit 2j+1 at [8j+4, 8j+8).  All 36
+    // loads of a thread are issued before the first store (one round trip).
     auto write_query = [&](int b) {
       const int64_t qrow = int64_t(b) * H + int64_t(g) * kHeadsPerCta + row;
       const bool valid_row = qrow < int64_t(B) * H;
-      // All 36 loads are unconditional (a padding row reads row 0 and is
-      // zeroed afterwards) so they are in flight together.
       const uint4* src = reinterpret_cast<const uint4*>(q_cat + (valid_row ? qrow : 0) * kR);
       uint4 v[36];
 #pragma unroll
-      for (int j = 0; j < 32; ++j)   // four 64-column groups: words [64c + half*32, +32)
-        v[j] = src[((j / 8) * 64 + (lo_half ? 0 : 32) + (j % 8) * 4) >> 2];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)    // last 32 columns: words [256 + half*16, +16)
-        v[32 + j] = src[(256 + (lo_half ? 0 : 16) + j * 4) >> 2];
+      for (int j = 0; j < 36; ++j) v[j] = src[2 * j + (lo_half ? 0 : 1)];
       if (!valid_row) {
 #pragma unroll
         for (int j = 0; j < 36; ++j) v[j] = make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          r[4 * q4] = v[8 * c + q4].x; r[4 * q4 + 1] = v[8 * c + q4].y;
-          r[4 * q4 + 2] = v[8 * c + q4].z; r[4 * q4 + 3] = v[8 * c + q4].w;
-        }
-        tmem_st16x2_32<32>(lo_base + kColQ + uint32_t(64 * c), r);
-      }
-      {
-        uint32_t r[16];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          r[4 * q4] = v[32 + q4].x; r[4 * q4 + 1] = v[32 + q4].y;
-          r[4 * q4 + 2] = v[32 + q4].z; r[4 * q4 + 3] = v[32 + q4].w;
-        }
-        tmem_st16x2_16<16>(lo_base + kColQ + 256u, r);
-      }
+      for (int j = 0; j < 36; ++j) tmem_st16x2_4<4>(lo_base + kColQ + uint32_t(8 * j), v[j]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->q_ready);
+    };
+    // The contiguous 64-row query block of sequence b into L2 ahead of use.
+    auto prefetch_query = [&](int b) {
+      if (b >= 0 && tid == 0) {
+        const int64_t r0 = int64_t(b) * H + int64_t(g) * kHeadsPerCta;
+        const int64_t rows = min(int64_t(kHeadsPerCta), int64_t(B) * H - r0);
+        if (rows > 0) bulk_prefetch_l2(q_cat + r0 * kR, uint32_t(rows * kR * 2));
+      }
     };
 
     // The sequence of the worker's range that follows sequence `after`
@@ -447,6 +434,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     for_each_segment(tp, t_begin, t_end,
                      [&](int b, int64_t lo, int64_t hi, int64_t L) {
       const int slot = b + w;
+      prefetch_query(next_sequence(b));
       for (int64_t t = lo; t < hi; ++t, ++i) {
         const int st = i % kStages, sb = i & 1;
         if (!(ok = warp_wait(&bars->s_full[sb], (i >> 1) & 1, abort_flag))) return false;

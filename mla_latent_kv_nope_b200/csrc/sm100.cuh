@@ -204,6 +204,12 @@ __device__ __forceinline__ void tmem_st16x2_16(uint32_t taddr, const uint32_t (&
       "r"(r[15]), "n"(kSplit)
       : "memory");
 }
+template <int kSplit>
+__device__ __forceinline__ void tmem_st16x2_4(uint32_t taddr, const uint4& v) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x4.b32 [%0], %5, {%1, %2, %3, %4};" ::"r"(taddr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "n"(kSplit)
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
