@@ -291,6 +291,45 @@ def test_full_step_small(w):
     assert e < tol(w) and el < tol(w) and els < tol(w), (e, el, els)
 
 
+@pytest.mark.parametrize("w", [W["ragged_append_bf16"].scaled(B=6, N=500, hidden=512),
+                               W["v3_bf16"].scaled(B=3, N=300, append=True, hidden=512)],
+                         ids=["ragged-append", "v3-append"])
+def test_decode_step_streams_and_graph(w):
+    """DecodeStep with absorb_q on a forked stream, and the same step replayed
+    from a CUDA graph, give bit-identical outputs to the single-stream step
+    (same kernels, same inputs, deterministic reductions)."""
+    lens = inputs.seqlens(w)
+    d = dims_of(w)
+    qn, qp = inputs.query(w)
+    Wuk, Wuv = inputs.weights(w)
+    h, Wdkv = inputs.append_inputs(w)
+    args = [dev(qn, w), dev(qp, w), torch.from_numpy(lens.astype(np.int32)).cuda()]
+    hd = dev(h, w)
+
+    def run(step, cache, seq, graph=False):
+        seq0 = seq.clone()
+        if graph:
+            g = step.capture(*args, cache, seq, h=hd, after=lambda: seq.copy_(seq0))
+            for _ in range(2):
+                g.replay()
+        else:
+            step(*args, cache, seq, h=hd)
+            seq.copy_(seq0)
+        torch.cuda.synchronize()
+        assert mla.get_device_status() == 0
+        return step.out.clone(), step.lse.clone()
+
+    outs = []
+    for overlap, graph in [(False, False), (True, False), (True, True)]:
+        cache = device_cache(w, lens)
+        seq = torch.from_numpy(lens).cuda()
+        step = mla.DecodeStep(d, dev(Wuk, w), dev(Wuv, w), dev(Wdkv, w), overlap=overlap)
+        outs.append(run(step, cache, seq, graph))
+    for o, l in outs[1:]:
+        assert torch.equal(o, outs[0][0])
+        assert torch.equal(l, outs[0][1])
+
+
 def _sample(w, n_seq, heads, seed=0):
     r = np.random.default_rng(seed)
     seqs = sorted(set([0, w.B - 1] + list(r.choice(w.B, size=min(n_seq, w.B), replace=False))))
