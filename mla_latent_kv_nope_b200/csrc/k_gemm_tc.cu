@@ -162,11 +162,14 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __rest
 }
 
 // ---------------------------------------------------------------------------
-// absorb_q: CTA per head; N chunks of up to 64 sequences; 4 accumulators
-// (d_c = 512 = 4 x 128 output rows).
-// smem: W_UK[i] 8 x [128 (K = r) x 128 B (64 c)] (128 KB) | X 2 x [64 x 128 B] | barriers
+// absorb_q: grid (head, 4 blocks of 128 output columns); N chunks of up to
+// 64 sequences.  Each CTA streams the 32 KB of W_UK[i] its columns need, and
+// takes a quarter of the head's RoPE pairs.
+// smem: W_UK[i][:, 128m : 128m+128] 2 x [128 (K = r) x 128 B (64 c)] (32 KB) |
+//       X 2 x [64 x 128 B] | barriers
 constexpr int kAbN = 64;
-constexpr size_t kAbSmem = 8 * 16384 + 2 * (kAbN * 128) + 64 + 1024;
+constexpr int kAbBlocks = 4;                 // d_c = 512 = 4 x 128 output columns
+constexpr size_t kAbSmem = 2 * 16384 + 2 * (kAbN * 128) + 64 + 1024;
 
 __global__ void __launch_bounds__(kThreadsG, 1)
 absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16* __restrict__ q_nope,
@@ -176,10 +179,11 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sW = sm;
-  uint8_t* sX = sm + 8 * 16384;
+  uint8_t* sX = sm + 2 * 16384;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sX + 2 * kAbN * 128);
   uint32_t* tbase = reinterpret_cast<uint32_t*>(bars + 2);
   const int i = blockIdx.x;
+  const int mb = blockIdx.y;                 // output columns [128 mb, 128 mb + 128)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kR = 576;
   // Rotation frequencies of the 32 RoPE pairs, computed once per CTA while
@@ -191,11 +195,12 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
     mbar_init(&bars[1], 1);
     fence_mbar_init();
     fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&bars[0], 8 * 16384);
-    for (int c = 0; c < 8; ++c) tma_load_2d(&tm_w, &bars[0], sW + c * 16384, c * kChunk, i * 128);
+    mbar_arrive_expect_tx(&bars[0], 2 * 16384);
+    for (int c = 0; c < 2; ++c)
+      tma_load_2d(&tm_w, &bars[0], sW + c * 16384, (2 * mb + c) * kChunk, i * 128);
   }
   if (warp == 0) {
-    tmem_alloc(tbase, 4 * kAbN);
+    tmem_alloc(tbase, kAbN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -228,36 +233,33 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
     if (pass == 0) ok = block_wait(&bars[0], 0) && ok;
     if (warp == 0) {
       tc_fence_after();
-      // A for output rows [128 m, 128 m + 128): c-chunks 2m, 2m+1 (LBO = 16 KB
-      // between 64-wide c groups), K-step k = rows 16k..16k+15 of W_UK[i].
+      // A for output rows [128 mb, 128 mb + 128): the two loaded c-chunks
+      // (LBO = 16 KB between 64-wide c groups), K-step k = rows 16k..16k+15
+      // of W_UK[i].
       const uint64_t a0 = smem_desc_sw128(smem_u32(sW), 16384, 1024);
       const uint64_t b0 = smem_desc_sw128(smem_u32(sX), 16, 1024);
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-          mma_bf16_ss_w(tmem + uint32_t(m * kAbN), a0 + uint64_t((2 * m * 16384 + k * 2048) >> 4),
-                        b0 + uint64_t(((k / 4) * kAbN * 128 + (k % 4) * 32) >> 4), idesc, k != 0);
+        mma_bf16_ss_w(tmem, a0 + uint64_t((k * 2048) >> 4),
+                      b0 + uint64_t(((k / 4) * kAbN * 128 + (k % 4) * 32) >> 4), idesc, k != 0);
       mma_commit_w(&bars[1]);
     }
     ok = block_wait(&bars[1], pass & 1) && ok;
     tc_fence_after();
     const int crow = 32 * warp + lane;
 #pragma unroll 1
-    for (int m = 0; m < 4; ++m)
-#pragma unroll 1
-      for (int c0 = 0; c0 < kAbN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + uint32_t(m * kAbN + c0), r);
-        tmem_wait_ld();
-        if (ok) {
+    for (int c0 = 0; c0 < kAbN; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + uint32_t(c0), r);
+      tmem_wait_ld();
+      if (ok) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c0 + e < nc)
-              q_cat[(int64_t(n0 + c0 + e) * H + i) * kR + m * 128 + crow] =
-                  __float2bfloat16_rn(__uint_as_float(r[e]));
-        }
+        for (int e = 0; e < 32; ++e)
+          if (c0 + e < nc)
+            q_cat[(int64_t(n0 + c0 + e) * H + i) * kR + mb * 128 + crow] =
+                __float2bfloat16_rn(__uint_as_float(r[e]));
       }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -266,13 +268,15 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
   // Pairs (b, k) are taken 8 per thread with every load issued before the
   // first rotation, so the pass costs one memory round trip per 8 pairs.
   constexpr int kRopeBatch = 8;
-  for (int u0 = 0; u0 < B * 32; u0 += kRopeBatch * kThreadsG) {
+  const int u_lo = int(int64_t(B) * 32 * mb / kAbBlocks);
+  const int u_hi = int(int64_t(B) * 32 * (mb + 1) / kAbBlocks);
+  for (int u0 = u_lo; u0 < u_hi; u0 += kRopeBatch * kThreadsG) {
     float x1[kRopeBatch], x2[kRopeBatch];
     int32_t pos[kRopeBatch];
 #pragma unroll
     for (int j = 0; j < kRopeBatch; ++j) {
       const int u = u0 + j * kThreadsG + threadIdx.x;
-      const bool in = u < B * 32;
+      const bool in = u < u_hi;
       const int b = in ? u / 32 : 0, k = u % 32;
       const int64_t row = int64_t(b) * H + i;
       x1[j] = __bfloat162float(q_pe[row * 64 + k]);
@@ -282,7 +286,7 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
 #pragma unroll
     for (int j = 0; j < kRopeBatch; ++j) {
       const int u = u0 + j * kThreadsG + threadIdx.x;
-      if (u >= B * 32) continue;
+      if (u >= u_hi) continue;
       const int b = u / 32, k = u % 32;
       const int64_t row = int64_t(b) * H + i;
       float y1 = x1[j], y2 = x2[j];
@@ -301,7 +305,7 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 4 * kAbN);
+    tmem_dealloc(tmem, kAbN);
   }
 }
 
@@ -452,7 +456,8 @@ cudaError_t launch_absorb_q_tc(const __nv_bfloat16* q_nope, const __nv_bfloat16*
   if (!make_map(&tm, W_UK, uint64_t(H) * 128, 512, 128)) return cudaErrorInvalidValue;
   cudaError_t e = set_smem(absorb_q_tc_kernel, kAbSmem);
   if (e != cudaSuccess) return e;
-  absorb_q_tc_kernel<<<H, kThreadsG, kAbSmem, stream>>>(tm, q_nope, q_pe, q_pos, rope_base, B, H,
+  absorb_q_tc_kernel<<<dim3(H, kAbBlocks), kThreadsG, kAbSmem, stream>>>(tm, q_nope, q_pe, q_pos,
+                                                                         rope_base, B, H,
                                                         q_cat, status);
   return cudaGetLastError();
 }
