@@ -158,6 +158,7 @@ def run_ours(args, rank, world, local_rank):
     import torch
 
     import mla_latent_kv_nope_b200 as mla
+    from mla_latent_kv_nope_b200 import dist as mdist
     from mla_latent_kv_nope_b200 import inputs
     from mla_latent_kv_nope_b200.build import build
 
@@ -168,7 +169,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = inputs.WORKLOADS[args.workload].scaled(seed=rank)
+    w = mdist.shard(inputs.WORKLOADS[args.workload], rank)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     dims = mla.Dims(w.B, w.H, w.d_c, w.d_r, w.d_nope, w.d_v, w.capacity, w.dtype)
 
@@ -238,9 +239,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device status error during warm-up")
 
     def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+        mdist.barrier(world)
 
     with ClockSampler(local_rank) as clk:
         barrier()
@@ -257,11 +256,7 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         ms_total = t0.elapsed_time(t1)
         dec_ms, decomb_ms = decode_only(max(args.steps, 5))
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = mdist.max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
 
     # e2e through the public API with host buffers: pinned H2D of the step's
@@ -305,11 +300,7 @@ def run_ours(args, rank, world, local_rank):
     b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / args.steps
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = mdist.max_over_ranks(e2e_ms, world, dev)
     if mla.get_device_status() != 0:
         raise RuntimeError("device status error during timing")
 
@@ -327,7 +318,7 @@ def run_ours(args, rank, world, local_rank):
     tokens = w.B * world
     res = {
         "metric": METRIC,
-        "value": tokens / (ms_step * 1e-3),
+        "value": mdist.job_tokens_per_s(w.B, world, ms_step),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -373,7 +364,7 @@ def run_ours(args, rank, world, local_rank):
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured"
                            else "fallback",
         },
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": mdist.job_tokens_per_s(w.B, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms},
         "gpu_launches": 6 * args.steps,
         "clocks": clk.summary(),
