@@ -267,36 +267,74 @@ def run_ours(args, rank, world, local_rank):
     bi = sum(t.numel() * t.element_size() for t in (h_qn, h_qp, h_pos, h_h))
     bo = h_out.numel() * h_out.element_size()
 
-    def e2e_in():
-        q_nope.copy_(h_qn, non_blocking=True)
-        q_pe.copy_(h_qp, non_blocking=True)
-        q_pos.copy_(h_pos, non_blocking=True)
-        hh.copy_(h_h, non_blocking=True)
-        if flush is not None:
-            flush.zero_()
+    host_in = (h_qn, h_qp, h_pos, h_h)
 
-    def e2e_out():
-        h_out.copy_(step.out, non_blocking=True)
-        seq.copy_(seq0)
+    if args.eager:
+        # One step at a time: inputs in, step, output out, all on one stream.
+        def e2e_run(n):
+            for _ in range(n):
+                for d_t, h_t in zip((q_nope, q_pe, q_pos, hh), host_in):
+                    d_t.copy_(h_t, non_blocking=True)
+                if flush is not None:
+                    flush.zero_()
+                step(q_nope, q_pe, q_pos, cache, seq, h=hh)
+                h_out.copy_(step.out, non_blocking=True)
+                seq.copy_(seq0)
+    else:
+        # Pipelined: two device input sets, each with a graph of the step; the
+        # copy stream brings step k+1's inputs in and takes step k's output
+        # out while step k computes.  Every step still copies its own inputs
+        # from pinned host memory and its result back to it.
+        copy_stream = torch.cuda.Stream(device=dev)
+        sets = []
+        for _ in range(2):
+            d_in = [t.clone() for t in (q_nope, q_pe, q_pos, hh)]
+            stage = torch.empty_like(step.out)
 
-    def e2e_eager():
-        e2e_in()
-        step(q_nope, q_pe, q_pos, cache, seq, h=hh)
-        e2e_out()
+            def after(stage=stage):
+                if flush is not None:
+                    flush.zero_()
+                stage.copy_(step.out)
+                seq.copy_(seq0)
+            g = step.capture(d_in[0], d_in[1], d_in[2], cache, seq, h=d_in[3], after=after)
+            sets.append((d_in, stage, g))
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    # Host-buffer steps are issued eagerly: with the copies inside a graph
-    # they measured slower on B200 (the copies dominate this path).
-    e2e_step = e2e_eager
+        def load_inputs(c):
+            for d_t, h_t in zip(sets[c][0], host_in):
+                d_t.copy_(h_t, non_blocking=True)
+            ev_in[c].record(copy_stream)
 
-    for _ in range(3):
-        e2e_step()
+        def e2e_run(n):
+            copy_stream.wait_stream(stream)
+            with torch.cuda.stream(copy_stream):
+                load_inputs(0)
+            for k in range(n):
+                c = k % 2
+                stream.wait_event(ev_in[c])
+                if k >= 2:
+                    stream.wait_event(ev_out[c])     # step k-2's result has left `stage`
+                sets[c][2].replay()
+                ev_done[c].record(stream)
+                with torch.cuda.stream(copy_stream):
+                    if k + 1 < n:
+                        if k >= 1:
+                            copy_stream.wait_event(ev_done[1 - c])  # step k-1 read that set
+                        load_inputs(1 - c)
+                    copy_stream.wait_event(ev_done[c])
+                    h_out.copy_(sets[c][1], non_blocking=True)
+                    ev_out[c].record(copy_stream)
+            stream.wait_stream(copy_stream)
+
+    e2e_run(3)
     torch.cuda.synchronize()
     barrier()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    e2e_run(args.steps)
     b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / args.steps
