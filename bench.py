@@ -422,6 +422,17 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_oracle_baseline(w, budget_s=15.0):
     """The float64 materialised-MHA oracle, as it stands, on a bounded sample
     of the same workload: whole (sequence, head) pairs, one appended token
@@ -459,6 +470,7 @@ def cpu_oracle_baseline(w, budget_s=15.0):
     per_pair = spent / len(done)
     step_s = per_pair * w.B * w.H
     return {"value": w.B / step_s, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "cpu_model": _cpu_model(), "host_cores": os.cpu_count(),
             "sample": f"{len(done)} (sequence, head) pairs of one step ({spent:.1f} s CPU), "
                       f"each append + materialised attention over its full length; "
                       f"scaled by B*H = {w.B * w.H} pairs per step"}
