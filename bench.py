@@ -176,6 +176,18 @@ def run_ours(args, rank, world, local_rank):
     lens = inputs.seqlens(w)
     cache = torch.empty(w.B, w.capacity, w.R, dtype=dt, device=dev)
     inputs.fill_cache(w, cache, lens, fill_rest=0.0)
+    table = None
+    if args.paged:
+        # The same rows in a pool of 64-row pages, pages shuffled, and the
+        # block table that finds them; every call below reads the pool.
+        nb = (w.capacity + mla.PAGE_ROWS - 1) // mla.PAGE_ROWS
+        padded = torch.zeros(w.B, nb * mla.PAGE_ROWS, w.R, dtype=dt, device=dev)
+        padded[:, :w.capacity] = cache
+        perm = torch.from_numpy(np.random.default_rng(1).permutation(w.B * nb)).to(dev)
+        cache = torch.empty(w.B * nb, mla.PAGE_ROWS, w.R, dtype=dt, device=dev)
+        cache[perm] = padded.reshape(w.B * nb, mla.PAGE_ROWS, w.R)
+        table = perm.to(torch.int32).reshape(w.B, nb).contiguous()
+        del padded
     seq0 = torch.from_numpy(lens).to(dev)
     seq = seq0.clone()
     qn, qp = inputs.query(w)
@@ -195,7 +207,7 @@ def run_ours(args, rank, world, local_rank):
     def eager_step():
         if flush is not None:
             flush.zero_()
-        step(q_nope, q_pe, q_pos, cache, seq, h=hh)
+        step(q_nope, q_pe, q_pos, cache, seq, h=hh, block_table=table)
         seq.copy_(seq0)
 
     # A step is replayed from a CUDA graph (one host launch per step) unless
@@ -208,21 +220,25 @@ def run_ours(args, rank, world, local_rank):
     else:
         graph = step.capture(q_nope, q_pe, q_pos, cache, seq, h=hh,
                              before=(flush.zero_ if flush is not None else None),
-                             after=lambda: seq.copy_(seq0))
+                             after=lambda: seq.copy_(seq0), block_table=table)
         one_step = graph.replay
 
     # Decode-kernel-only events (for the roofline): separate pass so that
     # the step timing has no extra event records inside it.
     def decode_only(n):
         evs = []
-        step.append(hh, cache, seq)
+        step.append(hh, cache, seq, table)
         mla.absorb_q(dims, q_nope, q_pe, W_UK, q_pos, step.q_cat, step.rope_base)
         for _ in range(n):
             if flush is not None:
                 flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            mla.decode(dims, step.q_cat, cache, seq, step.scale, step.ws, step.num_splits)
+            if table is None:
+                mla.decode(dims, step.q_cat, cache, seq, step.scale, step.ws, step.num_splits)
+            else:
+                mla.decode_paged(dims, step.q_cat, cache, table, seq, step.scale, step.ws,
+                                 step.num_splits)
             e1.record(stream)
             e2 = torch.cuda.Event(enable_timing=True)
             mla.combine(dims, seq, step.ws, step.splits_used, step.o_lat, step.lse)
@@ -277,7 +293,7 @@ def run_ours(args, rank, world, local_rank):
                     d_t.copy_(h_t, non_blocking=True)
                 if flush is not None:
                     flush.zero_()
-                step(q_nope, q_pe, q_pos, cache, seq, h=hh)
+                step(q_nope, q_pe, q_pos, cache, seq, h=hh, block_table=table)
                 h_out.copy_(step.out, non_blocking=True)
                 seq.copy_(seq0)
     else:
@@ -296,7 +312,8 @@ def run_ours(args, rank, world, local_rank):
                     flush.zero_()
                 stage.copy_(step.out)
                 seq.copy_(seq0)
-            g = step.capture(d_in[0], d_in[1], d_in[2], cache, seq, h=d_in[3], after=after)
+            g = step.capture(d_in[0], d_in[1], d_in[2], cache, seq, h=d_in[3], after=after,
+                             block_table=table)
             sets.append((d_in, stage, g))
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -377,6 +394,8 @@ def run_ours(args, rank, world, local_rank):
             "l2": ("inputs exceed L2 (cache %.0f MB)" % (cache_bytes / 1e6)) if flush is None
                   else "L2 flushed between steps",
             "num_splits": step.splits_used,
+            "cache": ("paged: 64-row pages, shuffled, block table" if args.paged
+                      else "contiguous [B, capacity, 576]"),
             "launch": "eager" if args.eager else "cuda_graph (absorb_q on a forked stream)",
         },
         "decode_only": {
@@ -513,6 +532,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--paged", action="store_true",
+                    help="keep the latent cache in shuffled 64-row pages behind a block table")
     ap.add_argument("--eager", action="store_true",
                     help="launch each kernel from the host every step instead of a CUDA graph")
     args = ap.parse_args()

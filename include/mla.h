@@ -159,6 +159,32 @@ MLA_API int mla_combine(const mla_dims* dims, const int32_t* seqlens,
 MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W_UV,
                  void* out, void* stream);
 
+/* --- paged latent cache --------------------------------------------------------
+ * No counterpart on the pages beyond the name: [MLA-とは] names PagedAttention
+ * as the serving-side cache organisation this method fits; the page size is
+ * fixed here at 64 rows, one decode work tile.
+ * The cache is a pool of num_pages pages, cache_pool [num_pages, 64, d_c + d_r]
+ * (dtype), and block_table [B, max_blocks] int32 maps sequence b's key j to
+ * row j % 64 of page block_table[b, j / 64].  dims->cache_capacity is the
+ * longest sequence allowed and must be <= 64 * max_blocks; entries for tiles
+ * at or beyond a sequence's length are never read.  Otherwise these calls are
+ * mla_decode and mla_cache_append with the same inputs, outputs, workspace,
+ * partial layout and errors (mla_combine merges the partials as usual).  A
+ * page id outside [0, num_pages) is not dereferenced: it is recorded as
+ * MLA_ERR_BOUNDS in the device status word (decode reads its rows as zeros;
+ * append writes nothing and leaves L_b unchanged). */
+MLA_API int mla_decode_paged(const mla_dims* dims, const void* q_cat, const void* cache_pool,
+                             int64_t num_pages, const int32_t* block_table, int32_t max_blocks,
+                             const int32_t* seqlens, float softmax_scale, int num_splits,
+                             void* workspace, size_t workspace_bytes, int* splits_used,
+                             void* stream);
+MLA_API int mla_cache_append_paged(const mla_dims* dims, int32_t hidden, const void* h,
+                                   const void* W_DKV, const float* gamma, float eps,
+                                   float rope_base, void* cache_pool, int64_t num_pages,
+                                   const int32_t* block_table, int32_t max_blocks,
+                                   int32_t* seqlens, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
 /* --- 3+4 without a workspace -------------------------------------------------
  * No counterpart on the pages: this is a convenience of this library.
  * For callers that cannot allocate device memory (code running while a stream

@@ -4,7 +4,8 @@ The compute lives in ``libmla_b200.so`` (hand-written CUDA kernels behind the C
 ABI declared in ``include/mla.h``); ``binding`` marshals torch tensors to it.
 """
 from .binding import (  # noqa: F401
-    Dims, DecodeStep, MLAError, absorb_q, cache_append, cache_append_workspace_bytes,
+    PAGE_ROWS, Dims, DecodeStep, MLAError, absorb_q, cache_append, cache_append_paged,
+    cache_append_workspace_bytes, decode_paged,
     cache_row_elems, combine, decode, decode_default_splits, decode_workspace_bytes,
     get_device_status, load_library, out_proj,
 )

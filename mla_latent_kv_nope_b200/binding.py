@@ -26,8 +26,10 @@ EXPORTED = (
     "mla_cache_row_elems", "mla_cache_append_workspace_bytes", "mla_cache_append",
     "mla_absorb_q", "mla_decode_default_splits", "mla_decode_workspace_bytes",
     "mla_decode", "mla_combine", "mla_out_proj", "mla_get_device_status",
-    "mla_status_string", "mla_decode_noalloc",
+    "mla_status_string", "mla_decode_noalloc", "mla_decode_paged", "mla_cache_append_paged",
 )
+
+PAGE_ROWS = 64   # rows per page of a paged latent cache (one decode work tile)
 
 
 class MLAError(RuntimeError):
@@ -97,6 +99,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_out_proj": (ctypes.c_int, [D, P, P, P, P]),
         "mla_get_device_status": (ctypes.c_int, [P]),
         "mla_decode_noalloc": (ctypes.c_int, [D, P, P, P, F, P, P, P]),
+        "mla_decode_paged": (ctypes.c_int, [D, P, P, I64, P, I32, P, F, ctypes.c_int, P, SZ,
+                                            ctypes.POINTER(ctypes.c_int), P]),
+        "mla_cache_append_paged": (ctypes.c_int, [D, I32, P, P, P, F, F, P, I64, P, I32, P, P,
+                                                  SZ, P]),
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -159,6 +165,51 @@ def cache_append(dims: Dims, h, W_DKV, gamma, cache, seqlens, workspace, eps=1e-
         _ptr(cache), _ptr(seqlens), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check("mla_cache_append", st)
+
+
+def _need_pages(dims: Dims, pool, block_table):
+    if pool.dim() != 3 or pool.shape[1:] != (PAGE_ROWS, dims.R):
+        raise ValueError(f"cache_pool must be [num_pages, {PAGE_ROWS}, {dims.R}]")
+    _need(pool, dims.torch_dtype, tuple(pool.shape), "cache_pool")
+    if block_table.dim() != 2 or block_table.shape[0] != dims.B:
+        raise ValueError("block_table must be [B, max_blocks]")
+    _need(block_table, torch.int32, tuple(block_table.shape), "block_table")
+
+
+def cache_append_paged(dims: Dims, h, W_DKV, gamma, cache_pool, block_table, seqlens,
+                       workspace, eps=1e-6, rope_base=10000.0, stream=None):
+    """mla_cache_append on a paged cache: cache_pool [num_pages, 64, R], block_table
+    [B, max_blocks] int32 page ids."""
+    dt = dims.torch_dtype
+    hidden = h.shape[-1]
+    _need(h, dt, (dims.B, hidden), "h")
+    _need(W_DKV, dt, (dims.R, hidden), "W_DKV")
+    _need_pages(dims, cache_pool, block_table)
+    _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    if gamma is not None:
+        _need(gamma, torch.float32, (dims.d_c,), "gamma")
+    st = load_library().mla_cache_append_paged(
+        ctypes.byref(dims.c()), hidden, _ptr(h), _ptr(W_DKV), _ptr(gamma), eps, rope_base,
+        _ptr(cache_pool), cache_pool.shape[0], _ptr(block_table), block_table.shape[1],
+        _ptr(seqlens), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check("mla_cache_append_paged", st)
+
+
+def decode_paged(dims: Dims, q_cat, cache_pool, block_table, seqlens, softmax_scale, workspace,
+                 num_splits=0, stream=None) -> int:
+    """mla_decode on a paged cache (see cache_append_paged)."""
+    _need(q_cat, dims.torch_dtype, (dims.B, dims.H, dims.R), "q_cat")
+    _need_pages(dims, cache_pool, block_table)
+    _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    used = ctypes.c_int(0)
+    st = load_library().mla_decode_paged(
+        ctypes.byref(dims.c()), _ptr(q_cat), _ptr(cache_pool), cache_pool.shape[0],
+        _ptr(block_table), block_table.shape[1], _ptr(seqlens), float(softmax_scale), num_splits,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), ctypes.byref(used),
+        _stream(stream))
+    _check("mla_decode_paged", st)
+    return used.value
 
 
 def absorb_q(dims: Dims, q_nope, q_pe, W_UK, q_pos, q_cat, rope_base=10000.0, stream=None):
@@ -255,29 +306,39 @@ class DecodeStep:
         self.splits_used = self.num_splits
         self._side = torch.cuda.Stream(device=device) if overlap else None
 
-    def append(self, h, cache, seqlens):
-        cache_append(self.dims, h, self.W_DKV, self.gamma, cache, seqlens, self.ws_append,
-                     self.eps, self.rope_base)
+    def append(self, h, cache, seqlens, block_table=None):
+        if block_table is None:
+            cache_append(self.dims, h, self.W_DKV, self.gamma, cache, seqlens, self.ws_append,
+                         self.eps, self.rope_base)
+        else:
+            cache_append_paged(self.dims, h, self.W_DKV, self.gamma, cache, block_table,
+                               seqlens, self.ws_append, self.eps, self.rope_base)
 
     def _absorb(self, q_nope, q_pe, q_pos):
         absorb_q(self.dims, q_nope, q_pe, self.W_UK, q_pos, self.q_cat, self.rope_base)
 
-    def _attend_latent(self, cache, seqlens):
-        self.splits_used = decode(self.dims, self.q_cat, cache, seqlens, self.scale, self.ws,
-                                  self.num_splits)
+    def _attend_latent(self, cache, seqlens, block_table=None):
+        if block_table is None:
+            self.splits_used = decode(self.dims, self.q_cat, cache, seqlens, self.scale, self.ws,
+                                      self.num_splits)
+        else:
+            self.splits_used = decode_paged(self.dims, self.q_cat, cache, block_table, seqlens,
+                                            self.scale, self.ws, self.num_splits)
         combine(self.dims, seqlens, self.ws, self.splits_used, self.o_lat, self.lse)
         out_proj(self.dims, self.o_lat, self.W_UV, self.out)
         return self.out
 
-    def attend(self, q_nope, q_pe, q_pos, cache, seqlens):
+    def attend(self, q_nope, q_pe, q_pos, cache, seqlens, block_table=None):
         self._absorb(q_nope, q_pe, q_pos)
-        return self._attend_latent(cache, seqlens)
+        return self._attend_latent(cache, seqlens, block_table)
 
-    def __call__(self, q_nope, q_pe, q_pos, cache, seqlens, h=None):
+    def __call__(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, block_table=None):
+        """One step.  With ``block_table`` the cache is a paged pool
+        [num_pages, 64, R] (see decode_paged)."""
         if self._side is None:
             if h is not None:
-                self.append(h, cache, seqlens)
-            return self.attend(q_nope, q_pe, q_pos, cache, seqlens)
+                self.append(h, cache, seqlens, block_table)
+            return self.attend(q_nope, q_pe, q_pos, cache, seqlens, block_table)
         main = torch.cuda.current_stream()
         # Fork: the side stream starts after everything issued so far (the
         # previous step's decode has finished reading q_cat).
@@ -285,11 +346,12 @@ class DecodeStep:
         with torch.cuda.stream(self._side):
             self._absorb(q_nope, q_pe, q_pos)
         if h is not None:
-            self.append(h, cache, seqlens)
+            self.append(h, cache, seqlens, block_table)
         main.wait_stream(self._side)
-        return self._attend_latent(cache, seqlens)
+        return self._attend_latent(cache, seqlens, block_table)
 
-    def capture(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, before=None, after=None):
+    def capture(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, before=None, after=None,
+                block_table=None):
         """Record one step into a CUDA graph; ``before``/``after`` are optional
         callables whose device work is recorded around it.  Replay with
         ``graph.replay()``; inputs are read from the same tensors each time."""
@@ -297,7 +359,7 @@ class DecodeStep:
         with torch.cuda.graph(g):
             if before is not None:
                 before()
-            self(q_nope, q_pe, q_pos, cache, seqlens, h=h)
+            self(q_nope, q_pe, q_pos, cache, seqlens, h=h, block_table=block_table)
             if after is not None:
                 after()
         return g

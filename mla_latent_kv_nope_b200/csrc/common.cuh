@@ -60,6 +60,34 @@ __device__ __forceinline__ int64_t tiles_of(int64_t L) {
   return L > 0 ? (L + kTileKeys - 1) / kTileKeys : 0;
 }
 
+// Where the cached rows of a sequence live.  Contiguous: sequence b owns rows
+// [b*cap, (b+1)*cap) of the cache viewed as [rows, d_c + d_r].  Paged: the
+// cache is a pool of pages of kTileKeys rows and key j of sequence b is row
+// j % kTileKeys of page table[b*max_blocks + j / kTileKeys] (a page holds
+// exactly one work tile).
+struct PageMap {
+  const int32_t* table;   // [B][max_blocks] page ids, or nullptr (contiguous)
+  int32_t max_blocks;
+  int64_t num_pages;
+  int64_t cap;
+
+  // First row of tile t of sequence b; -1 for a page id outside the pool.
+  __device__ __forceinline__ int64_t tile_row(int b, int64_t t) const {
+    if (!table) return int64_t(b) * cap + t * kTileKeys;
+    const int32_t pg = table[int64_t(b) * max_blocks + t];
+    return (pg < 0 || int64_t(pg) >= num_pages) ? -1 : int64_t(pg) * kTileKeys;
+  }
+  // Row of key j of sequence b; -1 for a page id outside the pool.
+  __device__ __forceinline__ int64_t row(int b, int64_t j) const {
+    const int64_t r = tile_row(b, j / kTileKeys);
+    return r < 0 ? -1 : r + j % kTileKeys;
+  }
+  // Rows addressed by the map (the extent of the cache tensor).
+  __host__ __device__ int64_t total_rows(int B) const {
+    return table ? num_pages * kTileKeys : int64_t(B) * cap;
+  }
+};
+
 // First tile owned by worker w of W over T tiles: floor(w*T/W).
 __device__ __forceinline__ int64_t worker_tile_begin(int64_t w, int64_t T, int64_t W) {
   return (w * T) / W;

@@ -73,7 +73,7 @@ template <typename T>
 __global__ void __launch_bounds__(1024)
 append_finalize_kernel(const float* __restrict__ part, int n_parts,
                        const float* __restrict__ gamma, float eps, float rope_base, int d_c,
-                       int d_r, int64_t cap, T* __restrict__ cache,
+                       int d_r, int64_t cap, T* __restrict__ cache, const PageMap pm,
                        int32_t* __restrict__ seqlens, int* __restrict__ status) {
   const int b = blockIdx.x;
   const int B = gridDim.x;
@@ -114,7 +114,12 @@ append_finalize_kernel(const float* __restrict__ part, int n_parts,
 #pragma unroll
   for (int wdx = 0; wdx < int(blockDim.x / 32); ++wdx) tot += s_part[wdx];
   const float inv = 1.f / sqrtf(tot / float(d_c) + eps);
-  T* row = cache + (int64_t(b) * cap + L) * R;
+  const int64_t r = pm.row(b, L);
+  if (r < 0) {   // page id outside the pool: nothing written, length unchanged
+    if (threadIdx.x == 0) record_status(status, MLA_ERR_BOUNDS);
+    return;
+  }
+  T* row = cache + r * R;
   for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
     const float g = gamma ? gamma[c] : 1.f;
     row[c] = Storage<T>::from_f(xb[c] * inv * g);
@@ -136,42 +141,44 @@ append_finalize_kernel(const float* __restrict__ part, int n_parts,
 template <typename T>
 cudaError_t launch_cache_append(const T* h, const T* W_DKV, const float* gamma, float eps,
                                 float rope_base, int B, int d_c, int d_r, int hidden,
-                                int64_t cap, T* cache, int32_t* seqlens, float* x_ws,
-                                int* status, cudaStream_t stream) {
+                                int64_t cap, T* cache, const PageMap& pm, int32_t* seqlens,
+                                float* x_ws, int* status, cudaStream_t stream) {
   const int R = d_c + d_r;
   append_project_kernel<T><<<(R + kApRows - 1) / kApRows, kApThreads, 0, stream>>>(
       h, W_DKV, B, R, hidden, x_ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_append_finalize<T>(x_ws, 1, gamma, eps, rope_base, B, d_c, d_r, cap, cache,
+  return launch_append_finalize<T>(x_ws, 1, gamma, eps, rope_base, B, d_c, d_r, cap, cache, pm,
                                    seqlens, status, stream);
 }
 
 template <typename T>
 cudaError_t launch_append_finalize(const float* part, int n_parts, const float* gamma, float eps,
                                    float rope_base, int B, int d_c, int d_r, int64_t cap,
-                                   T* cache, int32_t* seqlens, int* status, cudaStream_t stream) {
+                                   T* cache, const PageMap& pm, int32_t* seqlens, int* status,
+                                   cudaStream_t stream) {
   const size_t smem = sizeof(float) * size_t(d_c + d_r);
   const int threads = min(1024, (d_c + d_r + 31) / 32 * 32);
   append_finalize_kernel<T><<<B, threads, smem, stream>>>(part, n_parts, gamma, eps, rope_base,
-                                                             d_c, d_r, cap, cache, seqlens,
+                                                             d_c, d_r, cap, cache, pm, seqlens,
                                                              status);
   return cudaGetLastError();
 }
 
 template cudaError_t launch_append_finalize<float>(const float*, int, const float*, float, float,
-                                                   int, int, int, int64_t, float*, int32_t*, int*,
-                                                   cudaStream_t);
+                                                   int, int, int, int64_t, float*,
+                                                   const PageMap&, int32_t*, int*, cudaStream_t);
 template cudaError_t launch_append_finalize<__nv_bfloat16>(const float*, int, const float*, float,
                                                            float, int, int, int, int64_t,
-                                                           __nv_bfloat16*, int32_t*, int*,
-                                                           cudaStream_t);
+                                                           __nv_bfloat16*, const PageMap&,
+                                                           int32_t*, int*, cudaStream_t);
 
 template cudaError_t launch_cache_append<float>(const float*, const float*, const float*,
                                                 float, float, int, int, int, int, int64_t,
-                                                float*, int32_t*, float*, int*, cudaStream_t);
+                                                float*, const PageMap&, int32_t*, float*, int*,
+                                                cudaStream_t);
 template cudaError_t launch_cache_append<__nv_bfloat16>(
     const __nv_bfloat16*, const __nv_bfloat16*, const float*, float, float, int, int, int,
-    int, int64_t, __nv_bfloat16*, int32_t*, float*, int*, cudaStream_t);
+    int, int64_t, __nv_bfloat16*, const PageMap&, int32_t*, float*, int*, cudaStream_t);
 
 }  // namespace mla

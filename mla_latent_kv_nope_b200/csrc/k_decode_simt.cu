@@ -23,7 +23,7 @@ constexpr int kMaxAccPerLane = 32;  // d_c <= 1024
 
 template <typename T>
 __global__ void __launch_bounds__(kSimtHeads * 32)
-decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache,
+decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache, const PageMap pm,
                    const int32_t* __restrict__ seqlens, int B, int H, int d_c,
                    int R, int64_t cap, float scale, int W,
                    float* __restrict__ o_part, float* __restrict__ lse_part,
@@ -59,7 +59,6 @@ decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache,
     if (lo_t < hi_t) {
       const int64_t key_lo = (lo_t - prefix) * kTileKeys;
       const int64_t key_hi = min((hi_t - prefix) * int64_t(kTileKeys), L);
-      const T* rows_b = cache + int64_t(b) * cap * R;
 
       // Stage this block's queries.
       __syncthreads();
@@ -77,7 +76,9 @@ decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache,
         __syncthreads();
         for (int idx = threadIdx.x; idx < nk * R; idx += blockDim.x) {
           const int j = idx / R, c = idx % R;
-          s_rows[j * ldr + c] = Storage<T>::to_f(rows_b[(k0 + j) * R + c]);
+          const int64_t r = pm.row(b, k0 + j);   // -1: page id outside the pool
+          if (r < 0 && c == 0) record_status(status, MLA_ERR_BOUNDS);
+          s_rows[j * ldr + c] = r < 0 ? 0.f : Storage<T>::to_f(cache[r * R + c]);
         }
         __syncthreads();
         // Score: lane j takes key j.
@@ -126,7 +127,8 @@ decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache,
 }  // namespace
 
 template <typename T>
-cudaError_t launch_decode_simt(const T* q_cat, const T* cache, const int32_t* seqlens,
+cudaError_t launch_decode_simt(const T* q_cat, const T* cache, const PageMap& pm,
+                               const int32_t* seqlens,
                                int B, int H, int d_c, int d_r, int64_t cap,
                                float scale, int W, float* o_part, float* lse_part,
                                int* status, cudaStream_t stream) {
@@ -137,16 +139,18 @@ cudaError_t launch_decode_simt(const T* q_cat, const T* cache, const int32_t* se
                                        int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(W, (H + kSimtHeads - 1) / kSimtHeads);
-  kern<<<grid, kSimtHeads * 32, smem, stream>>>(q_cat, cache, seqlens, B, H, d_c, R,
+  kern<<<grid, kSimtHeads * 32, smem, stream>>>(q_cat, cache, pm, seqlens, B, H, d_c, R,
                                                  cap, scale, W, o_part, lse_part, status);
   return cudaGetLastError();
 }
 
-template cudaError_t launch_decode_simt<float>(const float*, const float*, const int32_t*,
+template cudaError_t launch_decode_simt<float>(const float*, const float*, const PageMap&,
+                                               const int32_t*,
                                                int, int, int, int, int64_t, float, int,
                                                float*, float*, int*, cudaStream_t);
 template cudaError_t launch_decode_simt<__nv_bfloat16>(const __nv_bfloat16*,
-                                                       const __nv_bfloat16*, const int32_t*,
+                                                       const __nv_bfloat16*, const PageMap&,
+                                                       const int32_t*,
                                                        int, int, int, int, int64_t, float,
                                                        int, float*, float*, int*,
                                                        cudaStream_t);

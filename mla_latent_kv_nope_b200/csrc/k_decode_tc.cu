@@ -168,6 +168,7 @@ __device__ __forceinline__ void for_each_segment(const TilePrefix& tp, int64_t t
 
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* __restrict__ cache,
+                 const PageMap pm,
                  const __nv_bfloat16* __restrict__ q_cat,
                  const int32_t* __restrict__ seqlens, int B, int H, int64_t cap,
                  float scale_log2, int W, float* __restrict__ o_part,
@@ -260,19 +261,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
         // One CTA per tile range (head group 0) pulls tiles into L2 ahead of
         // their loads: a tile's rows are one contiguous range of the cache,
         // so one bulk prefetch covers it (clamped to this sequence's rows).
-        const int64_t row0 = int64_t(b) * cap;
         auto prefetch = [&](int64_t t) {
           if (g != 0 || t >= hi) return;
-          const int64_t rows = min(int64_t(kTileKeys), cap - t * kTileKeys);
-          bulk_prefetch_l2(cache + (row0 + t * kTileKeys) * kR, uint32_t(rows * kR * 2));
+          const int64_t r = pm.tile_row(b, t);
+          if (r < 0) return;
+          const int64_t rows = pm.table ? int64_t(kTileKeys)
+                                        : min(int64_t(kTileKeys), cap - t * kTileKeys);
+          bulk_prefetch_l2(cache + r * kR, uint32_t(rows * kR * 2));
         };
         for (int64_t t = lo; t < hi; ++t, ++i) {
           const int s = i % kStages;
+          // The tile's first row (a page-table read when paged) is looked up
+          // before the stage wait so its latency hides behind it.  A page id
+          // outside the pool is reported and read as zeros (a row past the
+          // tensor map).
+          int64_t r = pm.tile_row(b, t);
           if (i >= kStages && !(ok = mbar_wait(&bars->empty[s], ((i / kStages) - 1) & 1,
                                                abort_flag, kWaitLimitCycles)))
             return false;
+          if (r < 0) {
+            record_status(status, MLA_ERR_BOUNDS);
+            r = pm.total_rows(B);
+          }
           mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
-          const int32_t crow = int32_t(row0 + t * kTileKeys);
+          const int32_t crow = int32_t(r);
           uint8_t* dst = sStage + s * kStageBytes;
           for (int c = 0; c < kChunks; ++c)
             tma_load_2d(&tm_c, &bars->full[s], dst + c * kChunkBytes, c * kChunkElems, crow);
@@ -601,13 +613,13 @@ bool make_cache_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
 int decode_tc_head_groups(int H) { return (H + kHeadsPerCta - 1) / kHeadsPerCta; }
 
 cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* cache,
-                             const int32_t* seqlens, int B, int H, int64_t cap, float scale,
-                             int W, float* o_part, float* lse_part, int* status,
+                             const PageMap& pm, const int32_t* seqlens, int B, int H, int64_t cap,
+                             float scale, int W, float* o_part, float* lse_part, int* status,
                              cudaStream_t stream) {
-  if (int64_t(B) * cap >= (int64_t(1) << 31) || int64_t(B) * H >= (int64_t(1) << 31))
+  if (pm.total_rows(B) >= (int64_t(1) << 31) || int64_t(B) * H >= (int64_t(1) << 31))
     return cudaErrorInvalidValue;
   CUtensorMap tm_c;
-  if (!make_cache_rows_map(&tm_c, cache, uint64_t(B) * uint64_t(cap))) return cudaErrorInvalidValue;
+  if (!make_cache_rows_map(&tm_c, cache, uint64_t(pm.total_rows(B)))) return cudaErrorInvalidValue;
   static bool attr_done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -620,7 +632,7 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
   }
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(decode_tc_head_groups(H), W);
-  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_c, cache, q_cat, seqlens, B, H, cap,
+  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_c, cache, pm, q_cat, seqlens, B, H, cap,
                                                            scale_log2, W, o_part, lse_part,
                                                            status);
   return cudaGetLastError();

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace mla {
 
 template <typename T>
@@ -15,7 +17,8 @@ cudaError_t launch_absorb_q(const T* q_nope, const T* q_pe, const T* W_UK,
                             int d_r, int d_n, T* q_cat, cudaStream_t stream);
 
 template <typename T>
-cudaError_t launch_decode_simt(const T* q_cat, const T* cache, const int32_t* seqlens,
+cudaError_t launch_decode_simt(const T* q_cat, const T* cache, const PageMap& pm,
+                               const int32_t* seqlens,
                                int B, int H, int d_c, int d_r, int64_t cap, float scale,
                                int W, float* o_part, float* lse_part, int* status,
                                cudaStream_t stream);
@@ -24,8 +27,8 @@ size_t decode_simt_smem_bytes(int d_c, int d_r);
 // Tensor-core decode (bf16, d_c = 512, d_r = 64).  Returns cudaErrorNotSupported
 // when the build has no sm_100a kernel.
 cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* cache,
-                             const int32_t* seqlens, int B, int H, int64_t cap, float scale,
-                             int W, float* o_part, float* lse_part, int* status,
+                             const PageMap& pm, const int32_t* seqlens, int B, int H, int64_t cap,
+                             float scale, int W, float* o_part, float* lse_part, int* status,
                              cudaStream_t stream);
 int decode_tc_head_groups(int H);
 // 2D TMA map over the cache viewed as [rows, 576] bf16: 64 x 64 boxes, 128-byte
@@ -44,14 +47,15 @@ cudaError_t launch_out_proj(const float* o_lat, const T* W_UV, int B, int H, int
 template <typename T>
 cudaError_t launch_cache_append(const T* h, const T* W_DKV, const float* gamma, float eps,
                                 float rope_base, int B, int d_c, int d_r, int hidden,
-                                int64_t cap, T* cache, int32_t* seqlens, float* x_ws,
-                                int* status, cudaStream_t stream);
+                                int64_t cap, T* cache, const PageMap& pm, int32_t* seqlens,
+                                float* x_ws, int* status, cudaStream_t stream);
 // Finalize only (norm, rotation, store, length bump) over n_parts partial sums
 // part[p][b][r] of the projection.
 template <typename T>
 cudaError_t launch_append_finalize(const float* part, int n_parts, const float* gamma, float eps,
                                    float rope_base, int B, int d_c, int d_r, int64_t cap,
-                                   T* cache, int32_t* seqlens, int* status, cudaStream_t stream);
+                                   T* cache, const PageMap& pm, int32_t* seqlens, int* status,
+                                   cudaStream_t stream);
 
 // Tensor-core kernels for the bf16 step (d_c = 512, d_r = 64, d_nope = d_v = 128).
 bool gemm_tc_supported(int d_c, int d_r, int d_n, int d_v);

@@ -59,16 +59,28 @@ int check_dims(const mla_dims* d) {
 inline bool decode_uses_tc(const mla_dims* d) { return d->dtype == MLA_BF16; }
 
 cudaError_t launch_decode_any(const mla_dims* d, const void* q_cat, const void* cache,
-                              const int32_t* seqlens, float scale, int W, float* o_part,
-                              float* lse_part, int* status, cudaStream_t s) {
+                              const PageMap& pm, const int32_t* seqlens, float scale, int W,
+                              float* o_part, float* lse_part, int* status, cudaStream_t s) {
   if (decode_uses_tc(d))
     return launch_decode_tc(static_cast<const __nv_bfloat16*>(q_cat),
-                            static_cast<const __nv_bfloat16*>(cache), seqlens, d->B, d->H,
+                            static_cast<const __nv_bfloat16*>(cache), pm, seqlens, d->B, d->H,
                             d->cache_capacity, scale, W, o_part, lse_part, status, s);
   return launch_decode_simt<float>(static_cast<const float*>(q_cat),
-                                   static_cast<const float*>(cache), seqlens, d->B, d->H, d->d_c,
-                                   d->d_r, d->cache_capacity, scale, W, o_part, lse_part, status,
-                                   s);
+                                   static_cast<const float*>(cache), pm, seqlens, d->B, d->H,
+                                   d->d_c, d->d_r, d->cache_capacity, scale, W, o_part, lse_part,
+                                   status, s);
+}
+
+PageMap contiguous_map(const mla_dims* d) { return PageMap{nullptr, 0, 0, d->cache_capacity}; }
+
+// Checks of a page table argument: capacity covered by max_blocks pages.
+int check_pages(const mla_dims* d, int64_t num_pages, const int32_t* block_table,
+                int32_t max_blocks) {
+  if (!block_table || num_pages <= 0 || max_blocks <= 0) return MLA_ERR_INVALID_ARG;
+  if (d->cache_capacity > int64_t(max_blocks) * kTileKeys) return MLA_ERR_INVALID_ARG;
+  if (num_pages * kTileKeys >= (int64_t(1) << 31)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(block_table)) return MLA_ERR_ALIGNMENT;
+  return MLA_OK;
 }
 
 int decode_shape_supported(const mla_dims* d) {
@@ -143,9 +155,11 @@ size_t mla_cache_append_workspace_bytes(const mla_dims* d, int32_t hidden) {
   return round_up(parts * size_t(d->B) * size_t(d->d_c + d->d_r) * sizeof(float), 256);
 }
 
-int mla_cache_append(const mla_dims* d, int32_t hidden, const void* h, const void* W_DKV,
-                     const float* gamma, float eps, float rope_base, void* cache,
-                     int32_t* seqlens, void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+int cache_append_impl(const mla_dims* d, int32_t hidden, const void* h, const void* W_DKV,
+                      const float* gamma, float eps, float rope_base, void* cache,
+                      const PageMap& pm, int32_t* seqlens, void* workspace,
+                      size_t workspace_bytes, void* stream) {
   int st = check_dims(d);
   if (st) return st;
   if (hidden <= 0 || !h || !W_DKV || !cache || !seqlens) return MLA_ERR_INVALID_ARG;
@@ -165,17 +179,43 @@ int mla_cache_append(const mla_dims* d, int32_t hidden, const void* h, const voi
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     return cuda_status(launch_append_finalize<__nv_bfloat16>(
         x, append_tc_splits(hidden), gamma, eps, rope_base, d->B, d->d_c, d->d_r,
-        d->cache_capacity, static_cast<__nv_bfloat16*>(cache), seqlens, status_ptr(), s));
+        d->cache_capacity, static_cast<__nv_bfloat16*>(cache), pm, seqlens, status_ptr(), s));
   }
   if (d->dtype == MLA_BF16)
     return cuda_status(launch_cache_append<__nv_bfloat16>(
         static_cast<const __nv_bfloat16*>(h), static_cast<const __nv_bfloat16*>(W_DKV), gamma,
         eps, rope_base, d->B, d->d_c, d->d_r, hidden, d->cache_capacity,
-        static_cast<__nv_bfloat16*>(cache), seqlens, x, status_ptr(), s));
+        static_cast<__nv_bfloat16*>(cache), pm, seqlens, x, status_ptr(), s));
   return cuda_status(launch_cache_append<float>(
       static_cast<const float*>(h), static_cast<const float*>(W_DKV), gamma, eps, rope_base,
-      d->B, d->d_c, d->d_r, hidden, d->cache_capacity, static_cast<float*>(cache), seqlens, x,
-      status_ptr(), s));
+      d->B, d->d_c, d->d_r, hidden, d->cache_capacity, static_cast<float*>(cache), pm, seqlens,
+      x, status_ptr(), s));
+}
+
+int decode_impl(const mla_dims* d, const void* q_cat, const void* cache, const PageMap& pm,
+                const int32_t* seqlens, float softmax_scale, int num_splits, void* workspace,
+                size_t workspace_bytes, int* splits_used, void* stream);
+}  // namespace
+
+int mla_cache_append(const mla_dims* d, int32_t hidden, const void* h, const void* W_DKV,
+                     const float* gamma, float eps, float rope_base, void* cache,
+                     int32_t* seqlens, void* workspace, size_t workspace_bytes, void* stream) {
+  if (check_dims(d)) return check_dims(d);
+  return cache_append_impl(d, hidden, h, W_DKV, gamma, eps, rope_base, cache, contiguous_map(d),
+                           seqlens, workspace, workspace_bytes, stream);
+}
+
+int mla_cache_append_paged(const mla_dims* d, int32_t hidden, const void* h, const void* W_DKV,
+                           const float* gamma, float eps, float rope_base, void* cache_pool,
+                           int64_t num_pages, const int32_t* block_table, int32_t max_blocks,
+                           int32_t* seqlens, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if ((st = check_pages(d, num_pages, block_table, max_blocks))) return st;
+  return cache_append_impl(d, hidden, h, W_DKV, gamma, eps, rope_base, cache_pool,
+                           PageMap{block_table, max_blocks, num_pages, d->cache_capacity}, seqlens,
+                           workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -229,9 +269,10 @@ size_t mla_decode_workspace_bytes(const mla_dims* d, int num_splits) {
   return ws_layout(d, W).total;
 }
 
-int mla_decode(const mla_dims* d, const void* q_cat, const void* cache, const int32_t* seqlens,
-               float softmax_scale, int num_splits, void* workspace, size_t workspace_bytes,
-               int* splits_used, void* stream) {
+namespace {
+int decode_impl(const mla_dims* d, const void* q_cat, const void* cache, const PageMap& pm,
+                const int32_t* seqlens, float softmax_scale, int num_splits, void* workspace,
+                size_t workspace_bytes, int* splits_used, void* stream) {
   int st = check_dims(d);
   if (st) return st;
   if ((st = decode_shape_supported(d))) return st;
@@ -249,8 +290,29 @@ int mla_decode(const mla_dims* d, const void* q_cat, const void* cache, const in
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + l.o_off);
   float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + l.lse_off);
-  return cuda_status(launch_decode_any(d, q_cat, cache, seqlens, softmax_scale, W, o_part,
+  return cuda_status(launch_decode_any(d, q_cat, cache, pm, seqlens, softmax_scale, W, o_part,
                                        lse_part, status_ptr(), s));
+}
+}  // namespace
+
+int mla_decode(const mla_dims* d, const void* q_cat, const void* cache, const int32_t* seqlens,
+               float softmax_scale, int num_splits, void* workspace, size_t workspace_bytes,
+               int* splits_used, void* stream) {
+  if (check_dims(d)) return check_dims(d);
+  return decode_impl(d, q_cat, cache, contiguous_map(d), seqlens, softmax_scale, num_splits,
+                     workspace, workspace_bytes, splits_used, stream);
+}
+
+int mla_decode_paged(const mla_dims* d, const void* q_cat, const void* cache_pool,
+                     int64_t num_pages, const int32_t* block_table, int32_t max_blocks,
+                     const int32_t* seqlens, float softmax_scale, int num_splits,
+                     void* workspace, size_t workspace_bytes, int* splits_used, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if ((st = check_pages(d, num_pages, block_table, max_blocks))) return st;
+  return decode_impl(d, q_cat, cache_pool,
+                     PageMap{block_table, max_blocks, num_pages, d->cache_capacity}, seqlens,
+                     softmax_scale, num_splits, workspace, workspace_bytes, splits_used, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -350,8 +412,8 @@ extern "C" int mla_decode_noalloc(const mla_dims* d, const void* q_cat, const vo
   float* o_part = reinterpret_cast<float*>(static_cast<char*>(scratch) + l.o_off);
   float* lse_part = reinterpret_cast<float*>(static_cast<char*>(scratch) + l.lse_off);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const cudaError_t e = launch_decode_any(d, q_cat, cache, seqlens, softmax_scale, W, o_part,
-                                          lse_part, status_ptr(), s);
+  const cudaError_t e = launch_decode_any(d, q_cat, cache, contiguous_map(d), seqlens,
+                                          softmax_scale, W, o_part, lse_part, status_ptr(), s);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   return cuda_status(launch_combine(seqlens, d->cache_capacity, d->B, d->H, d->d_c, W, o_part,
                                     lse_part, o_lat, lse, s));

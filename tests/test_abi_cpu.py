@@ -135,6 +135,29 @@ def test_other_entry_point_errors(lib):
     assert ap(ws=None) == WS
 
 
+def test_paged_entry_point_errors(lib):
+    d = _dims(cache_capacity=4096)          # 64 pages of 64 rows per sequence at most
+    need = lib.mla_decode_workspace_bytes(ctypes.byref(d), 8)
+    used = ctypes.c_int(-1)
+    dp = lambda pool=GOOD, npages=100, table=GOOD2, mb=64, ws=GOOD2, n=need: lib.mla_decode_paged(  # noqa: E731
+        ctypes.byref(d), GOOD, pool, npages, table, mb, GOOD, 0.07, 8, ws, n, ctypes.byref(used),
+        None)
+    assert dp(table=None) == INVALID
+    assert dp(npages=0) == INVALID
+    assert dp(mb=63) == INVALID              # 63 pages cannot hold 4096 rows
+    assert dp(table=BAD) == ALIGN
+    assert dp(pool=BAD) == ALIGN
+    assert dp(npages=1 << 26) == UNSUP       # rows of the pool beyond a 32-bit TMA coordinate
+    assert dp(n=need - 1) == WS
+    wsb = lib.mla_cache_append_workspace_bytes(ctypes.byref(d), 7168)
+    ap = lambda table=GOOD2, mb=64: lib.mla_cache_append_paged(  # noqa: E731
+        ctypes.byref(d), 7168, GOOD, GOOD, None, 1e-6, 1e4, GOOD, 100, table, mb, GOOD, GOOD2,
+        wsb, None)
+    assert ap(table=None) == INVALID
+    assert ap(mb=10) == INVALID
+    assert used.value == -1
+
+
 def _deal(lens, W, tile=64):
     """Host restatement of the documented split-KV dealing: worker w takes
     tiles [w*T//W, (w+1)*T//W) of the concatenated per-sequence tiles."""

@@ -189,6 +189,106 @@ def test_decode_combine(name, w, lens, nsplit, boost):
     assert _lse_err(got_l, ref_l) < tol(w)
 
 
+def _paged_copy(cache, seed=7, spare=5):
+    """The contiguous cache [B, cap, R] (cap a multiple of 64) as a shuffled
+    pool of 64-row pages with spare pages, and its block table."""
+    B, cap, R = cache.shape
+    nb = cap // mla.PAGE_ROWS
+    n_pages = B * nb + spare
+    perm = torch.from_numpy(np.random.default_rng(seed).permutation(n_pages)[:B * nb]).cuda()
+    pool = torch.full((n_pages, mla.PAGE_ROWS, R), float("nan"), dtype=cache.dtype,
+                      device="cuda")
+    pool[perm] = cache.reshape(B * nb, mla.PAGE_ROWS, R)
+    table = perm.to(torch.int32).reshape(B, nb).contiguous()
+    return pool, table
+
+
+PAGED_CASES = [
+    ("bf16-H128", W["v3_bf16"].scaled(B=3, N=600), [600, 129, 1], 0),
+    ("bf16-H64-W7", W["ragged_append_bf16"].scaled(B=5, N=700), [700, 1, 333, 64, 0], 7),
+    ("f32-tiny", W["tiny_f32"].scaled(B=3), [64, 1, 130], 3),
+]
+
+
+@pytest.mark.parametrize("name,w,lens,nsplit", PAGED_CASES, ids=[c[0] for c in PAGED_CASES])
+def test_paged_decode_matches_contiguous(name, w, lens, nsplit):
+    """The paged decode reads the same rows through the block table: its
+    partials, merged, are bit-identical to the contiguous decode's, and both
+    match the oracle."""
+    lens = np.array(lens, dtype=np.int32)
+    cap = (int(lens.max()) + 63) // 64 * 64
+    d = dims_of(w, capacity=cap)
+    cache = device_cache(w, lens, capacity=cap, fill_rest=float("nan"))
+    pool, table = _paged_copy(cache)
+    seq = torch.from_numpy(lens).cuda()
+    q_cat = inputs.normal((w.B, w.H, w.R), 0.5, 31, len(lens))
+    qd = dev(q_cat, w)
+    Wn = nsplit or mla.decode_default_splits(d)
+    outs = []
+    for paged in (False, True):
+        ws = torch.full((mla.decode_workspace_bytes(d, Wn) // 4,), float("nan"), device="cuda")
+        if paged:
+            used = mla.decode_paged(d, qd, pool, table, seq, w.softmax_scale, ws, Wn)
+        else:
+            used = mla.decode(d, qd, cache, seq, w.softmax_scale, ws, Wn)
+        o_lat = torch.empty(w.B, w.H, w.d_c, device="cuda")
+        lse = torch.empty(w.B, w.H, device="cuda")
+        mla.combine(d, seq, ws, used, o_lat, lse)
+        assert mla.get_device_status() == 0
+        outs.append((o_lat, lse))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    ref_o, ref_l = _oracle_latent(w, lens, q_cat, w.softmax_scale)
+    nz = lens > 0
+    assert rel_l2(f64(outs[1][0])[nz], ref_o[nz]) < tol(w)
+    assert _lse_err(f64(outs[1][1]), ref_l) < tol(w)
+
+
+@pytest.mark.parametrize("w", [W["ragged_append_bf16"].scaled(B=5, N=300, hidden=512),
+                               W["tiny_f32"].scaled(B=3, hidden=64)], ids=["bf16", "f32"])
+def test_paged_append_matches_contiguous(w):
+    """Appending through the block table writes the same bytes into the page
+    that holds row L_b, and nothing else; lengths advance the same way."""
+    lens = inputs.seqlens(w)
+    cap = (int(lens.max()) + 1 + 63) // 64 * 64
+    d = dims_of(w, capacity=cap)
+    cache = device_cache(w, lens, capacity=cap, fill_rest=float("nan"))
+    pool, table = _paged_copy(cache)
+    h, Wdkv = inputs.append_inputs(w)
+    hd, Wd = dev(h, w), dev(Wdkv, w)
+    ws = torch.empty(mla.cache_append_workspace_bytes(d, w.hidden) // 4, device="cuda")
+    seq_a = torch.from_numpy(lens).cuda()
+    seq_b = seq_a.clone()
+    mla.cache_append(d, hd, Wd, None, cache, seq_a, ws)
+    pool_before = pool.clone()
+    mla.cache_append_paged(d, hd, Wd, None, pool, table, seq_b, ws)
+    assert mla.get_device_status() == 0
+    assert torch.equal(seq_a, seq_b)
+    gathered = pool[table.long().reshape(-1)].reshape(w.B, cap, w.R)
+    assert torch.equal(gathered.view(torch.int16 if w.dtype == "bf16" else torch.int32),
+                       cache.view(torch.int16 if w.dtype == "bf16" else torch.int32))
+    # the spare pages are untouched
+    used_pages = set(table.reshape(-1).tolist())
+    spare = [p for p in range(pool.shape[0]) if p not in used_pages]
+    assert torch.equal(pool[spare].isnan(), pool_before[spare].isnan())
+
+
+def test_paged_bad_page_is_reported():
+    """A page id outside the pool is never dereferenced: the decode reads zeros
+    for it and the status word reports MLA_ERR_BOUNDS."""
+    w = W["v3_bf16"].scaled(B=2, N=128)
+    lens = np.array([128, 64], dtype=np.int32)
+    d = dims_of(w, capacity=128)
+    cache = device_cache(w, lens, capacity=128)
+    pool, table = _paged_copy(cache)
+    table[0, 1] = pool.shape[0] + 3           # outside the pool
+    seq = torch.from_numpy(lens).cuda()
+    ws = torch.empty(mla.decode_workspace_bytes(d, 4) // 4, device="cuda")
+    mla.decode_paged(d, dev(inputs.normal((2, w.H, w.R), 0.5, 1, 1), w), pool, table, seq,
+                     w.softmax_scale, ws, 4)
+    assert mla.get_device_status() == 7      # MLA_ERR_BOUNDS
+    assert mla.get_device_status() == 0
+
+
 def test_combine_alone():
     """Synthetic partials placed in the documented workspace slots; the merge
     must equal the log-sum-exp combination of exactly those partials."""
