@@ -81,9 +81,11 @@ while True:
 
 
 class ClockSampler:
-    """SM clock and throttle reasons sampled through NVML every ~2 ms by a
-    separate process; only samples inside the [start, stop] window of the
-    timed steps are kept."""
+    """SM clock and throttle reasons sampled through NVML during the timed
+    steps: every ~2 ms by a separate process (samples inside the [start, stop]
+    window kept), and, while the GPU is still working through the enqueued
+    steps, by this process itself (``poll_until``), so even a short timed
+    region is sampled."""
     REASONS = {  # NVML clocks-event-reason bits
         0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
         0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown",
@@ -92,6 +94,23 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.t_start = self.t_stop = None
+        self.inproc = []   # (sm_mhz, reasons) read while the timed steps ran
+
+    def poll_until(self, done, nvml=None, max_samples=100000):
+        """Read the SM clock and throttle reasons until ``done()`` is true (the
+        end-of-timing event has completed).  Never raises: on any NVML error
+        the process sampler's readings stand alone."""
+        try:
+            if nvml is None:
+                import pynvml as nvml
+            nvml.nvmlInit()
+            h = nvml.nvmlDeviceGetHandleByIndex(int(self.index))
+            while len(self.inproc) < max_samples and not done():
+                self.inproc.append((int(nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM)),
+                                    int(nvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                time.sleep(0.0002)
+        except Exception:
+            pass
 
     def __enter__(self):
         import subprocess
@@ -122,7 +141,7 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        rows = []
+        rows = list(self.inproc)
         for ln in getattr(self, "lines", []):
             f = ln.split()
             if len(f) != 3:
@@ -139,9 +158,10 @@ class ClockSampler:
             for bit, name in self.REASONS.items():
                 if rs & bit:
                     reasons.add(name)
-        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": self.max_mhz,
+        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": getattr(self, "max_mhz", None),
                 "sm_min_mhz": sms[0], "samples": len(rows), "reasons": sorted(reasons),
-                "source": "NVML from a separate process, ~2 ms period, timed window only"}
+                "source": "NVML during the timed steps (this process while they run, and a "
+                          "separate process every ~2 ms inside the window)"}
 
 
 # ---------------------------------------------------------------------------
@@ -267,6 +287,7 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(args.steps):
             one_step()
         t1.record(stream)
+        clk.poll_until(t1.query)
         torch.cuda.synchronize()
         clk.stop()
         barrier()
