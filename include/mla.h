@@ -74,7 +74,7 @@ typedef struct {
 enum {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive or inconsistent size */
-  MLA_ERR_UNSUPPORTED = 2,    /* shape/dtype this build has no kernel for */
+  MLA_ERR_UNSUPPORTED = 2,    /* shape/dtype the library has no kernel for */
   MLA_ERR_ALIGNMENT = 3,      /* a pointer is not 16-byte aligned */
   MLA_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
   MLA_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
