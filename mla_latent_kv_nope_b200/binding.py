@@ -143,15 +143,19 @@ def _need(t, dtype, shape, name):
 
 # ---------------------------------------------------------------------------
 def cache_row_elems(d_c: int, d_r: int) -> int:
+    """Elements of one latent cache row, d_c + d_r (mla_cache_row_elems)."""
     return int(load_library().mla_cache_row_elems(d_c, d_r))
 
 
 def cache_append_workspace_bytes(dims: Dims, hidden: int) -> int:
+    """Bytes of fp32 workspace mla_cache_append needs for this hidden size."""
     return int(load_library().mla_cache_append_workspace_bytes(ctypes.byref(dims.c()), hidden))
 
 
 def cache_append(dims: Dims, h, W_DKV, gamma, cache, seqlens, workspace, eps=1e-6,
                  rope_base=10000.0, stream=None):
+    """mla_cache_append: write row L_b = [RMSNorm(W^DKV h) * gamma || RoPE(W^KR h, L_b)]
+    of every sequence and increment L_b (cache [B, capacity, R])."""
     dt = dims.torch_dtype
     hidden = h.shape[-1]
     _need(h, dt, (dims.B, hidden), "h")
@@ -213,6 +217,8 @@ def decode_paged(dims: Dims, q_cat, cache_pool, block_table, seqlens, softmax_sc
 
 
 def absorb_q(dims: Dims, q_nope, q_pe, W_UK, q_pos, q_cat, rope_base=10000.0, stream=None):
+    """mla_absorb_q: q_cat[b,i] = [W^UK_i^T q_nope[b,i] ; RoPE(q_pe[b,i], q_pos[b])]
+    (no rotation when q_pos is None)."""
     dt = dims.torch_dtype
     _need(q_nope, dt, (dims.B, dims.H, dims.d_nope), "q_nope")
     _need(q_pe, dt, (dims.B, dims.H, dims.d_r), "q_pe")
@@ -227,15 +233,19 @@ def absorb_q(dims: Dims, q_nope, q_pe, W_UK, q_pos, q_cat, rope_base=10000.0, st
 
 
 def decode_default_splits(dims: Dims) -> int:
+    """The split count mla_decode uses on the current device when asked for 0."""
     return int(load_library().mla_decode_default_splits(ctypes.byref(dims.c())))
 
 
 def decode_workspace_bytes(dims: Dims, num_splits: int = 0) -> int:
+    """Bytes of workspace mla_decode needs for this many splits (0 = default)."""
     return int(load_library().mla_decode_workspace_bytes(ctypes.byref(dims.c()), num_splits))
 
 
 def decode(dims: Dims, q_cat, cache, seqlens, softmax_scale, workspace, num_splits=0,
            stream=None) -> int:
+    """mla_decode: split-KV latent attention of q_cat over the cache; writes the
+    partials into ``workspace`` and returns the number of splits used."""
     dt = dims.torch_dtype
     _need(q_cat, dt, (dims.B, dims.H, dims.R), "q_cat")
     _need(cache, dt, (dims.B, dims.cache_capacity, dims.R), "cache")
@@ -250,6 +260,8 @@ def decode(dims: Dims, q_cat, cache, seqlens, softmax_scale, workspace, num_spli
 
 
 def combine(dims: Dims, seqlens, workspace, splits_used, o_lat, lse=None, stream=None):
+    """mla_combine: log-sum-exp merge of the partials into o_lat [B,H,d_c] fp32 (and
+    lse [B,H] fp32 when given)."""
     _need(o_lat, torch.float32, (dims.B, dims.H, dims.d_c), "o_lat")
     if lse is not None:
         _need(lse, torch.float32, (dims.B, dims.H), "lse")
@@ -260,6 +272,7 @@ def combine(dims: Dims, seqlens, workspace, splits_used, o_lat, lse=None, stream
 
 
 def out_proj(dims: Dims, o_lat, W_UV, out, stream=None):
+    """mla_out_proj: out[b,i] = W^UV_i o_lat[b,i]."""
     dt = dims.torch_dtype
     _need(o_lat, torch.float32, (dims.B, dims.H, dims.d_c), "o_lat")
     _need(W_UV, dt, (dims.H, dims.d_v, dims.d_c), "W_UV")
@@ -270,6 +283,7 @@ def out_proj(dims: Dims, o_lat, W_UV, out, stream=None):
 
 
 def get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
     return int(load_library().mla_get_device_status(_stream(stream)))
 
 
