@@ -19,8 +19,10 @@ Sources (cited by page title and section, as the pages name them):
   "Decoupled RoPE", "KVキャッシュ容量の比較", "実装上のトレードオフ".
 * [attention-variants] youngju.dev "model internals: attention variants",
   sections "MLA: キャッシュする対象そのものを変える" and "一つの表で比べる".
-* [yuuk-wiki] notes.yuuk.io wiki "Multi-Head Latent Attention", section
-  "横断的知見" (MQA as the special case of MLA).
+* [yuuk-wiki] notes.yuuk.io wiki "Multi-Head Latent Attention", sections
+  "横断的知見" (MQA as the special case of MLA) and "未解決の問い" (FP8/FP4).
+* [abeam] abeam.tech "Multi-Head Latent Attention" (DeepSeek-V2 reading),
+  section "モデル全体でも推論効率が大きく改善した" (KV-cache quantisation).
 
 Conventions (column vectors, y = W x, as [MLA-とは] states in its preamble):
 
@@ -57,6 +59,15 @@ __all__ = [
     "latent_attention",
     "combine_partials",
     "out_proj",
+    "output_projection",
+    "fold_output_weights",
+    "folded_output",
+    "E4M3_MAX",
+    "e4m3_decode",
+    "e4m3_encode",
+    "latent_row_scale",
+    "quantize_latent_rows",
+    "dequantize_latent_rows",
     "cache_elems_per_token",
     "mults_per_cached_token",
 ]
@@ -331,6 +342,133 @@ def out_proj(o_lat, W_UV) -> np.ndarray:
     after the latent-space weighted sum ([MLA-とは] "Value側の吸収", second
     equation for o_{t,i}).  o_lat: [B,H,d_c]; W_UV: [H,d_v,d_c] -> [B,H,d_v]."""
     return np.einsum("ivd,bid->biv", _f64(W_UV), _f64(o_lat))
+
+
+# ---------------------------------------------------------------------------
+# Output projection W^O, and its fold with W^UV
+# ---------------------------------------------------------------------------
+def output_projection(out, W_O) -> np.ndarray:
+    """u[b] = sum_i W^O_i out[b,i], where W^O_i in R^{d x d_v} is the column
+    block of W^O that belongs to head i ([MLA-とは] "Value側の吸収", the
+    equation for u_t, left-hand form).
+
+    out: [B, H, d_v]; W_O: [d, H*d_v] (column convention, u = W^O o with the
+    heads' outputs concatenated) -> u [B, d]."""
+    out, W_O = _f64(out), _f64(W_O)
+    B, H, d_v = out.shape
+    u = np.zeros((B, W_O.shape[0]))
+    for i in range(H):
+        u += out[:, i, :] @ W_O[:, i * d_v:(i + 1) * d_v].T
+    return u
+
+
+def fold_output_weights(W_O, W_UV) -> np.ndarray:
+    """B_i = W^O_i W^UV_i in R^{d x d_c}: W^UV absorbed into the output
+    projection once, at load time ([MLA-とは] "Value側の吸収", the
+    definition of B_i under the equation for u_t).
+
+    W_O: [d, H*d_v]; W_UV: [H, d_v, d_c] -> B [H, d, d_c]."""
+    W_O, W_UV = _f64(W_O), _f64(W_UV)
+    H, d_v, _ = W_UV.shape
+    return np.stack([W_O[:, i * d_v:(i + 1) * d_v] @ W_UV[i]
+                     for i in range(H)])
+
+
+def folded_output(o_lat, B_fold) -> np.ndarray:
+    """u[b] = sum_i B_i o_lat[b,i]: the latent-space weighted sums go straight
+    through the folded weights ([MLA-とは] "Value側の吸収", the right-hand form
+    of the equation for u_t).  o_lat: [B, H, d_c]; B_fold: [H, d, d_c] -> [B, d]."""
+    return np.einsum("idc,bic->bd", _f64(B_fold), _f64(o_lat))
+
+
+# ---------------------------------------------------------------------------
+# FP8 latent cache: E4M3 codes for c^KV with one power-of-two scale per token
+#
+# The pages name KV-cache quantisation ([abeam] "モデル全体でも推論効率が大きく
+# 改善した") and FP8 for MLA as an open question ([yuuk-wiki] "未解決の問い")
+# without fixing a format.  The reading taken here: c^KV is stored as OCP FP8
+# E4M3 codes (the finite-only variant, largest magnitude 448), each cached
+# token carries one scale 2^k chosen so that its largest |c| fits under 448,
+# and the decoupled key k^R stays in the 16-bit cache type.  A per-token
+# scale keeps an append a purely local write; a power-of-two scale makes
+# code * scale exact in bf16, so the only rounding is the E4M3 one.
+# ---------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each E4M3 byte, from the format's definition: bit 7 the sign,
+    bits 6..3 the exponent field e (bias 7), bits 2..0 the mantissa m.
+    e = 0 is subnormal, m/8 * 2^-6; otherwise (1 + m/8) * 2^(e-7); the one
+    pattern e = 15, m = 7 is NaN (there are no infinities)."""
+    code = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(code & 0x80, -1.0, 1.0)
+    e = (code >> 3) & 0xF
+    m = (code & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6,
+                   (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    mag = np.where((e == 15) & (code & 0x7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 code of each value, rounded to nearest with ties to even and
+    saturated to +-448 (finite inputs above 448, and infinities, give the
+    largest code of their sign; NaN gives 0x7F).  The sign bit follows the
+    input's sign, so a negative value that rounds to zero gives 0x80.
+
+    The magnitude is rounded on the grid of its binade: spacing 2^(E-3) for
+    2^E <= |x| < 2^(E+1) with E >= -6, and 2^-9 below 2^-6 (subnormals)."""
+    x = _f64(x)
+    neg = np.signbit(x)
+    a = np.minimum(np.abs(x), E4M3_MAX)          # saturate (inf included)
+    nan = np.isnan(x)
+    a = np.where(nan, 0.0, a)
+    _, k = np.frexp(a)                            # a = f 2^k, f in [0.5, 1)
+    E = np.maximum(k - 1, -6)
+    quantum = np.exp2((E - 3).astype(np.float64))
+    r = np.round(a / quantum) * quantum           # numpy rounds ties to even
+    # Back to the bit pattern of r (r <= 448 is always representable).
+    _, k2 = np.frexp(r)
+    E2 = k2 - 1
+    sub = r < 2.0 ** -6
+    mant_sub = np.round(r / 2.0 ** -9).astype(np.int64)
+    field = np.where(sub, 0, E2 + 7).astype(np.int64)
+    mant_norm = np.round((r / np.exp2(E2.astype(np.float64)) - 1.0) * 8.0)
+    mant = np.where(sub, mant_sub, mant_norm.astype(np.int64))
+    code = (field << 3) | mant
+    code = np.where(neg, code | 0x80, code)
+    code = np.where(nan, 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def latent_row_scale(c) -> np.ndarray:
+    """Per-token scale 2^k with k the smallest integer such that
+    max_j |c_j| / 2^k <= 448; a row of zeros gets scale 1.
+    c: [..., d_c] -> [...] float64 (exact powers of two)."""
+    c = _f64(c)
+    amax = np.max(np.abs(c), axis=-1)
+    safe = np.where(amax > 0, amax, E4M3_MAX)
+    k = np.ceil(np.log2(safe / E4M3_MAX))
+    # Guard the log2 rounding at exact binade edges: settle k by comparison.
+    k = np.where(safe / np.exp2(k) > E4M3_MAX, k + 1, k)
+    k = np.where(safe / np.exp2(k - 1) <= E4M3_MAX, k - 1, k)
+    return np.exp2(k)
+
+
+def quantize_latent_rows(c):
+    """(codes, scale) of each cached latent: scale = latent_row_scale(c) and
+    codes = E4M3(c / scale).  Division by a power of two is exact, so each
+    code is the E4M3 rounding of the latent value itself.
+    c: [..., d_c] -> codes uint8 [..., d_c], scale float64 [...]."""
+    c = _f64(c)
+    scale = latent_row_scale(c)
+    return e4m3_encode(c / scale[..., None]), scale
+
+
+def dequantize_latent_rows(codes, scale) -> np.ndarray:
+    """c~ = E4M3 value of each code times its token's scale (float64, exact)."""
+    return e4m3_decode(codes) * _f64(scale)[..., None]
 
 
 # ---------------------------------------------------------------------------

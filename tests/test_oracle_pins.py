@@ -5,6 +5,7 @@ Each test names the passage it pins.  Page keys:
   [MLA-とは]  disassemble-channel.com "Multi-head Latent Attention（MLA）とは？"
   [variants] youngju.dev "model internals: attention variants"
   [yuuk]     notes.yuuk.io wiki "Multi-Head Latent Attention"
+  [abeam]    abeam.tech "Multi-Head Latent Attention" (DeepSeek-V2 reading)
 """
 import json
 import math
@@ -529,3 +530,179 @@ def test_cache_size_closed_forms():
     h = O.mults_per_cached_token("MHA", m["n_h"], m["d_h"], m["d_c"])
     assert (n, a, h) == (m["naive"], m["absorbed"], m["MHA"])
     assert a // h == m["absorbed_over_MHA"] and n // a == m["naive_over_absorbed"]
+
+
+# ---------------------------------------------------------------------------
+# W^O fold: B_i = W^O_i W^UV_i ([MLA-とは] "Value側の吸収")
+# ---------------------------------------------------------------------------
+def test_output_fold_matches_pages_value_side(pages, gold):
+    """[MLA-とは] 数値検証 (Value側): projecting the materialised per-head
+    outputs through W^O equals pushing the latent sums through the folded
+    B_i; the page prints a float64 gap of about 1.1e-15."""
+    x = pages
+    d, d_c, d_cq, d_h, n_h, T, d_r = x["dims"]
+    P = x["attn"]
+    W_O = x["w_o"].T  # snippet's row-vector [n_h*d_h, d] -> column [d, n_h*d_h]
+    out = np.zeros((T, n_h, d_h))
+    o_lat = np.zeros((T, n_h, d_c))
+    for t in range(T):
+        for i in range(n_h):
+            out[t, i] = O.materialised_values(P[t, :, i], x["c_kv"], x["W_UV"][i])
+            o_lat[t, i] = P[t, :, i] @ x["c_kv"]
+    u_unfolded = O.output_projection(out, W_O)
+    Bf = O.fold_output_weights(W_O, x["W_UV"])
+    assert Bf.shape == (n_h, d, d_c)  # B_i in R^{d x d_c}, as the page states
+    u_folded = O.folded_output(o_lat, Bf)
+    # The page's own naive path, written independently of the oracle.
+    V = (x["c_kv"] @ x["w_uv"]).reshape(T, n_h, d_h)
+    u_page = np.einsum("tji,jih->tih", P, V).reshape(T, n_h * d_h) @ x["w_o"]
+    assert np.abs(u_unfolded - u_page).max() < 1e-12
+    err = np.abs(u_folded - u_page).max()
+    assert err < 1e-12
+    assert gold["value_side_max_abs_err"] < 1e-12
+
+
+def test_output_fold_special_cases():
+    """W^UV_i = I (d_v = d_c) leaves W^O's head blocks unchanged; a W^O that
+    selects one head's output returns that head's W^UV; the fold's rank is at
+    most d_v (it factors through a d_v-dimensional space)."""
+    rng = np.random.default_rng(21)
+    H, d, d_c = 3, 7, 5
+    W_O = rng.normal(size=(d, H * d_c))
+    Bf = O.fold_output_weights(W_O, np.stack([np.eye(d_c)] * H))
+    for i in range(H):
+        np.testing.assert_array_equal(Bf[i], W_O[:, i * d_c:(i + 1) * d_c])
+    d_v = 2
+    W_UV = rng.normal(size=(H, d_v, d_c))
+    sel = np.zeros((d_v, H * d_v))
+    sel[:, d_v:2 * d_v] = np.eye(d_v)  # picks head 1
+    Bs = O.fold_output_weights(sel, W_UV)
+    np.testing.assert_array_equal(Bs[1], W_UV[1])
+    assert np.all(Bs[0] == 0) and np.all(Bs[2] == 0)
+    Bg = O.fold_output_weights(rng.normal(size=(d, H * d_v)), W_UV)
+    assert all(np.linalg.matrix_rank(Bg[i]) <= d_v for i in range(H))
+    # Brute force: u = sum_i sum_a sum_c W_O[:, i*d_v + a] W_UV[i, a, c] o[i, c].
+    o = rng.normal(size=(1, H, d_c))
+    W_O2 = rng.normal(size=(d, H * d_v))
+    u = O.folded_output(o, O.fold_output_weights(W_O2, W_UV))[0]
+    ref = [sum(W_O2[r, i * d_v + a] * W_UV[i, a, c] * o[0, i, c]
+               for i in range(H) for a in range(d_v) for c in range(d_c))
+           for r in range(d)]
+    np.testing.assert_allclose(u, ref, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# FP8 latent cache: E4M3 codes with a power-of-two scale per token.  The pages
+# name KV quantisation ([abeam] "モデル全体でも推論効率が大きく改善した") and
+# FP8 for MLA ([yuuk] "未解決の問い") but no format; the format is a reading,
+# and these pins fix the oracle to the E4M3 definition it states.
+# ---------------------------------------------------------------------------
+def test_e4m3_decode_table():
+    """Every byte against the format's closed-form values and against torch's
+    float8_e4m3fn (a library routine)."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    v = O.e4m3_decode(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    nan = np.isnan(v)
+    np.testing.assert_array_equal(nan, np.isnan(lib))
+    np.testing.assert_array_equal(v[~nan], lib[~nan].astype(np.float64))
+    assert list(np.flatnonzero(nan)) == [0x7F, 0xFF]
+    spot = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6,
+            0x38: 1.0, 0x39: 1.125, 0x40: 2.0, 0x7E: 448.0, 0xB8: -1.0,
+            0xFE: -448.0, 0x80: 0.0}
+    for c, val in spot.items():
+        assert v[c] == val, hex(c)
+    pos = v[:0x7F]
+    assert np.all(np.diff(pos) > 0)  # the positive codes are ordered
+    np.testing.assert_array_equal(v[0x80:0xFF], -v[:0x7F])
+
+
+def test_e4m3_encode_rounding_and_saturation():
+    """Round-trip of every finite code; ties to even at each midpoint; one
+    float32 ulp either side of a midpoint goes to the nearer code; agreement
+    with torch's conversion wherever it does not overflow (|x| <= 464);
+    saturation to +-448 beyond."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    v = O.e4m3_decode(codes)
+    fin = ~np.isnan(v) & (codes != 0x80)
+    np.testing.assert_array_equal(O.e4m3_encode(v[fin]), codes[fin])
+    pos = v[:0x7F]
+    mid = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)  # exact in float32
+    got = O.e4m3_encode(mid)
+    even = np.where(np.arange(0x7E) % 2 == 0, np.arange(0x7E), np.arange(1, 0x7F))
+    np.testing.assert_array_equal(got, even.astype(np.uint8))
+    up = np.nextafter(mid, np.float32(np.inf))
+    dn = np.nextafter(mid, np.float32(0))
+    np.testing.assert_array_equal(O.e4m3_encode(up), np.arange(1, 0x7F, dtype=np.uint8))
+    np.testing.assert_array_equal(O.e4m3_encode(dn), np.arange(0, 0x7E, dtype=np.uint8))
+    rng = np.random.default_rng(22)
+    mag = np.exp2(rng.uniform(-12, np.log2(464), size=20000))
+    x = (mag * rng.choice([-1, 1], size=mag.size)).astype(np.float32)
+    x = np.concatenate([x, mid, -mid, up, dn]).astype(np.float32)
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.e4m3_encode(x), lib)
+    sat = np.array([465.0, 1e6, np.inf, -500.0, -np.inf, np.nan, -0.0, -1e-9])
+    np.testing.assert_array_equal(O.e4m3_encode(sat),
+                                  [0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F, 0x80, 0x80])
+
+
+def test_latent_row_scale_and_quantisation_bounds():
+    """The scale is the smallest power of two that brings the row's largest
+    |c| under 448 (so that element lands in [224, 448]); each element is then
+    within half a step of its binade: |c~ - c| <= 2^-4 |c| in the normal range
+    and <= 2^-10 scale in the subnormal one; c~ re-encodes to the same codes."""
+    rng = np.random.default_rng(23)
+    c = rng.normal(size=(64, 96)) * np.exp2(rng.integers(-20, 20, size=(64, 1)))
+    c[3] = 0.0
+    c[5, :] = 1e-3
+    c[5, 7] = 448.0 * 2.0 ** -5          # exactly on a binade edge
+    c[6, :] = 0.5
+    c[6, 0] = 448.0 * 2.0 ** 3 * (1 + 2.0 ** -30)  # just above one
+    codes, scale = O.quantize_latent_rows(c)
+    k = np.log2(scale)
+    assert np.all(k == np.round(k))
+    assert scale[3] == 1.0 and np.all(codes[3] == 0)
+    assert scale[5] == 2.0 ** -5 and scale[6] == 2.0 ** 4
+    amax = np.abs(c).max(axis=1)
+    nz = amax > 0
+    r = amax[nz] / scale[nz]
+    assert np.all(r <= 448) and np.all(r > 224)
+    deq = O.dequantize_latent_rows(codes, scale)
+    y = np.abs(c / scale[:, None])
+    normal = y >= 2.0 ** -6
+    err = np.abs(deq - c)
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(c)[normal] * (1 + 1e-12))
+    sub_bound = (2.0 ** -10 * scale[:, None] * np.ones_like(c))[~normal]
+    assert np.all(err[~normal] <= sub_bound * (1 + 1e-12))
+    np.testing.assert_array_equal(O.e4m3_encode(deq / scale[:, None]), codes)
+    # The row maximum keeps its sign and stays the largest magnitude.
+    j = np.abs(c).argmax(axis=1)
+    assert np.all(np.sign(deq[np.arange(64), j]) == np.sign(c[np.arange(64), j]))
+
+
+def test_decode_over_lossless_fp8_cache_equals_unquantised():
+    """When every latent is already an E4M3 value times a power of two, the
+    quantised cache holds the same numbers, and decode over its dequantised
+    rows equals decode over the original cache exactly."""
+    rng = np.random.default_rng(24)
+    B, H, d_c, d_r, d_n, d_v, cap = 2, 3, 8, 4, 5, 6, 7
+    lens = [7, 3]
+    p = _rand_problem(rng, B, H, d_c, d_r, d_n, d_v, cap, lens)
+    codes = rng.integers(0, 0x7E, size=(B, cap, d_c)).astype(np.uint8)
+    codes[..., 0] = 0x7E  # the row maximum is 448 * scale
+    codes |= (rng.integers(0, 2, size=codes.shape) * 0x80).astype(np.uint8)
+    sc = np.exp2(rng.integers(-12, -4, size=(B, cap)).astype(np.float64))
+    c = O.dequantize_latent_rows(codes, sc)
+    p["cache"][..., :d_c] = c
+    q_codes, q_sc = O.quantize_latent_rows(c)
+    np.testing.assert_array_equal(q_sc, sc)
+    np.testing.assert_array_equal(O.e4m3_decode(q_codes), O.e4m3_decode(codes))
+    deq_cache = p["cache"].copy()
+    deq_cache[..., :d_c] = O.dequantize_latent_rows(q_codes, q_sc)
+    args = (p["q_nope"], p["q_pe"], p["q_pos"], p["W_UK"], p["W_UV"])
+    a = O.mla_decode_materialised(*args, p["cache"], p["seqlens"], 0.3)
+    b = O.mla_decode_materialised(*args, deq_cache, p["seqlens"], 0.3)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
