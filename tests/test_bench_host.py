@@ -62,3 +62,32 @@ def test_reference_budget_is_bounded():
     src = open(os.path.join(ROOT, "bench.py")).read()
     assert "90.0 / max(1, args.steps + args.warmup)" in src
     assert hasattr(b, "OracleSampler")
+
+
+def test_reference_arm_json_line_on_cpu(monkeypatch):
+    """The reference arm runs the oracle on host cores only: on the tiny
+    workload, with each step's oracle budget cut to a few milliseconds, it
+    prints the contract's keys with its own metric in e2e and cpu_baseline."""
+    import argparse
+    import json
+
+    b = _bench()
+    real_run = b.OracleSampler.run
+    monkeypatch.setattr(b.OracleSampler, "run", lambda self, budget: real_run(self, 0.002))
+    args = argparse.Namespace(workload="tiny_f32", steps=2, warmup=3)
+    res = b.run_reference(args, rank=0, world=1)
+    line = json.loads(json.dumps(res))
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == b.METRIC
+    assert line["value"] > 0 and line["unit"] == "tokens/s"
+    assert abs(line["ms_per_step"] - 1e3 / line["value"]) < 1e-9 * line["ms_per_step"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert "tiny_f32" in line["config"]["workload"]
+    # Ranks other than 0 do no work and print nothing.
+    assert b.run_reference(args, rank=1, world=2) is None
