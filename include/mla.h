@@ -135,7 +135,10 @@ MLA_API int mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q
  * are contiguous), then, 256-byte aligned, lse_part [B + W - 1][H].
  * Rows j >= L_b never influence the result (they may hold anything).
  * num_splits = 0 picks the default for the current device; the number used is
- * returned through splits_used (may be NULL). */
+ * returned through splits_used (may be NULL).
+ * MLA_ERR_UNSUPPORTED: bf16 needs d_c = 512 and d_r = 64, and a contiguous
+ * bf16 cache must hold fewer than 2^31 rows (B * cache_capacity), the range
+ * of the tensor-copy row coordinate. */
 MLA_API int mla_decode_default_splits(const mla_dims* dims);
 MLA_API size_t mla_decode_workspace_bytes(const mla_dims* dims, int num_splits);
 MLA_API int mla_decode(const mla_dims* dims, const void* q_cat, const void* cache,

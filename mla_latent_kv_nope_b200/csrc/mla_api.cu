@@ -83,8 +83,14 @@ int check_pages(const mla_dims* d, int64_t num_pages, const int32_t* block_table
   return MLA_OK;
 }
 
-int decode_shape_supported(const mla_dims* d) {
+// Shapes the decode kernels take.  The tensor-core path addresses cache rows
+// with a 32-bit TMA coordinate, so a contiguous cache of 2^31 rows or more
+// (B * capacity) is refused here rather than failing at launch.
+int decode_shape_supported(const mla_dims* d, bool contiguous) {
   if (d->dtype == MLA_BF16 && (d->d_c != 512 || d->d_r != 64)) return MLA_ERR_UNSUPPORTED;
+  if (d->dtype == MLA_BF16 && contiguous &&
+      int64_t(d->B) * d->cache_capacity >= (int64_t(1) << 31))
+    return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
 
@@ -275,7 +281,7 @@ int decode_impl(const mla_dims* d, const void* q_cat, const void* cache, const P
                 size_t workspace_bytes, int* splits_used, void* stream) {
   int st = check_dims(d);
   if (st) return st;
-  if ((st = decode_shape_supported(d))) return st;
+  if ((st = decode_shape_supported(d, pm.table == nullptr))) return st;
   if (!q_cat || !cache || !seqlens || num_splits < 0 || num_splits > kMaxSplits ||
       !(softmax_scale > 0.f) || softmax_scale == INFINITY)
     return MLA_ERR_INVALID_ARG;
@@ -394,7 +400,7 @@ extern "C" int mla_decode_noalloc(const mla_dims* d, const void* q_cat, const vo
                                   float* lse, void* stream) {
   int st = check_dims(d);
   if (st) return st;
-  if ((st = decode_shape_supported(d))) return st;
+  if ((st = decode_shape_supported(d, true))) return st;
   if (!q_cat || !cache || !seqlens || !o_lat || !(softmax_scale > 0.f) ||
       softmax_scale == INFINITY)
     return MLA_ERR_INVALID_ARG;

@@ -95,6 +95,13 @@ def test_decode_argument_errors(lib):
         lib.mla_decode(ctypes.byref(dd), q, c, s, scale, W, ws, wsb, ctypes.byref(used), None)  # noqa: E731
     assert call(_dims(d_c=256)) == UNSUP            # bf16 decode tile is 512 + 64
     assert call(_dims(d_r=32)) == UNSUP
+    # 2^31 contiguous rows are past the 32-bit tensor-copy row coordinate.
+    big = _dims(B=1 << 15, cache_capacity=1 << 16)
+    big_ws = lib.mla_decode_workspace_bytes(ctypes.byref(big), 8)
+    assert lib.mla_decode(ctypes.byref(big), GOOD, GOOD, GOOD, 0.07, 8, GOOD2, big_ws,
+                          ctypes.byref(used), None) == UNSUP
+    assert lib.mla_decode_noalloc(ctypes.byref(big), GOOD, GOOD, GOOD, 0.07, GOOD2, None,
+                                  None) == UNSUP
     assert call(d, q=None) == INVALID
     assert call(d, scale=0.0) == INVALID
     assert call(d, scale=float("nan")) == INVALID
