@@ -141,6 +141,14 @@ def _need(t, dtype, shape, name):
                          f"{t.device} {t.dtype} {tuple(t.shape)}")
 
 
+def _need_ws(t, name="workspace"):
+    """A scratch buffer: any dtype, but device memory and contiguous (the
+    library writes it from kernels, so a host tensor must never reach it)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+        got = t.device if isinstance(t, torch.Tensor) else type(t).__name__
+        raise ValueError(f"{name}: expected a contiguous CUDA tensor, got {got}")
+
+
 # ---------------------------------------------------------------------------
 def cache_row_elems(d_c: int, d_r: int) -> int:
     """Elements of one latent cache row, d_c + d_r (mla_cache_row_elems)."""
@@ -164,6 +172,7 @@ def cache_append(dims: Dims, h, W_DKV, gamma, cache, seqlens, workspace, eps=1e-
     _need(seqlens, torch.int32, (dims.B,), "seqlens")
     if gamma is not None:
         _need(gamma, torch.float32, (dims.d_c,), "gamma")
+    _need_ws(workspace)
     st = load_library().mla_cache_append(
         ctypes.byref(dims.c()), hidden, _ptr(h), _ptr(W_DKV), _ptr(gamma), eps, rope_base,
         _ptr(cache), _ptr(seqlens), _ptr(workspace),
@@ -192,6 +201,7 @@ def cache_append_paged(dims: Dims, h, W_DKV, gamma, cache_pool, block_table, seq
     _need(seqlens, torch.int32, (dims.B,), "seqlens")
     if gamma is not None:
         _need(gamma, torch.float32, (dims.d_c,), "gamma")
+    _need_ws(workspace)
     st = load_library().mla_cache_append_paged(
         ctypes.byref(dims.c()), hidden, _ptr(h), _ptr(W_DKV), _ptr(gamma), eps, rope_base,
         _ptr(cache_pool), cache_pool.shape[0], _ptr(block_table), block_table.shape[1],
@@ -206,6 +216,7 @@ def decode_paged(dims: Dims, q_cat, cache_pool, block_table, seqlens, softmax_sc
     _need(q_cat, dims.torch_dtype, (dims.B, dims.H, dims.R), "q_cat")
     _need_pages(dims, cache_pool, block_table)
     _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    _need_ws(workspace)
     used = ctypes.c_int(0)
     st = load_library().mla_decode_paged(
         ctypes.byref(dims.c()), _ptr(q_cat), _ptr(cache_pool), cache_pool.shape[0],
@@ -250,6 +261,7 @@ def decode(dims: Dims, q_cat, cache, seqlens, softmax_scale, workspace, num_spli
     _need(q_cat, dt, (dims.B, dims.H, dims.R), "q_cat")
     _need(cache, dt, (dims.B, dims.cache_capacity, dims.R), "cache")
     _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    _need_ws(workspace)
     used = ctypes.c_int(0)
     st = load_library().mla_decode(ctypes.byref(dims.c()), _ptr(q_cat), _ptr(cache),
                                    _ptr(seqlens), float(softmax_scale), num_splits,
@@ -262,6 +274,8 @@ def decode(dims: Dims, q_cat, cache, seqlens, softmax_scale, workspace, num_spli
 def combine(dims: Dims, seqlens, workspace, splits_used, o_lat, lse=None, stream=None):
     """mla_combine: log-sum-exp merge of the partials into o_lat [B,H,d_c] fp32 (and
     lse [B,H] fp32 when given)."""
+    _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    _need_ws(workspace)
     _need(o_lat, torch.float32, (dims.B, dims.H, dims.d_c), "o_lat")
     if lse is not None:
         _need(lse, torch.float32, (dims.B, dims.H), "lse")
