@@ -59,6 +59,8 @@ __all__ = [
     "latent_attention",
     "combine_partials",
     "out_proj",
+    "prefill_scores",
+    "prefill_materialised",
     "output_projection",
     "fold_output_weights",
     "folded_output",
@@ -342,6 +344,52 @@ def out_proj(o_lat, W_UV) -> np.ndarray:
     after the latent-space weighted sum ([MLA-とは] "Value側の吸収", second
     equation for o_{t,i}).  o_lat: [B,H,d_c]; W_UV: [H,d_v,d_c] -> [B,H,d_v]."""
     return np.einsum("ivd,bid->biv", _f64(W_UV), _f64(o_lat))
+
+
+# ---------------------------------------------------------------------------
+# Prefill: many query tokens of one sequence, K and V materialised
+# ---------------------------------------------------------------------------
+def prefill_scores(q_nope, q_pe, q_pos, W_UK_i, c, k_pe, rope_base: float = 10000.0):
+    """Raw logits of head i for T query tokens against L cached rows, with the
+    causal mask: query t (at position q_pos[t]) sees rows j <= q_pos[t], and
+    the others get -inf.  Each unmasked entry is head_logits' dot product
+    [q^C ; RoPE(q^R, q_pos[t])] . [W^UK_i c_j ; k^R_j].
+
+    q_nope: [T, d_h]; q_pe: [T, d_r]; q_pos: [T]; W_UK_i: [d_h, d_c];
+    c: [L, d_c]; k_pe: [L, d_r] (stored rotated).  Returns [T, L]."""
+    q_nope, q_pe = _f64(q_nope), _f64(q_pe)
+    T, L = q_nope.shape[0], _f64(c).shape[0]
+    K = np.concatenate([_f64(c) @ _f64(W_UK_i).T, _f64(k_pe)], axis=1)   # [L, d_h + d_r]
+    Q = np.concatenate([q_nope, rope(q_pe, _f64(q_pos), rope_base)], axis=1)
+    S = Q @ K.T
+    j = np.arange(L)[None, :]
+    return np.where(j <= np.asarray(q_pos)[:, None], S, -math.inf)
+
+
+def prefill_materialised(q_nope, q_pe, q_pos, W_UK, W_UV, rows, d_c: int,
+                         softmax_scale: float, rope_base: float = 10000.0):
+    """Prefill of one sequence in the materialised form the pages recommend
+    when the step is compute-bound ([MLA-とは] "実装上のトレードオフ",
+    プリフィルとデコードで最適な形が違う): k^C = W^UK c and v^C = W^UV c are
+    formed for every cached row and the heads run ordinary causal attention.
+
+    q_nope: [T, H, d_h]; q_pe: [T, H, d_r]; q_pos: [T] positions (query t sees
+    rows j <= q_pos[t]); rows: [L, d_c + d_r] latent cache rows (the prompt's
+    own rows included).  Returns out [T, H, d_v] and lse [T, H] (float64)."""
+    q_nope, q_pe, W_UK, W_UV, rows = map(_f64, (q_nope, q_pe, W_UK, W_UV, rows))
+    T, H, _ = q_nope.shape
+    c, k_pe = rows[:, :d_c], rows[:, d_c:]
+    out = np.zeros((T, H, W_UV.shape[1]))
+    lse = np.full((T, H), -math.inf)
+    for i in range(H):
+        S = softmax_scale * prefill_scores(q_nope[:, i], q_pe[:, i], q_pos, W_UK[i], c, k_pe,
+                                           rope_base)
+        V = c @ W_UV[i].T                                                   # [L, d_v]
+        for t in range(T):
+            n = min(int(q_pos[t]) + 1, rows.shape[0])   # rows query t may see
+            p, lse[t, i] = softmax_lse(S[t, :n])
+            out[t, i] = p @ V[:n]
+    return out, lse
 
 
 # ---------------------------------------------------------------------------

@@ -706,3 +706,52 @@ def test_decode_over_lossless_fp8_cache_equals_unquantised():
     b = O.mla_decode_materialised(*args, deq_cache, p["seqlens"], 0.3)
     for x, y in zip(a, b):
         np.testing.assert_array_equal(x, y)
+
+
+# ---------------------------------------------------------------------------
+# Prefill in materialised form ([MLA-とは] "実装上のトレードオフ")
+# ---------------------------------------------------------------------------
+def test_prefill_scores_match_pages_key_side(pages, gold):
+    """[MLA-とは] 数値検証: the page's T x T content scores (no RoPE) from its
+    seeded inputs; entry [3, 1, 0] is printed.  The causal mask keeps it
+    (key 1 is before query 3) and hides every key after the query."""
+    x = pages
+    d, d_c, d_cq, d_h, n_h, T, d_r = x["dims"]
+    pos = np.arange(T)
+    S0 = O.prefill_scores(x["Q"][:, 0], np.zeros((T, 0)), pos, x["W_UK"][0], x["c_kv"],
+                          np.zeros((T, 0)))
+    assert abs(S0[3, 1] - gold["S_naive_3_1_0"]) < 1e-9
+    K = (x["c_kv"] @ x["w_uk"]).reshape(T, n_h, d_h)        # the page's naive K
+    S_page = np.einsum("th,jh->tj", x["Q"][:, 0], K[:, 0])
+    lower = np.tril(np.ones((T, T), dtype=bool))
+    np.testing.assert_allclose(S0[lower], S_page[lower], atol=1e-12)
+    assert np.all(np.isneginf(S0[~lower]))
+
+
+def test_prefill_rows_equal_single_token_decode():
+    """Every prefill row is the single-token decode of its query over the rows
+    it may see (the decode oracle is pinned independently above); the last
+    row is the plain decode; a key after a query never changes that row."""
+    rng = np.random.default_rng(25)
+    H, d_c, d_r, d_n, d_v, L, T = 3, 8, 4, 5, 6, 9, 4
+    W_UK = rng.normal(size=(H, d_n, d_c))
+    W_UV = rng.normal(size=(H, d_v, d_c))
+    rows = rng.normal(size=(L, d_c + d_r))
+    q_nope = rng.normal(size=(T, H, d_n))
+    q_pe = rng.normal(size=(T, H, d_r))
+    q_pos = np.array([L - 4, L - 3, L - 2, L - 1])
+    scale = 0.37
+    out, lse = O.prefill_materialised(q_nope, q_pe, q_pos, W_UK, W_UV, rows, d_c, scale)
+    for t in range(T):
+        n = q_pos[t] + 1
+        cache = rows[None, :n].copy()
+        o_d, _, l_d = O.mla_decode_materialised(q_nope[t][None], q_pe[t][None], [q_pos[t]],
+                                                W_UK, W_UV, cache, [n], scale)
+        np.testing.assert_allclose(out[t], o_d[0], atol=1e-12)
+        np.testing.assert_allclose(lse[t], l_d[0], atol=1e-12)
+    # Causality: perturbing the last row changes only the query that sees it.
+    rows2 = rows.copy()
+    rows2[L - 1] += 5.0
+    out2, _ = O.prefill_materialised(q_nope, q_pe, q_pos, W_UK, W_UV, rows2, d_c, scale)
+    np.testing.assert_array_equal(out2[:T - 1], out[:T - 1])
+    assert np.abs(out2[T - 1] - out[T - 1]).max() > 1e-6
