@@ -155,6 +155,23 @@ MLA_API int mla_combine(const mla_dims* dims, const int32_t* seqlens,
                 const void* workspace, size_t workspace_bytes, int splits_used,
                 float* o_lat, float* lse, void* stream);
 
+/* --- sequence-sharded decode: merge of per-range results -----------------------
+ * No counterpart on the pages: a long context can be split by tokens across
+ * devices, each holding a contiguous token range of every sequence and
+ * running mla_decode + mla_combine on it.  The n range results, gathered into
+ * one array, are merged here with the same log-sum-exp identity as the
+ * split-KV partials:
+ *   lse[b,i] = log sum_k exp(lse_k[b,i]),  o_lat[b,i] = sum_k exp(lse_k[b,i] - lse[b,i]) o_k[b,i]
+ * A result with lse_k = -inf (a range holding no key of sequence b) adds
+ * nothing and its o_k is not read; if every lse_k is -inf, o_lat = 0 and
+ * lse = -inf.
+ * o_parts [n_parts][B][H][d_c] fp32 and lse_parts [n_parts][B][H] fp32 are
+ * the stacked mla_combine outputs; o_lat [B][H][d_c] fp32; lse [B][H] fp32
+ * (may be NULL).  MLA_ERR_INVALID_ARG: n_parts outside [1, 1024] or a NULL
+ * array. */
+MLA_API int mla_merge_partials(const mla_dims* dims, int n_parts, const float* o_parts,
+                               const float* lse_parts, float* o_lat, float* lse, void* stream);
+
 /* --- 5. value up-projection -------------------------------------------------
  * [MLA-とは] "Value側の吸収": o_{t,i} = W^UV_i (sum_j a_{tj,i} c^KV_j).
  *   out[b,i,v] = sum_c W_UV[i,v,c] o_lat[b,i,c]

@@ -27,6 +27,7 @@ EXPORTED = (
     "mla_absorb_q", "mla_decode_default_splits", "mla_decode_workspace_bytes",
     "mla_decode", "mla_combine", "mla_out_proj", "mla_get_device_status",
     "mla_status_string", "mla_decode_noalloc", "mla_decode_paged", "mla_cache_append_paged",
+    "mla_merge_partials",
 )
 
 PAGE_ROWS = 64   # rows per page of a paged latent cache (one decode work tile)
@@ -103,6 +104,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                             ctypes.POINTER(ctypes.c_int), P]),
         "mla_cache_append_paged": (ctypes.c_int, [D, I32, P, P, P, F, F, P, I64, P, I32, P, P,
                                                   SZ, P]),
+        "mla_merge_partials": (ctypes.c_int, [D, ctypes.c_int, P, P, P, P, P]),
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -283,6 +285,22 @@ def combine(dims: Dims, seqlens, workspace, splits_used, o_lat, lse=None, stream
                                     workspace.numel() * workspace.element_size(), splits_used,
                                     _ptr(o_lat), _ptr(lse), _stream(stream))
     _check("mla_combine", st)
+
+
+def merge_partials(dims: Dims, o_parts, lse_parts, o_lat, lse=None, stream=None):
+    """mla_merge_partials: log-sum-exp merge of n per-token-range results,
+    o_parts [n,B,H,d_c] fp32 and lse_parts [n,B,H] fp32 (stacked combine
+    outputs), into o_lat [B,H,d_c] (and lse [B,H] when given)."""
+    n = o_parts.shape[0]
+    _need(o_parts, torch.float32, (n, dims.B, dims.H, dims.d_c), "o_parts")
+    _need(lse_parts, torch.float32, (n, dims.B, dims.H), "lse_parts")
+    _need(o_lat, torch.float32, (dims.B, dims.H, dims.d_c), "o_lat")
+    if lse is not None:
+        _need(lse, torch.float32, (dims.B, dims.H), "lse")
+    st = load_library().mla_merge_partials(ctypes.byref(dims.c()), n, _ptr(o_parts),
+                                           _ptr(lse_parts), _ptr(o_lat), _ptr(lse),
+                                           _stream(stream))
+    _check("mla_merge_partials", st)
 
 
 def out_proj(dims: Dims, o_lat, W_UV, out, stream=None):

@@ -39,6 +39,11 @@ bool make_cache_rows_map(CUtensorMap* map, const void* base, uint64_t rows);
 cudaError_t launch_combine(const int32_t* seqlens, int64_t cap, int B, int H, int d_c, int W,
                            const float* o_part, const float* lse_part, float* o_lat,
                            float* lse, cudaStream_t stream);
+// Log-sum-exp merge of n per-range results: o_parts [n][BH][d_c], lse_parts
+// [n][BH] -> o_lat [BH][d_c], lse [BH] (lse may be null).
+cudaError_t launch_merge_partials(int64_t BH, int d_c, int n, const float* o_parts,
+                                  const float* lse_parts, float* o_lat, float* lse,
+                                  cudaStream_t stream);
 
 template <typename T>
 cudaError_t launch_out_proj(const float* o_lat, const T* W_UV, int B, int H, int d_c,

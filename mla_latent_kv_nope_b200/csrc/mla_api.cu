@@ -341,6 +341,21 @@ int mla_combine(const mla_dims* d, const int32_t* seqlens, const void* workspace
 }
 
 // ---------------------------------------------------------------------------
+int mla_merge_partials(const mla_dims* d, int n_parts, const float* o_parts,
+                       const float* lse_parts, float* o_lat, float* lse, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if (n_parts <= 0 || n_parts > kMaxSplits || !o_parts || !lse_parts || !o_lat)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(lse_parts) || !aligned16(o_lat) ||
+      (lse && !aligned16(lse)))
+    return MLA_ERR_ALIGNMENT;
+  return cuda_status(launch_merge_partials(int64_t(d->B) * d->H, d->d_c, n_parts, o_parts,
+                                           lse_parts, o_lat, lse,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------------------
 int mla_out_proj(const mla_dims* d, const float* o_lat, const void* W_UV, void* out,
                  void* stream) {
   int st = check_dims(d);
