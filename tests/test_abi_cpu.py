@@ -121,6 +121,16 @@ def test_other_entry_point_errors(lib):
     assert lib.mla_combine(ctypes.byref(d), GOOD, GOOD2, need, 0, GOOD, None, None) == INVALID
     assert lib.mla_combine(ctypes.byref(d), GOOD, GOOD2, need - 4, 8, GOOD, None, None) == WS
     assert lib.mla_combine(ctypes.byref(d), GOOD, BAD, need, 8, GOOD, None, None) == ALIGN
+    # merge of per-range results (sequence sharding)
+    mg = lambda n=2, o=GOOD, l=GOOD, out=GOOD2, ls=None: lib.mla_merge_partials(  # noqa: E731
+        ctypes.byref(d), n, o, l, out, ls, None)
+    assert mg(n=0) == INVALID
+    assert mg(n=1025) == INVALID
+    assert mg(o=None) == INVALID
+    assert mg(l=None) == INVALID
+    assert mg(out=None) == INVALID
+    assert mg(o=BAD) == ALIGN
+    assert mg(ls=BAD) == ALIGN
     # out_proj
     assert lib.mla_out_proj(ctypes.byref(d), None, GOOD, GOOD2, None) == INVALID
     assert lib.mla_out_proj(ctypes.byref(d), GOOD, BAD, GOOD2, None) == ALIGN
