@@ -755,3 +755,41 @@ def test_prefill_rows_equal_single_token_decode():
     out2, _ = O.prefill_materialised(q_nope, q_pe, q_pos, W_UK, W_UV, rows2, d_c, scale)
     np.testing.assert_array_equal(out2[:T - 1], out[:T - 1])
     assert np.abs(out2[T - 1] - out[T - 1]).max() > 1e-6
+
+
+def test_two_level_merge_equals_one_level():
+    """The log-sum-exp merge composes: merging the partials of each group
+    (one rank's split-KV partials) and then merging the groups' results (the
+    ranks) equals one merge of all partials, and both equal attention over the
+    union of the key sets.  Sequence sharding relies on exactly this."""
+    rng = np.random.default_rng(26)
+    B, H, d_c, d_r = 2, 3, 6, 2
+    L = 23
+    rows = rng.normal(size=(B, L, d_c + d_r))
+    q = rng.normal(size=(B, H, d_c + d_r))
+    cuts = [0, 4, 9, 9, 15, 23]            # six chunks, one of them empty
+    parts = [O.latent_attention(q, rows, None, 0.8, d_c,
+                                key_range=[(cuts[k], cuts[k + 1])] * B)
+             for k in range(len(cuts) - 1)]
+    o_all = np.stack([p[0] for p in parts], axis=2)
+    l_all = np.stack([p[1] for p in parts], axis=2)
+    one_o, one_l = O.combine_partials(o_all, l_all)
+    groups = [[0, 1], [2, 3], [4]]         # ranks holding consecutive chunks
+    g = [O.combine_partials(o_all[:, :, idx], l_all[:, :, idx]) for idx in groups]
+    two_o, two_l = O.combine_partials(np.stack([x[0] for x in g], axis=2),
+                                      np.stack([x[1] for x in g], axis=2))
+    ref_o, ref_l = O.latent_attention(q, rows, [L] * B, 0.8, d_c)
+    for o, lse in ((one_o, one_l), (two_o, two_l)):
+        np.testing.assert_allclose(o, ref_o, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, atol=1e-12)
+
+
+def test_rope_rotations_compose():
+    """RoPE at position a then at b equals RoPE at a + b (each pair is a plane
+    rotation by an angle linear in the position), and rotating back by -a
+    restores the input."""
+    rng = np.random.default_rng(27)
+    x = rng.normal(size=(5, 16))
+    for a, b in [(3, 4), (1000, 17), (0, 9)]:
+        np.testing.assert_allclose(O.rope(O.rope(x, a), b), O.rope(x, a + b), atol=1e-9)
+        np.testing.assert_allclose(O.rope(O.rope(x, a), -a), x, atol=1e-9)
