@@ -382,6 +382,10 @@ SMALL_STEPS = [
     W["v2lite_bf16"].scaled(B=2, N=300),
     W["v3_bf16"].scaled(B=2, N=260),
     W["ragged_append_bf16"].scaled(B=6, N=500, hidden=512),
+    # NoPE ([yuuk] 横断的知見: MLA layers without RoPE): d_r = 0, so the cache
+    # row is c^KV alone and the query has no decoupled part (fp32 path).
+    W["tiny_f32"].scaled(name="tiny_f32_nope", B=3, N=150, d_r=0, ragged=True, append=True,
+                         hidden=64),
 ]
 
 
