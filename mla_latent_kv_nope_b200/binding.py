@@ -360,7 +360,8 @@ class DecodeStep:
             cache_append_paged(self.dims, h, self.W_DKV, self.gamma, cache, block_table,
                                seqlens, self.ws_append, self.eps, self.rope_base)
 
-    def _absorb(self, q_nope, q_pe, q_pos):
+    def absorb(self, q_nope, q_pe, q_pos):
+        """absorb_q into the step's q_cat buffer."""
         absorb_q(self.dims, q_nope, q_pe, self.W_UK, q_pos, self.q_cat, self.rope_base)
 
     def _attend_latent(self, cache, seqlens, block_table=None):
@@ -375,7 +376,7 @@ class DecodeStep:
         return self.out
 
     def attend(self, q_nope, q_pe, q_pos, cache, seqlens, block_table=None):
-        self._absorb(q_nope, q_pe, q_pos)
+        self.absorb(q_nope, q_pe, q_pos)
         return self._attend_latent(cache, seqlens, block_table)
 
     def __call__(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, block_table=None):
@@ -390,7 +391,7 @@ class DecodeStep:
         # previous step's decode has finished reading q_cat).
         self._side.wait_stream(main)
         with torch.cuda.stream(self._side):
-            self._absorb(q_nope, q_pe, q_pos)
+            self.absorb(q_nope, q_pe, q_pos)
         if h is not None:
             self.append(h, cache, seqlens, block_table)
         main.wait_stream(self._side)

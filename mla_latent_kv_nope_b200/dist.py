@@ -122,7 +122,7 @@ def sequence_sharded_attend(step, q_nope, q_pe, q_pos, local_cache, local_seqlen
     from . import binding as bd
 
     dims = step.dims
-    step._absorb(q_nope, q_pe, q_pos)
+    step.absorb(q_nope, q_pe, q_pos)
     used = bd.decode(dims, step.q_cat, local_cache, local_seqlens, step.scale, step.ws,
                      step.num_splits)
     bd.combine(dims, local_seqlens, step.ws, used, step.o_lat, step.lse)
