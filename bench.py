@@ -45,7 +45,7 @@ def _peaks():
 
 def _decode_source_hash():
     h = hashlib.sha256()
-    for name in ("k_decode_tc.cu", "common.cuh"):
+    for name in ("k_decode_tc.cu", "k_decode_pair.cu", "tile_deal.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "mla_latent_kv_nope_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -529,7 +529,8 @@ class OracleSampler:
             done += 1
         step_s = spent / done * w.B * w.H
         return {"value": w.B / step_s, "unit": "tokens/s", "cores": _blas_threads(),
-                "kind": "oracle", "cpu_model": _cpu_model(), "host_cores": os.cpu_count(),
+                "kind": "oracle", "extrapolated": True, "cpu_model": _cpu_model(),
+                "host_cores": os.cpu_count(),
                 "sample": f"{done} (sequence, head) pairs from {len(self.caches)} seeded random "
                           f"sequences ({spent:.1f} s of oracle time), each append + "
                           f"materialised attention over its full length; scaled by "
@@ -563,10 +564,63 @@ def run_reference(args, rank, world):
         "data": "synthetic (seeded)",
         "config": {"workload": _workload_desc(w), "global_batch": w.B * world,
                    "seq_len": w.N + 1, "parallelism": "cpu (oracle, rank 0)"},
+        # Each step times a bounded sample of (sequence, head) pairs; the step
+        # time is the sampled per-pair time x B*H pairs (extrapolated).
+        "extrapolated": True,
         "cpu_baseline": {"kind": "oracle", "cores": vals[-1]["cores"], "sample": vals[-1]["sample"],
-                         "value": v, "unit": "tokens/s"},
+                         "value": v, "unit": "tokens/s", "extrapolated": True},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def _relaunch_per_gpu(n):
+    """`--gpus N` (N > 1) started without a launcher: run this same command as
+    N ranks, one process per GPU, under torch.distributed.run (rendezvous on
+    127.0.0.1); rank 0 prints the JSON line.  Returns the launcher's exit code."""
+    import socket
+    import subprocess
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.run(cmd).returncode
+
+
+def run_dry(args, rank, world):
+    """Host-only check of the multi-rank plumbing (gloo, no GPU, no kernels):
+    each rank 'steps' for a rank-dependent time, the job time is the maximum
+    over ranks, and rank 0 reports the world size it ran with.  Its numbers
+    are not measurements of the decode."""
+    import datetime
+
+    import torch.distributed as dist
+
+    from mla_latent_kv_nope_b200 import dist as mdist
+
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        per_step = 1e-3 * (rank + 1)
+        for _ in range(args.warmup):
+            time.sleep(per_step)
+        mdist.barrier(world)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            time.sleep(per_step)
+        ms = (time.perf_counter() - t0) * 1e3
+        ms_max = mdist.max_over_ranks(ms, world)
+        mdist.barrier(world)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {"dry_run": True, "metric": METRIC, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "rank0_ms_per_step": ms / args.steps}
 
 
 def main():
@@ -583,13 +637,24 @@ def main():
                     help="keep the latent cache in shuffled 64-row pages behind a block table")
     ap.add_argument("--eager", action="store_true",
                     help="launch each kernel from the host every step instead of a CUDA graph")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="host-only check of the multi-rank launch and timing (gloo, no GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        sys.exit(_relaunch_per_gpu(args.gpus))
+    world = int(world_env or "1")
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but the launcher started {world} rank(s)")
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
+    if args.dry_run:
+        res = run_dry(args, rank, world)
+    elif args.impl == "reference":
         res = run_reference(args, rank, world)
     else:
         if world > 1:

@@ -91,3 +91,39 @@ def test_reference_arm_json_line_on_cpu(monkeypatch):
     assert "tiny_f32" in line["config"]["workload"]
     # Ranks other than 0 do no work and print nothing.
     assert b.run_reference(args, rank=1, world=2) is None
+
+
+def _json_lines(out):
+    import json
+    return [json.loads(ln) for ln in out.splitlines() if ln.startswith("{")]
+
+
+def test_gpus_flag_launches_one_rank_per_gpu():
+    """`bench.py --gpus 2` without a launcher re-runs itself as two ranks under
+    torch.distributed.run; in the host-only dry run (gloo, no GPU) rank 0
+    reports two ranks and the slowest rank's time (rank 1 steps 2 ms, rank 0
+    1 ms), never a one-rank result."""
+    import subprocess
+
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--dry-run", "--steps", "5", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1, r.stdout
+    line = lines[0]
+    assert line["dry_run"] is True and line["n_gpus"] == 2
+    assert line["ms_per_step"] >= 2.0 and line["ms_per_step"] >= line["rank0_ms_per_step"]
+
+
+def test_gpus_flag_must_match_the_launcher():
+    import subprocess
+
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                        "--dry-run", "--steps", "2", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=120, env=env, cwd=ROOT)
+    assert r.returncode != 0 and "launcher started 1 rank" in r.stderr
+    assert not _json_lines(r.stdout)
