@@ -34,7 +34,8 @@
  *     capacity, a wait that gave up) are recorded in a per-device status word
  *     read by mla_get_device_status.  No exception crosses the ABI.
  *   - dtype MLA_BF16: bf16 tensors, fp32 accumulation; decode requires
- *     d_c = 512 and d_r = 64 (the tensor-core kernel's tile shape).
+ *     d_c = 512 and d_r = 64, or d_r = 0 (NoPE: rows are c^KV alone) -- the
+ *     tensor-core kernels' tile shapes.
  *     dtype MLA_F32: fp32 tensors throughout; d_c, d_nope, d_v multiples of 4,
  *     d_r even, d_c <= 1024, d_r <= 256.
  *   - o_lat and lse are fp32 in both dtypes.
@@ -122,9 +123,11 @@ MLA_API int mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q
 /* --- 3. split-KV latent decode --------------------------------------------
  * [MLA-とは] "実装上のトレードオフ" (absorbed form = MQA with head dim
  * d_c + d_r), "Value側の吸収" (weighted sum in latent space), "Decoupled
- * RoPE" (softmax scale 1/sqrt(d_h + d_h^R) in the pages' configs).
+ * RoPE" (softmax scale 1/sqrt(d_h + d_h^R)).
  * For sequence b, head i and cached rows j < L_b:
  *   s_j = softmax_scale * (q_cat[b,i] . cache[b,j,:])
+ * softmax_scale = 0 selects the pages' scale 1/sqrt(d_nope + d_r); a
+ * negative, infinite or NaN scale is MLA_ERR_INVALID_ARG.
  * The key space of all sequences, cut into tiles of 64 rows, is dealt into
  * `num_splits` contiguous ranges (worker w takes tiles [w*T/W, (w+1)*T/W) of
  * the concatenated per-sequence tile lists, T = sum_b ceil(L_b/64)).  Worker w
@@ -136,7 +139,7 @@ MLA_API int mla_absorb_q(const mla_dims* dims, const void* q_nope, const void* q
  * Rows j >= L_b never influence the result (they may hold anything).
  * num_splits = 0 picks the default for the current device; the number used is
  * returned through splits_used (may be NULL).
- * MLA_ERR_UNSUPPORTED: bf16 needs d_c = 512 and d_r = 64, and a contiguous
+ * MLA_ERR_UNSUPPORTED: bf16 needs d_c = 512 and d_r = 64 or 0, and a contiguous
  * bf16 cache must hold fewer than 2^31 rows (B * cache_capacity), the range
  * of the tensor-copy row coordinate. */
 MLA_API int mla_decode_default_splits(const mla_dims* dims);
@@ -207,18 +210,21 @@ MLA_API int mla_cache_append_paged(const mla_dims* dims, int32_t hidden, const v
 
 /* --- 3+4 without a workspace -------------------------------------------------
  * No counterpart on the pages: this is a convenience of this library.
- * For callers that cannot allocate device memory (code running while a stream
- * is captured into a CUDA graph, where cudaMalloc is not allowed; plugins that
- * only receive fixed buffers from a host framework), this runs mla_decode and
- * mla_combine with the split-KV partials kept in a fixed array inside the
- * library instead of a caller workspace.  Inputs and outputs are as for
+ * For callers that cannot allocate device memory (plugins that only receive
+ * fixed buffers from a host framework, runtimes whose device memory is owned
+ * by another allocator), this runs mla_decode and mla_combine with the
+ * split-KV partials kept in a fixed array inside the library instead of a
+ * caller workspace.  Inputs and outputs are as for
  * mla_decode + mla_combine (q_cat, cache, seqlens in; o_lat [B,H,d_c] fp32 and
  * lse [B,H] fp32 (may be NULL) out); nothing is allocated or freed.
  *   - The array holds MLA_DECODE_NOALLOC_SCRATCH_BYTES on every device that
- *     loads the library, until the process exits.  The split count is the
- *     device default, lowered until the partials, (B + W - 1) * H * (d_c + 1)
- *     floats, fit; if even one split does not fit (B * H * (d_c + 1) * 4 bytes
- *     above the limit) the call returns MLA_ERR_WORKSPACE and launches nothing.
+ *     loads the library, until the process exits.  The split count W is the
+ *     device default, lowered until the partials (mla_decode's workspace for
+ *     W splits) fit:
+ *       round_up((B + W - 1) * H * d_c * 4, 256) + round_up((B + W - 1) * H * 4, 256)
+ *         <= MLA_DECODE_NOALLOC_SCRATCH_BYTES
+ *     if even W = 1 does not fit the call returns MLA_ERR_WORKSPACE and
+ *     launches nothing.
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
  *   - All calls share the one array and it keeps the previous call's
@@ -229,6 +235,18 @@ MLA_API int mla_cache_append_paged(const mla_dims* dims, int32_t hidden, const v
 MLA_API int mla_decode_noalloc(const mla_dims* dims, const void* q_cat, const void* cache,
                                const int32_t* seqlens, float softmax_scale, float* o_lat,
                                float* lse, void* stream);
+
+/* --- failure-detection test hook ------------------------------------------------
+ * No counterpart on the pages.  Every wait inside the tensor-core kernels is
+ * bounded: a wait that runs out sets MLA_ERR_DEVICE_TIMEOUT in the device
+ * status word, the kernel drains its own copies and products and returns, and
+ * the context stays usable.  This hook lets a test exercise that path without
+ * any fault: with cycles > 0, every later bf16 mla_decode / mla_decode_paged /
+ * mla_decode_noalloc launch first waits `cycles` SM cycles on a barrier that
+ * nothing ever arrives on, then gives up; its outputs are then undefined.
+ * cycles = 0 (the default) turns it off.  Process-wide; not for production
+ * use. */
+MLA_API int mla_debug_inject_wait(uint64_t cycles);
 
 /* --- status ------------------------------------------------------------------
  * Synchronises `stream`, then returns and clears the current device's status

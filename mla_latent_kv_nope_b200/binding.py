@@ -27,7 +27,7 @@ EXPORTED = (
     "mla_absorb_q", "mla_decode_default_splits", "mla_decode_workspace_bytes",
     "mla_decode", "mla_combine", "mla_out_proj", "mla_get_device_status",
     "mla_status_string", "mla_decode_noalloc", "mla_decode_paged", "mla_cache_append_paged",
-    "mla_merge_partials",
+    "mla_merge_partials", "mla_debug_inject_wait",
 )
 
 PAGE_ROWS = 64   # rows per page of a paged latent cache (one decode work tile)
@@ -106,6 +106,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                   SZ, P]),
         "mla_merge_partials": (ctypes.c_int, [D, ctypes.c_int, P, P, P, P, P]),
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "mla_debug_inject_wait": (ctypes.c_int, [ctypes.c_uint64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -314,6 +315,13 @@ def out_proj(dims: Dims, o_lat, W_UV, out, stream=None):
     _check("mla_out_proj", st)
 
 
+def debug_inject_wait(cycles: int) -> None:
+    """mla_debug_inject_wait: test hook that makes later bf16 decode launches
+    wait ``cycles`` SM cycles on a barrier nothing arrives on and give up
+    (MLA_ERR_DEVICE_TIMEOUT in the status word); 0 turns it off."""
+    _check("mla_debug_inject_wait", load_library().mla_debug_inject_wait(int(cycles)))
+
+
 def get_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(load_library().mla_get_device_status(_stream(stream)))
@@ -335,8 +343,8 @@ class DecodeStep:
                  rope_base=10000.0, eps=1e-6, num_splits=0, device="cuda", overlap=True):
         self.dims = dims
         self.W_UK, self.W_UV, self.W_DKV, self.gamma = W_UK, W_UV, W_DKV, gamma
-        self.scale = (softmax_scale if softmax_scale is not None
-                      else (dims.d_nope + dims.d_r) ** -0.5)
+        # 0 asks the library for the pages' scale 1/sqrt(d_nope + d_r).
+        self.scale = 0.0 if softmax_scale is None else float(softmax_scale)
         self.rope_base, self.eps = rope_base, eps
         self.num_splits = num_splits or decode_default_splits(dims)
         ws = decode_workspace_bytes(dims, self.num_splits)

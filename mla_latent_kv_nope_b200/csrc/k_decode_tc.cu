@@ -1,10 +1,11 @@
-// Tensor-core split-KV latent decode for sm_100a (bf16, d_c = 512, d_r = 64).
+// Tensor-core split-KV latent decode for sm_100a (bf16, d_c = 512, d_r = 64,
+// or d_r = 0 for MLA without the decoupled RoPE part).
 //
 // What it computes ([MLA-とは] "実装上のトレードオフ": after absorption the
 // decode is MQA with head dim d_c + d_r = 576 -- one latent row per cached
 // token is the key of every head, its first 512 entries the value;
 // "Value側の吸収": the weighted sum stays in latent space):
-//   S = q_cat[b, heads] . C^T            (M = 64 heads, N = 64 keys, K = 576)
+//   S = q_cat[b, heads] . C^T            (M = 64 heads, N = 64 keys, K = 512 + d_r)
 //   online softmax over the keys of one work range
 //   O = P . C[:, 0:512]                  (M = 64 heads, N = 512, K = 64 keys)
 // The two products are dense because all heads share the same latent rows.
@@ -12,9 +13,11 @@
 // Structure (one CTA = 64 heads of one work range; CTAs of the same range for
 // the other head groups are launched next to it so the tile is read from HBM
 // once and from L2 after that):
-//   warp 4      TMA producer: per 64-key tile, 9 boxes of [64 keys x 64 dims]
-//               bf16 with 128-byte swizzle into a 3-stage ring, plus an L2
-//               prefetch a few tiles ahead.
+//   warp 4      TMA producer: per 64-key tile, 9 (or 8 without RoPE) boxes of
+//               [64 keys x 64 dims] bf16 with 128-byte swizzle into a 3-stage
+//               ring, plus an L2 prefetch a few tiles ahead.  A stage always
+//               has 9 chunks: the ninth (the RoPE keys, or nothing without
+//               RoPE) receives P once S has been computed.
 //   warp 5      QK^T issuer: S = Q C^T with Q read from tensor memory (only
 //               the cache tile is fetched from shared memory); it runs ahead
 //               as far as the stages and the two S buffers allow.
@@ -27,7 +30,7 @@
 // Tensor memory (an M = 64 tile occupies 16 of the 32 lanes of each
 // quadrant; "lo" = lanes 0-15, "hi" = lanes 16-31):
 //   lo lanes: cols [0,64) and [64,128) S double buffer; cols [128,416) Q
-//             (576 bf16 packed in pairs)
+//             (512 + d_r bf16 packed in pairs)
 //   hi lanes: cols [0,256) O[:, 0:256]; cols [256,512) O[:, 256:512]
 // All tensor-memory traffic of the softmax warps uses 16-lane accesses, so
 // each row is shared by two threads (keys 0-31 / 32-63 of S; columns
@@ -40,6 +43,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tile_deal.cuh"
 
 namespace mla {
 
@@ -48,11 +52,11 @@ namespace {
 using namespace sm100;
 
 constexpr int kHeadsPerCta = 64;
-constexpr int kR = 576;
+constexpr int kR = 576;                               // row width with RoPE
 constexpr int kDc = 512;
 constexpr int kChunkElems = 64;                       // one 128-byte swizzle row
-constexpr int kChunks = kR / kChunkElems;             // 9 (8 latent + 1 RoPE)
-constexpr int kRopeChunk = 8;
+constexpr int kChunks = kR / kChunkElems;             // 9 chunks per stage (8 latent + 1)
+constexpr int kRopeChunk = 8;                         // RoPE keys, then P
 constexpr int kChunkBytes = kTileKeys * 128;          // 8192
 constexpr int kStageBytes = kChunks * kChunkBytes;    // 73728
 constexpr int kStages = 3;
@@ -76,20 +80,15 @@ struct Barriers {
   uint64_t p_full[2];
   uint64_t o_free;
   uint64_t mma_drain, pv_drain;
+  uint64_t never;                 // injected test wait: nothing ever arrives on it
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// Exclusive prefix of per-sequence tile counts, built once per CTA so that no
-// role walks the length array through global memory (a chain of dependent
-// loads).  Batches with more sequences fall back to walking global memory.
-constexpr int kMaxSeqSmem = 1024;
-
 constexpr size_t kOffStage = 0;
 constexpr size_t kOffBar = size_t(kStages) * kStageBytes;
 constexpr size_t kOffPrefix = kOffBar + ((sizeof(Barriers) + 15) / 16) * 16;
-constexpr size_t kOffLens = kOffPrefix + sizeof(int32_t) * (kMaxSeqSmem + 1);
-constexpr size_t kSmemBytes = kOffLens + sizeof(int32_t) * kMaxSeqSmem + 1024;
+constexpr size_t kSmemBytes = kOffPrefix + kTilePrefixSmemBytes + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA");
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
@@ -101,7 +100,8 @@ __device__ __forceinline__ void raise_abort(Barriers* bars, int* status) {
 }
 
 // Warp-uniform bounded wait (all 32 lanes poll; lane 0 owns the limit).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit = kWaitLimitCycles) {
   if (__all_sync(0xffffffffu, mbar_try(bar, parity))) return true;
   const uint64_t t0 = sm_cycles();
   for (uint32_t it = 0;; ++it) {
@@ -110,69 +110,23 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     if ((it & 63) == 63) {
       int give_up = 0;
       if ((threadIdx.x & 31) == 0)
-        give_up = (*abort_flag != 0) || (sm_cycles() - t0 > kWaitLimitCycles);
+        give_up = (*abort_flag != 0) || (sm_cycles() - t0 > limit);
       if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
     }
   }
 }
 
-// Tile prefix of the batch: prefix(b) = sum of tiles of sequences < b, from
-// shared memory when the batch fits, else recomputed from the lengths.
-struct TilePrefix {
-  const int32_t* sp;       // shared prefix [B + 1] or nullptr
-  const int32_t* sl;       // shared clamped lengths [B] or nullptr
-  const int32_t* seqlens;
-  int B;
-  int64_t cap;
-  __device__ int64_t at(int b) const {
-    if (sp) return sp[b];
-    int64_t p = 0;
-    for (int k = 0; k < b; ++k) p += tiles_of(clamp_len(seqlens[k], cap));
-    return p;
-  }
-  __device__ int64_t len(int b) const { return sl ? sl[b] : clamp_len(seqlens[b], cap); }
-  // First sequence whose tiles end after tile t (binary search on the prefix).
-  __device__ int first_after(int64_t t) const {
-    if (!sp) {
-      int64_t p = 0;
-      for (int b = 0; b < B; ++b) {
-        p += tiles_of(len(b));
-        if (p > t) return b;
-      }
-      return B;
-    }
-    int lo = 0, hi = B;  // smallest b with sp[b + 1] > t
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (sp[mid + 1] > t) hi = mid; else lo = mid + 1;
-    }
-    return lo;
-  }
-};
-
-// Sequences overlapping this worker's tile range are visited in order; the
-// callback gets (b, first tile, end tile (both local to b), length) and
-// returns false to stop.
-template <typename F>
-__device__ __forceinline__ void for_each_segment(const TilePrefix& tp, int64_t t_begin,
-                                                 int64_t t_end, F&& f) {
-  for (int b = tp.first_after(t_begin); b < tp.B; ++b) {
-    const int64_t pre = tp.at(b);
-    if (pre >= t_end) return;
-    const int64_t L = tp.len(b);
-    const int64_t nt = tiles_of(L);
-    const int64_t lo = max(pre, t_begin), hi = min(pre + nt, t_end);
-    if (lo < hi && !f(b, lo - pre, hi - pre, L)) return;
-  }
-}
-
+template <int kDr>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* __restrict__ cache,
                  const PageMap pm,
                  const __nv_bfloat16* __restrict__ q_cat,
                  const int32_t* __restrict__ seqlens, int B, int H, int64_t cap,
                  float scale_log2, int W, float* __restrict__ o_part,
-                 float* __restrict__ lse_part, int* __restrict__ status) {
+                 float* __restrict__ lse_part, int* __restrict__ status, uint64_t inject_wait) {
+  constexpr int R = kDc + kDr;                    // cache row and q_cat row width
+  constexpr int kLoadChunks = R / kChunkElems;    // chunks that come from the cache
+  constexpr uint32_t kLoadBytes = kLoadChunks * kChunkBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -185,38 +139,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
 
   // Tile prefix of the batch (all threads load lengths in parallel; warp 0
   // scans 32 at a time with shuffles).
-  int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + kOffPrefix);
-  int32_t* s_lens = reinterpret_cast<int32_t*>(smem + kOffLens);
-  const bool prefix_in_smem = B <= kMaxSeqSmem;
-  int64_t n_tiles = 0;
-  if (prefix_in_smem) {
-    for (int b = threadIdx.x; b < B; b += kThreads) {
-      const int64_t L = clamp_len(seqlens[b], cap);
-      s_lens[b] = int32_t(L);
-      s_prefix[b + 1] = int32_t(tiles_of(L));
-    }
-    __syncthreads();
-    if (warp == 0) {
-      int32_t carry = 0;
-      for (int b0 = 0; b0 < B; b0 += 32) {
-        int32_t v = (b0 + lane < B) ? s_prefix[b0 + lane + 1] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
-          if (lane >= o) v += u;
-        }
-        if (b0 + lane < B) s_prefix[b0 + lane + 1] = carry + v;
-        carry += __shfl_sync(0xffffffffu, v, 31);
-      }
-      if (lane == 0) s_prefix[0] = 0;
-    }
-    __syncthreads();
-    n_tiles = s_prefix[B];
-  } else {
-    for (int b = 0; b < B; ++b) n_tiles += tiles_of(clamp_len(seqlens[b], cap));
-  }
-  const TilePrefix tp{prefix_in_smem ? s_prefix : nullptr, prefix_in_smem ? s_lens : nullptr,
-                      seqlens, B, cap};
+  TilePrefix tp;
+  const int64_t n_tiles = build_tile_prefix(smem + kOffPrefix, seqlens, B, cap, &tp);
   if (n_tiles == 0) return;
   const int64_t t_begin = worker_tile_begin(w, n_tiles, W);
   const int64_t t_end = worker_tile_begin(w + 1, n_tiles, W);
@@ -236,6 +160,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     mbar_init(&bars->o_free, 32 * kSoftmaxWarps);
     mbar_init(&bars->mma_drain, 1);
     mbar_init(&bars->pv_drain, 1);
+    mbar_init(&bars->never, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -250,6 +175,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
+  uint32_t n_issued = 0;   // loads issued by the producer (lane 0 of its warp)
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -267,7 +193,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
           if (r < 0) return;
           const int64_t rows = pm.table ? int64_t(kTileKeys)
                                         : min(int64_t(kTileKeys), cap - t * kTileKeys);
-          bulk_prefetch_l2(cache + r * kR, uint32_t(rows * kR * 2));
+          bulk_prefetch_l2(cache + r * R, uint32_t(rows * R * 2));
         };
         for (int64_t t = lo; t < hi; ++t, ++i) {
           const int s = i % kStages;
@@ -283,10 +209,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
             record_status(status, MLA_ERR_BOUNDS);
             r = pm.total_rows(B);
           }
-          mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
+          mbar_arrive_expect_tx(&bars->full[s], kLoadBytes);
           const int32_t crow = int32_t(r);
           uint8_t* dst = sStage + s * kStageBytes;
-          for (int c = 0; c < kChunks; ++c)
+          for (int c = 0; c < kLoadChunks; ++c)
             tma_load_2d(&tm_c, &bars->full[s], dst + c * kChunkBytes, c * kChunkElems, crow);
           // Loads of the first tiles go out before any prefetch.
           if (t == lo)
@@ -295,14 +221,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
         }
         return true;
       });
-      if (!ok) {
-        raise_abort(bars, status);
-        // Drain this CTA's own loads before it may exit: the last load into
-        // each stage (bounded, ignoring the flag).
-        volatile int no_abort = 0;
-        for (uint32_t k = (i > kStages ? i - kStages : 0); k < i; ++k)
-          mbar_wait(&bars->full[k % kStages], (k / kStages) & 1, &no_abort, kWaitLimitCycles);
-      }
+      if (!ok) raise_abort(bars, status);
+      n_issued = i;
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ QK^T issuer
@@ -312,7 +232,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     int seg = 0;
     bool ok = true;
     const uint32_t st_base = smem_u32(sStage);
-    for_each_segment(tp, t_begin, t_end, [&](int, int64_t lo, int64_t hi, int64_t) {
+    // Test hook: a wait on a barrier nothing arrives on, so the give-up path runs.
+    if (inject_wait) ok = warp_wait(&bars->never, 0, abort_flag, inject_wait);
+    if (ok) for_each_segment(tp, t_begin, t_end, [&](int, int64_t lo, int64_t hi, int64_t) {
       // The softmax warps have written this sequence's query block.
       if (!(ok = warp_wait(&bars->q_ready, seg & 1, abort_flag))) return false;
       for (int64_t t = lo; t < hi; ++t, ++i) {
@@ -328,7 +250,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
         const uint64_t b0 = smem_desc_sw128(st_base + uint32_t(st) * kStageBytes, 16, 1024);
         const uint32_t a0 = tmem + kColQ;
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
+        for (int c = 0; c < kLoadChunks; ++c) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_bf16_ts_w(d, a0 + uint32_t(c * 4 + k) * 8u,
@@ -402,18 +324,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     // unit 2j at columns [8j, 8j+4) and unit 2j+1 at [8j+4, 8j+8).  All 36
     // loads of a thread are issued before the first store (one round trip).
     auto write_query = [&](int b) {
+      constexpr int kUnits = R / 16;   // 16-byte units per half-warp thread: 36, or 32 without RoPE
       const int64_t qrow = int64_t(b) * H + int64_t(g) * kHeadsPerCta + row;
       const bool valid_row = qrow < int64_t(B) * H;
-      const uint4* src = reinterpret_cast<const uint4*>(q_cat + (valid_row ? qrow : 0) * kR);
-      uint4 v[36];
+      const uint4* src = reinterpret_cast<const uint4*>(q_cat + (valid_row ? qrow : 0) * R);
+      uint4 v[kUnits];
 #pragma unroll
-      for (int j = 0; j < 36; ++j) v[j] = src[2 * j + (lo_half ? 0 : 1)];
+      for (int j = 0; j < kUnits; ++j) v[j] = src[2 * j + (lo_half ? 0 : 1)];
       if (!valid_row) {
 #pragma unroll
-        for (int j = 0; j < 36; ++j) v[j] = make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < kUnits; ++j) v[j] = make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int j = 0; j < 36; ++j) tmem_st16x2_4<4>(lo_base + kColQ + uint32_t(8 * j), v[j]);
+      for (int j = 0; j < kUnits; ++j) tmem_st16x2_4<4>(lo_base + kColQ + uint32_t(8 * j), v[j]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->q_ready);
@@ -423,20 +346,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
       if (b >= 0 && tid == 0) {
         const int64_t r0 = int64_t(b) * H + int64_t(g) * kHeadsPerCta;
         const int64_t rows = min(int64_t(kHeadsPerCta), int64_t(B) * H - r0);
-        if (rows > 0) bulk_prefetch_l2(q_cat + r0 * kR, uint32_t(rows * kR * 2));
+        if (rows > 0) bulk_prefetch_l2(q_cat + r0 * R, uint32_t(rows * R * 2));
       }
     };
 
-    // The sequence of the worker's range that follows sequence `after`
-    // (-1 for the first), or -1 if there is none.
-    auto next_sequence = [&](int after) {
-      for (int bb = (after < 0 ? tp.first_after(t_begin) : after + 1); bb < B; ++bb) {
-        const int64_t pre = tp.at(bb);
-        if (pre >= t_end) return -1;
-        if (tiles_of(tp.len(bb)) > 0 && pre + tiles_of(tp.len(bb)) > t_begin) return bb;
-      }
-      return -1;
-    };
+    auto next_sequence = [&](int after) { return tp.next_sequence(after, t_begin, t_end); };
 
     // The first sequence's query block; each later one is written as soon as
     // the previous sequence's last S has been read (all its QK^T are done),
@@ -571,6 +485,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
 
   tc_fence_before();
   __syncthreads();
+  // Every role has stopped.  Each load the producer issued lands before the
+  // shared memory is released: after a give-up some were never waited for
+  // (the last load into each stage; on the normal path these waits return at
+  // once).
+  if (warp == kProducerWarp && lane == 0) {
+    volatile int no_abort = 0;
+    for (uint32_t k = (n_issued > kStages ? n_issued - kStages : 0); k < n_issued; ++k)
+      mbar_wait(&bars->full[k % kStages], (k / kStages) & 1, &no_abort, kWaitLimitCycles);
+  }
+  __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -599,10 +523,14 @@ static EncodeTiledFn encode_tiled() {
 }
 
 bool make_cache_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
+  return make_cache_rows_map_r(map, base, rows, kR);
+}
+
+bool make_cache_rows_map_r(CUtensorMap* map, const void* base, uint64_t rows, int R) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {cuuint64_t(kR), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(kR) * 2};
+  const cuuint64_t dims[2] = {cuuint64_t(R), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(R) * 2};
   const cuuint32_t box[2] = {cuuint32_t(kChunkElems), cuuint32_t(kTileKeys)};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
@@ -612,19 +540,18 @@ bool make_cache_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
 
 int decode_tc_head_groups(int H) { return (H + kHeadsPerCta - 1) / kHeadsPerCta; }
 
-cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* cache,
-                             const PageMap& pm, const int32_t* seqlens, int B, int H, int64_t cap,
-                             float scale, int W, float* o_part, float* lse_part, int* status,
-                             cudaStream_t stream) {
-  if (pm.total_rows(B) >= (int64_t(1) << 31) || int64_t(B) * H >= (int64_t(1) << 31))
-    return cudaErrorInvalidValue;
-  CUtensorMap tm_c;
-  if (!make_cache_rows_map(&tm_c, cache, uint64_t(pm.total_rows(B)))) return cudaErrorInvalidValue;
+namespace {
+template <int kDr>
+cudaError_t launch_decode_tc_t(const CUtensorMap& tm_c, const __nv_bfloat16* q_cat,
+                               const __nv_bfloat16* cache, const PageMap& pm,
+                               const int32_t* seqlens, int B, int H, int64_t cap, float scale,
+                               int W, float* o_part, float* lse_part, int* status,
+                               uint64_t inject_wait, cudaStream_t stream) {
   static bool attr_done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel,
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<kDr>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(kSmemBytes));
     if (e != cudaSuccess) return e;
@@ -632,10 +559,27 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
   }
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(decode_tc_head_groups(H), W);
-  decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_c, cache, pm, q_cat, seqlens, B, H, cap,
-                                                           scale_log2, W, o_part, lse_part,
-                                                           status);
+  decode_tc_kernel<kDr><<<grid, kThreads, kSmemBytes, stream>>>(
+      tm_c, cache, pm, q_cat, seqlens, B, H, cap, scale_log2, W, o_part, lse_part, status,
+      inject_wait);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* cache,
+                             const PageMap& pm, const int32_t* seqlens, int B, int H, int64_t cap,
+                             int d_r, float scale, int W, float* o_part, float* lse_part,
+                             int* status, uint64_t inject_wait, cudaStream_t stream) {
+  if (d_r != 64 && d_r != 0) return cudaErrorInvalidValue;
+  if (pm.total_rows(B) >= (int64_t(1) << 31) || int64_t(B) * H >= (int64_t(1) << 31))
+    return cudaErrorInvalidValue;
+  CUtensorMap tm_c;
+  if (!make_cache_rows_map_r(&tm_c, cache, uint64_t(pm.total_rows(B)), kDc + d_r))
+    return cudaErrorInvalidValue;
+  return d_r == 64 ? launch_decode_tc_t<64>(tm_c, q_cat, cache, pm, seqlens, B, H, cap, scale, W,
+                                            o_part, lse_part, status, inject_wait, stream)
+                   : launch_decode_tc_t<0>(tm_c, q_cat, cache, pm, seqlens, B, H, cap, scale, W,
+                                           o_part, lse_part, status, inject_wait, stream);
 }
 
 }  // namespace mla

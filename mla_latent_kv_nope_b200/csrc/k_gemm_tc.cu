@@ -174,7 +174,7 @@ constexpr size_t kAbSmem = 2 * 16384 + 2 * (kAbN * 128) + 64 + 1024;
 __global__ void __launch_bounds__(kThreadsG, 1)
 absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16* __restrict__ q_nope,
                    const __nv_bfloat16* __restrict__ q_pe, const int32_t* __restrict__ q_pos,
-                   float rope_base, int B, int H, __nv_bfloat16* __restrict__ q_cat,
+                   float rope_base, int B, int H, int d_r, __nv_bfloat16* __restrict__ q_cat,
                    int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -185,7 +185,7 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
   const int i = blockIdx.x;
   const int mb = blockIdx.y;                 // output columns [128 mb, 128 mb + 128)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kR = 576;
+  const int kR = 512 + d_r;   // q_cat row: 512 absorbed columns, then the RoPE block (64 or none)
   // Rotation frequencies of the 32 RoPE pairs, computed once per CTA while
   // the weight block loads.
   __shared__ double s_inv[32];
@@ -268,8 +268,9 @@ absorb_q_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16
   // Pairs (b, k) are taken 8 per thread with every load issued before the
   // first rotation, so the pass costs one memory round trip per 8 pairs.
   constexpr int kRopeBatch = 8;
-  const int u_lo = int(int64_t(B) * 32 * mb / kAbBlocks);
-  const int u_hi = int(int64_t(B) * 32 * (mb + 1) / kAbBlocks);
+  const int n_pairs = d_r / 2;   // 32, or 0 without a RoPE block
+  const int u_lo = int(int64_t(B) * n_pairs * mb / kAbBlocks);
+  const int u_hi = int(int64_t(B) * n_pairs * (mb + 1) / kAbBlocks);
   for (int u0 = u_lo; u0 < u_hi; u0 += kRopeBatch * kThreadsG) {
     float x1[kRopeBatch], x2[kRopeBatch];
     int32_t pos[kRopeBatch];
@@ -435,7 +436,7 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }  // namespace
 
 bool gemm_tc_supported(int d_c, int d_r, int d_n, int d_v) {
-  return d_c == 512 && d_r == 64 && d_n == 128 && d_v == 128;
+  return d_c == 512 && (d_r == 64 || d_r == 0) && d_n == 128 && d_v == 128;
 }
 
 cudaError_t launch_out_proj_tc(const float* o_lat, const __nv_bfloat16* W_UV, int B, int H,
@@ -450,15 +451,16 @@ cudaError_t launch_out_proj_tc(const float* o_lat, const __nv_bfloat16* W_UV, in
 
 cudaError_t launch_absorb_q_tc(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_pe,
                                const __nv_bfloat16* W_UK, const int32_t* q_pos, float rope_base,
-                               int B, int H, __nv_bfloat16* q_cat, int* status,
+                               int B, int H, int d_r, __nv_bfloat16* q_cat, int* status,
                                cudaStream_t stream) {
+  if (d_r != 64 && d_r != 0) return cudaErrorInvalidValue;
   CUtensorMap tm;
   if (!make_map(&tm, W_UK, uint64_t(H) * 128, 512, 128)) return cudaErrorInvalidValue;
   cudaError_t e = set_smem(absorb_q_tc_kernel, kAbSmem);
   if (e != cudaSuccess) return e;
   absorb_q_tc_kernel<<<dim3(H, kAbBlocks), kThreadsG, kAbSmem, stream>>>(tm, q_nope, q_pe, q_pos,
                                                                          rope_base, B, H,
-                                                        q_cat, status);
+                                                                         d_r, q_cat, status);
   return cudaGetLastError();
 }
 

@@ -24,16 +24,20 @@ cudaError_t launch_decode_simt(const T* q_cat, const T* cache, const PageMap& pm
                                cudaStream_t stream);
 size_t decode_simt_smem_bytes(int d_c, int d_r);
 
-// Tensor-core decode (bf16, d_c = 512, d_r = 64).  Returns cudaErrorNotSupported
-// when the build has no sm_100a kernel.
+// Tensor-core decode (bf16, d_c = 512, d_r = 64 or 0).  Returns
+// cudaErrorNotSupported when the build has no sm_100a kernel.  `inject_wait`
+// > 0 adds a wait of that many SM cycles on a barrier nothing arrives on (a
+// test of the give-up path).
 cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* cache,
                              const PageMap& pm, const int32_t* seqlens, int B, int H, int64_t cap,
-                             float scale, int W, float* o_part, float* lse_part, int* status,
-                             cudaStream_t stream);
+                             int d_r, float scale, int W, float* o_part, float* lse_part,
+                             int* status, uint64_t inject_wait, cudaStream_t stream);
 int decode_tc_head_groups(int H);
 // 2D TMA map over the cache viewed as [rows, 576] bf16: 64 x 64 boxes, 128-byte
 // swizzle.  False if the driver entry point is missing or encoding fails.
 bool make_cache_rows_map(CUtensorMap* map, const void* base, uint64_t rows);
+// The same over rows of R bf16 (R a multiple of 64).
+bool make_cache_rows_map_r(CUtensorMap* map, const void* base, uint64_t rows, int R);
 
 
 cudaError_t launch_combine(const int32_t* seqlens, int64_t cap, int B, int H, int d_c, int W,
@@ -62,13 +66,13 @@ cudaError_t launch_append_finalize(const float* part, int n_parts, const float* 
                                    T* cache, const PageMap& pm, int32_t* seqlens, int* status,
                                    cudaStream_t stream);
 
-// Tensor-core kernels for the bf16 step (d_c = 512, d_r = 64, d_nope = d_v = 128).
+// Tensor-core kernels for the bf16 step (d_c = 512, d_r = 64 or 0, d_nope = d_v = 128).
 bool gemm_tc_supported(int d_c, int d_r, int d_n, int d_v);
 cudaError_t launch_out_proj_tc(const float* o_lat, const __nv_bfloat16* W_UV, int B, int H,
                                __nv_bfloat16* out, int* status, cudaStream_t stream);
 cudaError_t launch_absorb_q_tc(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_pe,
                                const __nv_bfloat16* W_UK, const int32_t* q_pos, float rope_base,
-                               int B, int H, __nv_bfloat16* q_cat, int* status,
+                               int B, int H, int d_r, __nv_bfloat16* q_cat, int* status,
                                cudaStream_t stream);
 int append_tc_splits(int hidden);
 cudaError_t launch_append_proj_tc(const __nv_bfloat16* h, const __nv_bfloat16* W_DKV, int B,

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 
 #include "../../include/mla.h"
@@ -58,13 +59,17 @@ int check_dims(const mla_dims* d) {
 
 inline bool decode_uses_tc(const mla_dims* d) { return d->dtype == MLA_BF16; }
 
+// Cycles of the test-only wait injected into the tensor-core decode (0 = none).
+uint64_t g_inject_wait_cycles = 0;
+
 cudaError_t launch_decode_any(const mla_dims* d, const void* q_cat, const void* cache,
                               const PageMap& pm, const int32_t* seqlens, float scale, int W,
                               float* o_part, float* lse_part, int* status, cudaStream_t s) {
   if (decode_uses_tc(d))
     return launch_decode_tc(static_cast<const __nv_bfloat16*>(q_cat),
                             static_cast<const __nv_bfloat16*>(cache), pm, seqlens, d->B, d->H,
-                            d->cache_capacity, scale, W, o_part, lse_part, status, s);
+                            d->cache_capacity, d->d_r, scale, W, o_part, lse_part, status,
+                            g_inject_wait_cycles, s);
   return launch_decode_simt<float>(static_cast<const float*>(q_cat),
                                    static_cast<const float*>(cache), pm, seqlens, d->B, d->H,
                                    d->d_c, d->d_r, d->cache_capacity, scale, W, o_part, lse_part,
@@ -87,7 +92,8 @@ int check_pages(const mla_dims* d, int64_t num_pages, const int32_t* block_table
 // with a 32-bit TMA coordinate, so a contiguous cache of 2^31 rows or more
 // (B * capacity) is refused here rather than failing at launch.
 int decode_shape_supported(const mla_dims* d, bool contiguous) {
-  if (d->dtype == MLA_BF16 && (d->d_c != 512 || d->d_r != 64)) return MLA_ERR_UNSUPPORTED;
+  if (d->dtype == MLA_BF16 && (d->d_c != 512 || (d->d_r != 64 && d->d_r != 0)))
+    return MLA_ERR_UNSUPPORTED;
   if (d->dtype == MLA_BF16 && contiguous &&
       int64_t(d->B) * d->cache_capacity >= (int64_t(1) << 31))
     return MLA_ERR_UNSUPPORTED;
@@ -115,6 +121,12 @@ WsLayout ws_layout(const mla_dims* d, int W) {
 }
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+// softmax_scale = 0 selects the pages' scale 1/sqrt(d_h + d_h^R) ([MLA-とは]
+// "Decoupled RoPE"): the query/key width per head is d_nope + d_r.
+inline float effective_scale(const mla_dims* d, float softmax_scale) {
+  return softmax_scale == 0.f ? float(1.0 / sqrt(double(d->d_nope + d->d_r))) : softmax_scale;
+}
 
 }  // namespace
 }  // namespace mla
@@ -146,6 +158,11 @@ int mla_get_device_status(void* stream) {
   const int zero = MLA_OK;
   if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
   return v;
+}
+
+int mla_debug_inject_wait(uint64_t cycles) {
+  g_inject_wait_cycles = cycles;
+  return MLA_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -238,7 +255,7 @@ int mla_absorb_q(const mla_dims* d, const void* q_nope, const void* q_pe, const 
   if (use_tc_gemm(d))
     return cuda_status(launch_absorb_q_tc(
         static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_pe),
-        static_cast<const __nv_bfloat16*>(W_UK), q_pos, rope_base, d->B, d->H,
+        static_cast<const __nv_bfloat16*>(W_UK), q_pos, rope_base, d->B, d->H, d->d_r,
         static_cast<__nv_bfloat16*>(q_cat), status_ptr(), s));
   if (d->dtype == MLA_BF16)
     return cuda_status(launch_absorb_q<__nv_bfloat16>(
@@ -283,8 +300,9 @@ int decode_impl(const mla_dims* d, const void* q_cat, const void* cache, const P
   if (st) return st;
   if ((st = decode_shape_supported(d, pm.table == nullptr))) return st;
   if (!q_cat || !cache || !seqlens || num_splits < 0 || num_splits > kMaxSplits ||
-      !(softmax_scale > 0.f) || softmax_scale == INFINITY)
+      !(softmax_scale >= 0.f) || softmax_scale == INFINITY)
     return MLA_ERR_INVALID_ARG;
+  softmax_scale = effective_scale(d, softmax_scale);
   if (!aligned16(q_cat) || !aligned16(cache) || !aligned16(seqlens) ||
       (workspace && !aligned16(workspace)))
     return MLA_ERR_ALIGNMENT;
@@ -380,10 +398,9 @@ int mla_out_proj(const mla_dims* d, const float* o_lat, const void* W_UV, void* 
 // ---------------------------------------------------------------------------
 // Decode + combine for callers that cannot allocate device memory.
 //
-// Some callers cannot call cudaMalloc at all: code running while a stream is
-// being captured into a CUDA graph (allocation is illegal there), plugins
-// handed a fixed set of buffers by a host framework, or runtimes whose memory
-// is owned by another allocator.  For them the split-KV partials live in the
+// Some callers cannot call cudaMalloc at all: plugins handed a fixed set of
+// buffers by a host framework, or runtimes whose device memory is owned by
+// another allocator.  For them the split-KV partials live in the
 // file-scope array below instead of a caller-provided workspace.  It is sized
 // once (MLA_DECODE_NOALLOC_SCRATCH_BYTES) and every device that loads this
 // library holds it until the process exits.
@@ -416,9 +433,10 @@ extern "C" int mla_decode_noalloc(const mla_dims* d, const void* q_cat, const vo
   int st = check_dims(d);
   if (st) return st;
   if ((st = decode_shape_supported(d, true))) return st;
-  if (!q_cat || !cache || !seqlens || !o_lat || !(softmax_scale > 0.f) ||
+  if (!q_cat || !cache || !seqlens || !o_lat || !(softmax_scale >= 0.f) ||
       softmax_scale == INFINITY)
     return MLA_ERR_INVALID_ARG;
+  softmax_scale = effective_scale(d, softmax_scale);
   if (!aligned16(q_cat) || !aligned16(cache) || !aligned16(seqlens) || !aligned16(o_lat) ||
       (lse && !aligned16(lse)))
     return MLA_ERR_ALIGNMENT;

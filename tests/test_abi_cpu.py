@@ -58,8 +58,9 @@ def test_row_elems_and_status_strings(lib):
 
 
 def test_workspace_layout_formula(lib):
-    for B, H, W in [(4, 16, 148), (32, 128, 74), (64, 64, 148), (1, 4, 3)]:
-        d = _dims(B=B, H=H)
+    for B, H, W, d_r in [(4, 16, 148, 64), (32, 128, 74, 64), (64, 64, 148, 64), (1, 4, 3, 64),
+                         (3, 192, 37, 64), (4, 16, 74, 0)]:
+        d = _dims(B=B, H=H, d_r=d_r)
         slots = B + W - 1
         r256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
         expect = r256(slots * H * 512 * 4) + r256(slots * H * 4)
@@ -103,7 +104,8 @@ def test_decode_argument_errors(lib):
     assert lib.mla_decode_noalloc(ctypes.byref(big), GOOD, GOOD, GOOD, 0.07, GOOD2, None,
                                   None) == UNSUP
     assert call(d, q=None) == INVALID
-    assert call(d, scale=0.0) == INVALID
+    assert call(d, scale=-0.5) == INVALID
+    assert call(d, scale=float("inf")) == INVALID
     assert call(d, scale=float("nan")) == INVALID
     assert call(d, W=-1) == INVALID
     assert call(d, W=5000) == INVALID

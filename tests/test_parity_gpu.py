@@ -173,6 +173,11 @@ DECODE_CASES = [
     ("bf16-H128-peaked-long", W["v3_bf16"].scaled(B=1, N=3000), [3000], 2, 10.0),
     ("bf16-H100", W["v3_bf16"].scaled(B=3, H=100, N=300), [300, 65, 0], 0, 1.0),
     ("bf16-H192", W["v3_bf16"].scaled(B=2, H=192, N=200), [200, 64], 0, 1.0),
+    # NoPE ([yuuk] 横断的知見: MLA layers without RoPE): d_r = 0, rows are c^KV alone
+    ("bf16-nope-H128", W["v3_bf16"].scaled(B=3, N=600, d_r=0), [600, 129, 1], 0, 1.0),
+    ("bf16-nope-H64", W["ragged_append_bf16"].scaled(B=4, N=300, d_r=0), [300, 64, 1, 0], 0,
+     1.0),
+    ("bf16-nope-H16-peaked", SMALL_BF16.scaled(B=2, d_r=0), [190, 64], 0, 10.0),
 ]
 
 
@@ -183,6 +188,23 @@ def test_decode_combine(name, w, lens, nsplit, boost):
     scale = w.softmax_scale * boost
     got_o, got_l = _run_decode(w, lens, q_cat, scale, nsplit)
     ref_o, ref_l = _oracle_latent(w, lens, q_cat, scale)
+    nz = lens > 0
+    assert rel_l2(got_o[nz], ref_o[nz]) < tol(w)
+    assert np.all(got_o[~nz] == 0)
+    assert _lse_err(got_l, ref_l) < tol(w)
+
+
+@pytest.mark.parametrize("w", [SMALL_BF16.scaled(B=1100, N=40),
+                               W["v3_bf16"].scaled(B=1030, N=24)],
+                         ids=["H16-B1100", "H128-B1030"])
+def test_decode_more_sequences_than_the_shared_prefix(w):
+    """More than 1024 sequences: the decode kernels walk the length array in
+    global memory instead of their shared-memory tile prefix.  Short ragged
+    lengths (0 included); every sequence is checked against the oracle."""
+    lens = np.random.default_rng(5).integers(0, w.N + 1, size=w.B).astype(np.int32)
+    q_cat = inputs.normal((w.B, w.H, w.R), 0.5, 31, w.B)
+    got_o, got_l = _run_decode(w, lens, q_cat, w.softmax_scale)
+    ref_o, ref_l = _oracle_latent(w, lens, q_cat, w.softmax_scale)
     nz = lens > 0
     assert rel_l2(got_o[nz], ref_o[nz]) < tol(w)
     assert np.all(got_o[~nz] == 0)
@@ -386,6 +408,11 @@ SMALL_STEPS = [
     # row is c^KV alone and the query has no decoupled part (fp32 path).
     W["tiny_f32"].scaled(name="tiny_f32_nope", B=3, N=150, d_r=0, ragged=True, append=True,
                          hidden=64),
+    # NoPE on the bf16 tensor-core path at the production latent width (d_c = 512):
+    # 128 heads (CTA pairs) and 64 heads, with the append
+    W["v3_bf16"].scaled(name="v3_bf16_nope", B=3, N=300, d_r=0, ragged=True, append=True,
+                        hidden=512),
+    W["ragged_append_bf16"].scaled(name="ragged_bf16_nope", B=5, N=400, d_r=0, hidden=512),
 ]
 
 

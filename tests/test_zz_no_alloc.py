@@ -1,10 +1,10 @@
 """The allocation-free decode entry point, mla_decode_noalloc, gives the same
 result as mla_decode + mla_combine with a caller workspace.
 
-It exists for callers that cannot allocate device memory (for example code
-that runs while a stream is being captured into a CUDA graph, or a plugin
-that only receives fixed buffers): its split-KV partials live in a fixed
-array inside the library.  The test calls it through the C ABI twice in a row
+It exists for callers that cannot allocate device memory (for example a
+plugin that only receives fixed buffers from its host framework, or a
+runtime whose device memory belongs to another allocator): its split-KV
+partials live in a fixed array inside the library.  The test calls it through the C ABI twice in a row
 on different inputs -- the shared array keeps the first call's contents, which
 must not leak into the second -- and compares each result with the workspace
 path, within the parity tolerances used elsewhere.  It builds and loads the
