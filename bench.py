@@ -165,12 +165,14 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-def _algorithmic(w, lens_after):
+def _algorithmic(w, lens_after, fp8=False):
     """Latent-cache bytes and FLOPs of one decode launch (cache read once;
-    QK^T over d_c + d_r and P.c over d_c per head and cached row)."""
+    QK^T over d_c + d_r and P.c over d_c per head and cached row).  An FP8
+    cache row is d_c code bytes + d_r bf16 RoPE keys + a 4-byte scale."""
     rows = int(sum(int(x) for x in lens_after))
     elem = 2 if w.dtype == "bf16" else 4
-    return rows * w.R * elem, 2.0 * w.H * rows * (w.R + w.d_c), rows
+    row_bytes = (w.d_c + 2 * w.d_r + 4) if fp8 else w.R * elem
+    return rows * row_bytes, 2.0 * w.H * rows * (w.R + w.d_c), rows
 
 
 def run_ours(args, rank, world, local_rank):
@@ -194,8 +196,17 @@ def run_ours(args, rank, world, local_rank):
     dims = mla.Dims(w.B, w.H, w.d_c, w.d_r, w.d_nope, w.d_v, w.capacity, w.dtype)
 
     lens = inputs.seqlens(w)
-    cache = torch.empty(w.B, w.capacity, w.R, dtype=dt, device=dev)
-    inputs.fill_cache(w, cache, lens, fill_rest=0.0)
+    fp8 = args.cache == "fp8"
+    scales = None
+    if fp8:
+        # The FP8 cache drawn in its stored format (codes, power-of-two
+        # scales, bf16 RoPE keys); the append writes its own rows.
+        cache = torch.empty(w.B, w.capacity, w.d_c + 2 * w.d_r, dtype=torch.uint8, device=dev)
+        scales = torch.empty(w.B, w.capacity, dtype=torch.float32, device=dev)
+        inputs.fill_fp8_cache(w, cache, scales, lens, fill_rest_byte=0)
+    else:
+        cache = torch.empty(w.B, w.capacity, w.R, dtype=dt, device=dev)
+        inputs.fill_cache(w, cache, lens, fill_rest=0.0)
     table = None
     if args.paged:
         # The same rows in a pool of 64-row pages, pages shuffled, and the
@@ -219,7 +230,7 @@ def run_ours(args, rank, world, local_rank):
     step = mla.DecodeStep(dims, W_UK, W_UV, W_DKV, num_splits=args.splits)
     stream = torch.cuda.current_stream()
 
-    cache_bytes = cache.numel() * cache.element_size()
+    cache_bytes = cache.numel() * cache.element_size() + (scales.numel() * 4 if fp8 else 0)
     flush = None
     if cache_bytes < 2 * L2_BYTES:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -227,7 +238,7 @@ def run_ours(args, rank, world, local_rank):
     def eager_step():
         if flush is not None:
             flush.zero_()
-        step(q_nope, q_pe, q_pos, cache, seq, h=hh, block_table=table)
+        step(q_nope, q_pe, q_pos, cache, seq, h=hh, block_table=table, scales=scales)
         seq.copy_(seq0)
 
     # A step is replayed from a CUDA graph (one host launch per step) unless
@@ -240,21 +251,24 @@ def run_ours(args, rank, world, local_rank):
     else:
         graph = step.capture(q_nope, q_pe, q_pos, cache, seq, h=hh,
                              before=(flush.zero_ if flush is not None else None),
-                             after=lambda: seq.copy_(seq0), block_table=table)
+                             after=lambda: seq.copy_(seq0), block_table=table, scales=scales)
         one_step = graph.replay
 
     # Decode-kernel-only events (for the roofline): separate pass so that
     # the step timing has no extra event records inside it.
     def decode_only(n):
         evs = []
-        step.append(hh, cache, seq, table)
+        step.append(hh, cache, seq, table, scales)
         mla.absorb_q(dims, q_nope, q_pe, W_UK, q_pos, step.q_cat, step.rope_base)
         for _ in range(n):
             if flush is not None:
                 flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            if table is None:
+            if fp8:
+                mla.decode_fp8(dims, step.q_cat, cache, scales, seq, step.scale, step.ws,
+                               step.num_splits)
+            elif table is None:
                 mla.decode(dims, step.q_cat, cache, seq, step.scale, step.ws, step.num_splits)
             else:
                 mla.decode_paged(dims, step.q_cat, cache, table, seq, step.scale, step.ws,
@@ -314,7 +328,7 @@ def run_ours(args, rank, world, local_rank):
                     d_t.copy_(h_t, non_blocking=True)
                 if flush is not None:
                     flush.zero_()
-                step(q_nope, q_pe, q_pos, cache, seq, h=hh, block_table=table)
+                step(q_nope, q_pe, q_pos, cache, seq, h=hh, block_table=table, scales=scales)
                 h_out.copy_(step.out, non_blocking=True)
                 seq.copy_(seq0)
     else:
@@ -334,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
                 stage.copy_(step.out)
                 seq.copy_(seq0)
             g = step.capture(d_in[0], d_in[1], d_in[2], cache, seq, h=d_in[3], after=after,
-                             block_table=table)
+                             block_table=table, scales=scales)
             sets.append((d_in, stage, g))
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -384,7 +398,7 @@ def run_ours(args, rank, world, local_rank):
         return None
     hbm, tf_burst, tf_sus, peak_src = _peaks()
     lens_after = lens + 1
-    byts, flops, rows = _algorithmic(w, lens_after)
+    byts, flops, rows = _algorithmic(w, lens_after, fp8)
     dec_avg = sum(dec_ms) / len(dec_ms)
     decomb_avg = sum(decomb_ms) / len(decomb_ms)
     achieved_gbs = byts / (dec_avg * 1e-3) / 1e9
@@ -414,7 +428,8 @@ def run_ours(args, rank, world, local_rank):
                   else "L2 flushed between steps",
             "num_splits": step.splits_used,
             "cache": ("paged: 64-row pages, shuffled, block table" if args.paged
-                      else "contiguous [B, capacity, 576]"),
+                      else "fp8: E4M3 latent codes + bf16 RoPE keys (640 B) + fp32 scale per token"
+                      if fp8 else "contiguous [B, capacity, 576]"),
             "launch": "eager" if args.eager else "cuda_graph (absorb_q on a forked stream)",
         },
         "decode_only": {
@@ -434,7 +449,7 @@ def run_ours(args, rank, world, local_rank):
             "peak": hbm if bound == "hbm" else tf_burst,
             "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "frac": (achieved_gbs / hbm) if bound == "hbm" else (achieved_tf / tf_burst),
-            "traffic": _ncu_traffic(args.workload),
+            "traffic": _ncu_traffic(args.workload + ("_fp8" if fp8 else "")),
             "algorithmic_bytes_per_launch": byts,
             "algorithmic_flops_per_launch": flops,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured"
@@ -446,7 +461,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_oracle_baseline(w, args.cpu_seconds)
+        res["cpu_baseline"] = cpu_oracle_baseline(w, args.cpu_seconds, fp8)
     return res
 
 
@@ -485,7 +500,7 @@ class OracleSampler:
     (cycling through the sample) until about ``budget_s`` of oracle time and
     scales to tokens/s by the number of (sequence, head) pairs in a step."""
 
-    def __init__(self, w, max_seqs=8):
+    def __init__(self, w, max_seqs=8, fp8=False):
         import numpy as np
 
         from mla_latent_kv_nope_b200 import inputs
@@ -501,10 +516,17 @@ class OracleSampler:
         rng = np.random.default_rng(0)
         seqs = sorted(int(b) for b in rng.choice(w.B, size=min(max_seqs, w.B), replace=False))
         self.caches = {}
+        self.fp8 = fp8
         for b in seqs:
             L = int(self.lens[b])
             c = np.zeros((1, L + 1, w.R))
-            c[0, :L] = inputs.cache_rows(w, b, L)
+            if fp8:
+                from oracle import mla_oracle as O
+                codes, k, rope = inputs.fp8_cache_rows(w, b, L)
+                c[0, :L, :w.d_c] = O.dequantize_latent_rows(codes, np.ldexp(1.0, k))
+                c[0, :L, w.d_c:] = rope
+            else:
+                c[0, :L] = inputs.cache_rows(w, b, L)
             self.caches[b] = c
         self.pairs = [(b, int(i)) for i in rng.permutation(w.H) for b in seqs]
         self.k = 0
@@ -532,13 +554,14 @@ class OracleSampler:
                 "kind": "oracle", "extrapolated": True, "cpu_model": _cpu_model(),
                 "host_cores": os.cpu_count(),
                 "sample": f"{done} (sequence, head) pairs from {len(self.caches)} seeded random "
+                          f"{'FP8 (dequantised) ' if self.fp8 else ''}"
                           f"sequences ({spent:.1f} s of oracle time), each append + "
                           f"materialised attention over its full length; scaled by "
                           f"B*H = {w.B * w.H} pairs per step"}
 
 
-def cpu_oracle_baseline(w, budget_s=15.0):
-    return OracleSampler(w).run(budget_s)
+def cpu_oracle_baseline(w, budget_s=15.0, fp8=False):
+    return OracleSampler(w, fp8=fp8).run(budget_s)
 
 
 def run_reference(args, rank, world):
@@ -633,6 +656,9 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"],
+                    help="latent cache format (fp8: E4M3 codes with a power-of-two scale "
+                         "per token, bf16 RoPE keys)")
     ap.add_argument("--paged", action="store_true",
                     help="keep the latent cache in shuffled 64-row pages behind a block table")
     ap.add_argument("--eager", action="store_true",
@@ -640,6 +666,8 @@ def main():
     ap.add_argument("--dry-run", action="store_true",
                     help="host-only check of the multi-rank launch and timing (gloo, no GPU)")
     args = ap.parse_args()
+    if args.cache == "fp8" and args.paged:
+        ap.error("the FP8 latent cache is contiguous only")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.gpus < 1:

@@ -182,6 +182,35 @@ MLA_API int mla_merge_partials(const mla_dims* dims, int n_parts, const float* o
 MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W_UV,
                  void* out, void* stream);
 
+/* --- FP8 latent cache ------------------------------------------------------------
+ * [abeam] "モデル全体でも推論効率が大きく改善した" names KV-cache quantisation as
+ * part of the system's serving efficiency, and [yuuk] "未解決の問い" leaves FP8
+ * for MLA open; the format is this library's (the pages fix none).  A cached
+ * token is a row of mla_cache_fp8_row_bytes(d_c, d_r) = d_c + 2 d_r bytes:
+ * d_c E4M3 codes (OCP E4M3, finite-only: largest 448, no infinities) of the
+ * normalised latent, then the d_r RoPE keys in bf16, plus one fp32 scale per
+ * token in a separate plane scales [B, cache_capacity]:
+ *   c~_j = E4M3(code_j) * scale,  scale = the smallest power of two 2^k with
+ *   max_j |c_j| / 2^k <= 448 (a row of zeros gets 1),
+ *   code_j = c_j / scale rounded to nearest E4M3 (ties to even), saturating.
+ * Shape: bf16, d_c = 512, d_r = 64, d_nope = d_v = 128; contiguous cache only.
+ * mla_cache_append_fp8 is mla_cache_append (same h, W_DKV, gamma, eps,
+ * rope_base, seqlens, workspace) writing row L_b of cache [B, capacity,
+ * 640 bytes] and scales[b, L_b].  mla_decode_fp8 is mla_decode over the
+ * dequantised rows [c~ || k^R] (same q_cat, seqlens, scale, splits,
+ * workspace, partial layout; mla_combine merges as usual).  Rows past L_b
+ * may hold anything. */
+MLA_API int64_t mla_cache_fp8_row_bytes(int32_t d_c, int32_t d_r);
+MLA_API int mla_cache_append_fp8(const mla_dims* dims, int32_t hidden, const void* h,
+                                 const void* W_DKV, const float* gamma, float eps,
+                                 float rope_base, void* cache_fp8, float* scales,
+                                 int32_t* seqlens, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+MLA_API int mla_decode_fp8(const mla_dims* dims, const void* q_cat, const void* cache_fp8,
+                           const float* scales, const int32_t* seqlens, float softmax_scale,
+                           int num_splits, void* workspace, size_t workspace_bytes,
+                           int* splits_used, void* stream);
+
 /* --- paged latent cache --------------------------------------------------------
  * No counterpart on the pages beyond the name: [MLA-とは] names PagedAttention
  * as the serving-side cache organisation this method fits; the page size is

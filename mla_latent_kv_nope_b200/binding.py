@@ -27,7 +27,8 @@ EXPORTED = (
     "mla_absorb_q", "mla_decode_default_splits", "mla_decode_workspace_bytes",
     "mla_decode", "mla_combine", "mla_out_proj", "mla_get_device_status",
     "mla_status_string", "mla_decode_noalloc", "mla_decode_paged", "mla_cache_append_paged",
-    "mla_merge_partials", "mla_debug_inject_wait",
+    "mla_merge_partials", "mla_debug_inject_wait", "mla_cache_fp8_row_bytes",
+    "mla_cache_append_fp8", "mla_decode_fp8",
 )
 
 PAGE_ROWS = 64   # rows per page of a paged latent cache (one decode work tile)
@@ -107,6 +108,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_merge_partials": (ctypes.c_int, [D, ctypes.c_int, P, P, P, P, P]),
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "mla_debug_inject_wait": (ctypes.c_int, [ctypes.c_uint64]),
+        "mla_cache_fp8_row_bytes": (I64, [I32, I32]),
+        "mla_cache_append_fp8": (ctypes.c_int, [D, I32, P, P, P, F, F, P, P, P, P, SZ, P]),
+        "mla_decode_fp8": (ctypes.c_int, [D, P, P, P, P, F, ctypes.c_int, P, SZ,
+                                          ctypes.POINTER(ctypes.c_int), P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -227,6 +232,54 @@ def decode_paged(dims: Dims, q_cat, cache_pool, block_table, seqlens, softmax_sc
         _ptr(workspace), workspace.numel() * workspace.element_size(), ctypes.byref(used),
         _stream(stream))
     _check("mla_decode_paged", st)
+    return used.value
+
+
+def cache_fp8_row_bytes(d_c: int, d_r: int) -> int:
+    """Bytes of one FP8 latent cache row: d_c E4M3 codes + d_r bf16 RoPE keys."""
+    return int(load_library().mla_cache_fp8_row_bytes(d_c, d_r))
+
+
+def _need_fp8_cache(dims: Dims, cache, scales):
+    rb = dims.d_c + 2 * dims.d_r
+    _need(cache, torch.uint8, (dims.B, dims.cache_capacity, rb), "cache_fp8")
+    _need(scales, torch.float32, (dims.B, dims.cache_capacity), "scales")
+
+
+def cache_append_fp8(dims: Dims, h, W_DKV, gamma, cache, scales, seqlens, workspace, eps=1e-6,
+                     rope_base=10000.0, stream=None):
+    """mla_cache_append_fp8: as cache_append, into an FP8 latent cache
+    (cache [B, capacity, d_c + 2 d_r] uint8, scales [B, capacity] fp32)."""
+    dt = dims.torch_dtype
+    hidden = h.shape[-1]
+    _need(h, dt, (dims.B, hidden), "h")
+    _need(W_DKV, dt, (dims.R, hidden), "W_DKV")
+    _need_fp8_cache(dims, cache, scales)
+    _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    if gamma is not None:
+        _need(gamma, torch.float32, (dims.d_c,), "gamma")
+    _need_ws(workspace)
+    st = load_library().mla_cache_append_fp8(
+        ctypes.byref(dims.c()), hidden, _ptr(h), _ptr(W_DKV), _ptr(gamma), eps, rope_base,
+        _ptr(cache), _ptr(scales), _ptr(seqlens), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("mla_cache_append_fp8", st)
+
+
+def decode_fp8(dims: Dims, q_cat, cache, scales, seqlens, softmax_scale, workspace,
+               num_splits=0, stream=None) -> int:
+    """mla_decode_fp8: mla_decode over an FP8 latent cache; returns the splits used."""
+    _need(q_cat, dims.torch_dtype, (dims.B, dims.H, dims.R), "q_cat")
+    _need_fp8_cache(dims, cache, scales)
+    _need(seqlens, torch.int32, (dims.B,), "seqlens")
+    _need_ws(workspace)
+    used = ctypes.c_int(0)
+    st = load_library().mla_decode_fp8(ctypes.byref(dims.c()), _ptr(q_cat), _ptr(cache),
+                                       _ptr(scales), _ptr(seqlens), float(softmax_scale),
+                                       num_splits, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       ctypes.byref(used), _stream(stream))
+    _check("mla_decode_fp8", st)
     return used.value
 
 
@@ -360,8 +413,11 @@ class DecodeStep:
         self.splits_used = self.num_splits
         self._side = torch.cuda.Stream(device=device) if overlap else None
 
-    def append(self, h, cache, seqlens, block_table=None):
-        if block_table is None:
+    def append(self, h, cache, seqlens, block_table=None, scales=None):
+        if scales is not None:
+            cache_append_fp8(self.dims, h, self.W_DKV, self.gamma, cache, scales, seqlens,
+                             self.ws_append, self.eps, self.rope_base)
+        elif block_table is None:
             cache_append(self.dims, h, self.W_DKV, self.gamma, cache, seqlens, self.ws_append,
                          self.eps, self.rope_base)
         else:
@@ -372,8 +428,11 @@ class DecodeStep:
         """absorb_q into the step's q_cat buffer."""
         absorb_q(self.dims, q_nope, q_pe, self.W_UK, q_pos, self.q_cat, self.rope_base)
 
-    def _attend_latent(self, cache, seqlens, block_table=None):
-        if block_table is None:
+    def _attend_latent(self, cache, seqlens, block_table=None, scales=None):
+        if scales is not None:
+            self.splits_used = decode_fp8(self.dims, self.q_cat, cache, scales, seqlens,
+                                          self.scale, self.ws, self.num_splits)
+        elif block_table is None:
             self.splits_used = decode(self.dims, self.q_cat, cache, seqlens, self.scale, self.ws,
                                       self.num_splits)
         else:
@@ -383,17 +442,20 @@ class DecodeStep:
         out_proj(self.dims, self.o_lat, self.W_UV, self.out)
         return self.out
 
-    def attend(self, q_nope, q_pe, q_pos, cache, seqlens, block_table=None):
+    def attend(self, q_nope, q_pe, q_pos, cache, seqlens, block_table=None, scales=None):
         self.absorb(q_nope, q_pe, q_pos)
-        return self._attend_latent(cache, seqlens, block_table)
+        return self._attend_latent(cache, seqlens, block_table, scales)
 
-    def __call__(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, block_table=None):
+    def __call__(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, block_table=None,
+                 scales=None):
         """One step.  With ``block_table`` the cache is a paged pool
-        [num_pages, 64, R] (see decode_paged)."""
+        [num_pages, 64, R] (see decode_paged); with ``scales`` it is an FP8
+        latent cache [B, capacity, d_c + 2 d_r] uint8 with its scale plane
+        [B, capacity] (see decode_fp8)."""
         if self._side is None:
             if h is not None:
-                self.append(h, cache, seqlens, block_table)
-            return self.attend(q_nope, q_pe, q_pos, cache, seqlens, block_table)
+                self.append(h, cache, seqlens, block_table, scales)
+            return self.attend(q_nope, q_pe, q_pos, cache, seqlens, block_table, scales)
         main = torch.cuda.current_stream()
         # Fork: the side stream starts after everything issued so far (the
         # previous step's decode has finished reading q_cat).
@@ -401,12 +463,12 @@ class DecodeStep:
         with torch.cuda.stream(self._side):
             self.absorb(q_nope, q_pe, q_pos)
         if h is not None:
-            self.append(h, cache, seqlens, block_table)
+            self.append(h, cache, seqlens, block_table, scales)
         main.wait_stream(self._side)
-        return self._attend_latent(cache, seqlens, block_table)
+        return self._attend_latent(cache, seqlens, block_table, scales)
 
     def capture(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, before=None, after=None,
-                block_table=None):
+                block_table=None, scales=None):
         """Record one step into a CUDA graph; ``before``/``after`` are optional
         callables whose device work is recorded around it.  Replay with
         ``graph.replay()``; inputs are read from the same tensors each time."""
@@ -414,7 +476,8 @@ class DecodeStep:
         with torch.cuda.graph(g):
             if before is not None:
                 before()
-            self(q_nope, q_pe, q_pos, cache, seqlens, h=h, block_table=block_table)
+            self(q_nope, q_pe, q_pos, cache, seqlens, h=h, block_table=block_table,
+                 scales=scales)
             if after is not None:
                 after()
         return g

@@ -10,6 +10,8 @@
 // dimension, then a block reduction; it writes x to the fp32 workspace.  The
 // finalize pass (block per sequence) applies the norm, the rotation and the
 // single rounding, checks the capacity, writes row L_b and bumps L_b.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -136,7 +138,114 @@ append_finalize_kernel(const float* __restrict__ part, int n_parts,
   if (threadIdx.x == 0) seqlens[b] = L + 1;
 }
 
+// FP8 latent cache row: d_c E4M3 codes (bytes) then d_r bf16 RoPE keys.
+// c = RMSNorm(x[0:d_c]) * gamma as above; its scale is the smallest power of
+// two 2^k with max|c| / 2^k <= 448 (a zero row gets 1), and each code is
+// c / 2^k rounded to nearest (ties to even) in E4M3, saturating at +-448.
+__global__ void __launch_bounds__(1024)
+append_finalize_fp8_kernel(const float* __restrict__ part, int n_parts,
+                           const float* __restrict__ gamma, float eps, float rope_base, int d_c,
+                           int d_r, int64_t cap, uint8_t* __restrict__ cache,
+                           float* __restrict__ scales, const PageMap pm,
+                           int32_t* __restrict__ seqlens, int* __restrict__ status) {
+  const int b = blockIdx.x;
+  const int B = gridDim.x;
+  const int R = d_c + d_r;
+  const int row_bytes = d_c + 2 * d_r;
+  extern __shared__ float s_x[];  // [R]
+  __shared__ float s_part[32];
+  __shared__ int32_t s_L;
+  if (threadIdx.x == 0) s_L = seqlens[b];
+  for (int c = threadIdx.x; c < R; c += blockDim.x) {
+    const float* src = part + int64_t(b) * R + c;
+    const int64_t stride = int64_t(B) * R;
+    float v = 0.f;
+    for (int p0 = 0; p0 < n_parts; p0 += kFinBatch) {
+      float x[kFinBatch];
+#pragma unroll
+      for (int j = 0; j < kFinBatch; ++j) x[j] = p0 + j < n_parts ? src[(p0 + j) * stride] : 0.f;
+#pragma unroll
+      for (int j = 0; j < kFinBatch; ++j) v += x[j];
+    }
+    s_x[c] = v;
+  }
+  __syncthreads();
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) ss = fmaf(s_x[c], s_x[c], ss);
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  const int32_t L = s_L;
+  if (L < 0 || int64_t(L) >= cap) {
+    if (threadIdx.x == 0) record_status(status, MLA_ERR_BOUNDS);
+    return;
+  }
+  float tot = 0.f;
+#pragma unroll
+  for (int wdx = 0; wdx < int(blockDim.x / 32); ++wdx) tot += s_part[wdx];
+  const float inv = 1.f / sqrtf(tot / float(d_c) + eps);
+  const int64_t r = pm.row(b, L);
+  if (r < 0) {
+    if (threadIdx.x == 0) record_status(status, MLA_ERR_BOUNDS);
+    return;
+  }
+  __syncthreads();   // every thread has read s_part before it is reused
+  // The normalised latent (fp32) and its largest magnitude.
+  float amax = 0.f;
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
+    const float v = s_x[c] * inv * (gamma ? gamma[c] : 1.f);
+    s_x[c] = v;
+    amax = fmaxf(amax, fabsf(v));
+  }
+  amax = warp_max(amax);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = 0.f;
+#pragma unroll
+  for (int wdx = 0; wdx < int(blockDim.x / 32); ++wdx) amax = fmaxf(amax, s_part[wdx]);
+  // amax = f * 2^e with f in [0.5, 1); 448 = 0.875 * 2^9, so the smallest k
+  // with amax / 2^k <= 448 is e - 9 when f <= 0.875, else e - 8.
+  int k = 0;
+  if (amax > 0.f) {
+    int e;
+    const float f = frexpf(amax, &e);
+    k = f <= 0.875f ? e - 9 : e - 8;
+  }
+  const float inv_scale = ldexpf(1.f, -k);
+  uint8_t* row = cache + r * row_bytes;
+  for (int c = 2 * threadIdx.x; c < d_c; c += 2 * blockDim.x) {
+    const __nv_fp8x2_storage_t q = __nv_cvt_float2_to_fp8x2(
+        make_float2(s_x[c] * inv_scale, s_x[c + 1] * inv_scale), __NV_SATFINITE, __NV_E4M3);
+    *reinterpret_cast<__nv_fp8x2_storage_t*>(row + c) = q;
+  }
+  __nv_bfloat16* rope = reinterpret_cast<__nv_bfloat16*>(row + d_c);
+  const int half = d_r / 2;
+  for (int kk = threadIdx.x; kk < half; kk += blockDim.x) {
+    float cs, sn;
+    rope_cos_sin(L, kk, d_r, rope_base, &cs, &sn);
+    const float x1 = s_x[d_c + kk], x2 = s_x[d_c + kk + half];
+    rope[kk] = __float2bfloat16_rn(x1 * cs - x2 * sn);
+    rope[kk + half] = __float2bfloat16_rn(x1 * sn + x2 * cs);
+  }
+  if (threadIdx.x == 0) scales[r] = ldexpf(1.f, k);
+  __syncthreads();
+  if (threadIdx.x == 0) seqlens[b] = L + 1;
+}
+
 }  // namespace
+
+cudaError_t launch_append_finalize_fp8(const float* part, int n_parts, const float* gamma,
+                                       float eps, float rope_base, int B, int d_c, int d_r,
+                                       int64_t cap, uint8_t* cache, float* scales,
+                                       const PageMap& pm, int32_t* seqlens, int* status,
+                                       cudaStream_t stream) {
+  const size_t smem = sizeof(float) * size_t(d_c + d_r);
+  const int threads = min(1024, (d_c + d_r + 31) / 32 * 32);
+  append_finalize_fp8_kernel<<<B, threads, smem, stream>>>(part, n_parts, gamma, eps, rope_base,
+                                                           d_c, d_r, cap, cache, scales, pm,
+                                                           seqlens, status);
+  return cudaGetLastError();
+}
 
 template <typename T>
 cudaError_t launch_cache_append(const T* h, const T* W_DKV, const float* gamma, float eps,

@@ -39,6 +39,7 @@
 // a shared abort flag, records MLA_ERR_DEVICE_TIMEOUT, drains its own loads
 // and MMAs, frees TMEM and exits.
 #include <cuda.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -64,7 +65,16 @@ constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;                           // QK^T; owns the TMEM allocation
 constexpr int kPvWarp = 6;                            // P.C
-constexpr int kThreads = 32 * (kSoftmaxWarps + 3);    // 224
+constexpr int kWidenWarp0 = 7;                        // FP8 cache: warps 7-10 widen codes
+constexpr int kWidenThreads = 128;
+// 224 threads; 352 with the FP8 cache's widen warps.
+template <bool kFp8>
+struct Threads { static constexpr int n = 32 * (kSoftmaxWarps + 3) + (kFp8 ? kWidenThreads : 0); };
+// FP8 cache rows: 512 E4M3 codes then 64 bf16 RoPE keys (640 bytes); a stage
+// receives the 4 code boxes [64 rows x 128 codes] in chunks 4-7 and the RoPE
+// box in chunk 8.
+constexpr int kFp8RowBytes = 512 + 2 * 64;
+constexpr uint32_t kFp8LoadBytes = 5 * 8192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;                         // lo lanes, 2 x 64 columns
 constexpr uint32_t kColQ = 128;                       // lo lanes, 288 columns
@@ -81,6 +91,8 @@ struct Barriers {
   uint64_t o_free;
   uint64_t mma_drain, pv_drain;
   uint64_t never;                 // injected test wait: nothing ever arrives on it
+  uint64_t widened[kStages];      // FP8 cache: the stage holds bf16 latent rows
+  uint64_t wsync[kStages];        // FP8 cache: every widen thread has read its codes
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -116,17 +128,37 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-template <int kDr>
-__global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* __restrict__ cache,
+// 8 E4M3 codes (little-endian in `c`) times the row's power-of-two scale, as
+// 8 bf16 (exact: an E4M3 value has 4 significant bits and scale * value stays
+// in range for the scales the append produces).
+__device__ __forceinline__ uint4 widen_e4m3x8(uint2 c, float scale) {
+  uint32_t out[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t word = p < 2 ? c.x : c.y;
+    const __nv_fp8x2_storage_t pair = __nv_fp8x2_storage_t((word >> (16 * (p & 1))) & 0xFFFFu);
+    const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+    out[p] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+template <int kDr, bool kFp8>
+__global__ void __launch_bounds__(Threads<kFp8>::n, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_codes,
+                 const __nv_bfloat16* __restrict__ cache, const float* __restrict__ scales,
                  const PageMap pm,
                  const __nv_bfloat16* __restrict__ q_cat,
                  const int32_t* __restrict__ seqlens, int B, int H, int64_t cap,
                  float scale_log2, int W, float* __restrict__ o_part,
                  float* __restrict__ lse_part, int* __restrict__ status, uint64_t inject_wait) {
+  static_assert(!kFp8 || kDr == 64, "the FP8 cache carries the 64-wide RoPE keys");
   constexpr int R = kDc + kDr;                    // cache row and q_cat row width
-  constexpr int kLoadChunks = R / kChunkElems;    // chunks that come from the cache
-  constexpr uint32_t kLoadBytes = kLoadChunks * kChunkBytes;
+  constexpr int kLoadChunks = R / kChunkElems;    // bf16 chunks the QK^T product reads
+  constexpr uint32_t kLoadBytes = kFp8 ? kFp8LoadBytes : kLoadChunks * kChunkBytes;
+  constexpr int kRowBytes = kFp8 ? kFp8RowBytes : R * 2;
+  const uint8_t* cache_bytes = reinterpret_cast<const uint8_t*>(cache);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -161,6 +193,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     mbar_init(&bars->mma_drain, 1);
     mbar_init(&bars->pv_drain, 1);
     mbar_init(&bars->never, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->widened[s], kWidenThreads);
+      mbar_init(&bars->wsync[s], kWidenThreads);
+    }
     bars->abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -169,7 +205,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) tma_prefetch_desc(&tm_c);
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&tm_c);
+    if (kFp8) tma_prefetch_desc(&tm_codes);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -193,7 +232,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
           if (r < 0) return;
           const int64_t rows = pm.table ? int64_t(kTileKeys)
                                         : min(int64_t(kTileKeys), cap - t * kTileKeys);
-          bulk_prefetch_l2(cache + r * R, uint32_t(rows * R * 2));
+          bulk_prefetch_l2(cache_bytes + r * kRowBytes, uint32_t(rows * kRowBytes));
         };
         for (int64_t t = lo; t < hi; ++t, ++i) {
           const int s = i % kStages;
@@ -212,8 +251,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
           mbar_arrive_expect_tx(&bars->full[s], kLoadBytes);
           const int32_t crow = int32_t(r);
           uint8_t* dst = sStage + s * kStageBytes;
-          for (int c = 0; c < kLoadChunks; ++c)
-            tma_load_2d(&tm_c, &bars->full[s], dst + c * kChunkBytes, c * kChunkElems, crow);
+          if (kFp8) {
+            // Codes: 4 boxes [64 rows x 128 bytes] into chunks 4-7 (128-byte
+            // swizzle); RoPE keys: bf16 columns 256..319 of the row into chunk 8.
+            for (int c = 0; c < 4; ++c)
+              tma_load_2d(&tm_codes, &bars->full[s], dst + (4 + c) * kChunkBytes, c * 128, crow);
+            tma_load_2d(&tm_c, &bars->full[s], dst + kRopeChunk * kChunkBytes, 256, crow);
+          } else {
+            for (int c = 0; c < kLoadChunks; ++c)
+              tma_load_2d(&tm_c, &bars->full[s], dst + c * kChunkBytes, c * kChunkElems, crow);
+          }
           // Loads of the first tiles go out before any prefetch.
           if (t == lo)
             for (int64_t u = t + kStages; u < t + kPrefetchTiles; ++u) prefetch(u);
@@ -239,7 +286,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
       if (!(ok = warp_wait(&bars->q_ready, seg & 1, abort_flag))) return false;
       for (int64_t t = lo; t < hi; ++t, ++i) {
         const int st = i % kStages, sb = i & 1;
-        if (!(ok = warp_wait(&bars->full[st], (i / kStages) & 1, abort_flag))) return false;
+        // The stage holds bf16 rows (for the FP8 cache: once widened).
+        if (!(ok = warp_wait(kFp8 ? &bars->widened[st] : &bars->full[st], (i / kStages) & 1,
+                             abort_flag)))
+          return false;
         if (i >= 2 && !(ok = warp_wait(&bars->s_free[sb], ((i >> 1) - 1) & 1, abort_flag)))
           return false;
         tc_fence_after();
@@ -304,6 +354,78 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     mma_commit_w(&bars->pv_drain);
     volatile int no_abort = 0;
     warp_wait(&bars->pv_drain, 0, &no_abort);
+  } else if (kFp8 && warp >= kWidenWarp0) {
+    // ------------------------------------------------------------ widen (FP8 cache)
+    // Thread (r, hh) expands row r of code boxes hh and 2 + hh: box c holds
+    // latent columns [128c, 128c + 128), i.e. bf16 chunks 2c and 2c + 1.
+    // Boxes 0-1 (chunks 4-5) are widened into chunks 0-3; boxes 2-3 are read
+    // into registers, every widen thread meets at `wsync` (so chunks 4-7 have
+    // been read by all), then written into chunks 4-7.
+    const int wt = threadIdx.x - 32 * kWidenWarp0;
+    const int r = wt >> 1, hh = wt & 1;
+    uint32_t i = 0;
+    bool ok = true;
+    auto store_units = [&](uint8_t* stage, int box, int v, uint4 lo, uint4 hi_) {
+      // 16 codes -> dims [128 box + 16 v, +16): bf16 units 2(v%4), 2(v%4)+1 of
+      // chunk 2 box + v / 4, 128-byte swizzled.
+      uint8_t* chunk = stage + (2 * box + v / 4) * kChunkBytes + r * 128;
+      const int u0 = 2 * (v % 4);
+      *reinterpret_cast<uint4*>(chunk + ((u0 ^ (r & 7)) * 16)) = lo;
+      *reinterpret_cast<uint4*>(chunk + (((u0 + 1) ^ (r & 7)) * 16)) = hi_;
+    };
+    // The row's scale for tile t of sequence b; rows past the capacity get 0
+    // (their keys are masked and their rows zeroed before P.C).
+    auto load_scale = [&](int b, int64_t t) {
+      if (b < 0) return 0.f;
+      const int64_t key = t * kTileKeys + r;
+      const int64_t prow = key < cap ? pm.row(b, key) : -1;
+      return prow >= 0 ? scales[prow] : 0.f;
+    };
+    // Scales are read one tile ahead of their use (a global load per row
+    // would otherwise put its latency on every tile).
+    float next_scale = 0.f;
+    {
+      const int b0 = tp.next_sequence(-1, t_begin, t_end);
+      if (b0 >= 0) next_scale = load_scale(b0, max(tp.at(b0), t_begin) - tp.at(b0));
+    }
+    for_each_segment(tp, t_begin, t_end, [&](int b, int64_t lo, int64_t hi, int64_t) {
+      for (int64_t t = lo; t < hi; ++t, ++i) {
+        const int s = i % kStages;
+        const float scale = next_scale;
+        // The next tile is t + 1 of this sequence, or tile 0 of the next
+        // sequence of the range (a range enters later sequences at tile 0).
+        if (t + 1 < hi) next_scale = load_scale(b, t + 1);
+        else next_scale = load_scale(tp.next_sequence(b, t_begin, t_end), 0);
+        if (!(ok = warp_wait(&bars->full[s], (i / kStages) & 1, abort_flag))) return false;
+        uint8_t* stage = sStage + s * kStageBytes;
+        // Code boxes arrive 128-byte swizzled like the bf16 chunks: unit v
+        // (16 codes) of row r sits at 16 (v ^ (r % 8)), so the rows a warp
+        // reads together fall in different banks.
+        auto code_unit = [&](int box, int v) {
+          return *reinterpret_cast<const uint4*>(stage + (4 + box) * kChunkBytes + r * 128 +
+                                                 ((v ^ (r & 7)) * 16));
+        };
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const uint4 c = code_unit(hh, v);
+          store_units(stage, hh, v, widen_e4m3x8(make_uint2(c.x, c.y), scale),
+                      widen_e4m3x8(make_uint2(c.z, c.w), scale));
+        }
+        uint4 c2[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) c2[v] = code_unit(2 + hh, v);
+        mbar_arrive(&bars->wsync[s]);
+        if (!(ok = warp_wait(&bars->wsync[s], (i / kStages) & 1, abort_flag))) return false;
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          store_units(stage, 2 + hh, v, widen_e4m3x8(make_uint2(c2[v].x, c2[v].y), scale),
+                      widen_e4m3x8(make_uint2(c2[v].z, c2[v].w), scale));
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->widened[s]);
+      }
+      return true;
+    });
+    if (!ok && lane == 0) raise_abort(bars, status);
   } else {
     // ------------------------------------------------------------ softmax
     const int q = warp;                      // TMEM lane quadrant
@@ -325,18 +447,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __nv_bfloat16* 
     // loads of a thread are issued before the first store (one round trip).
     auto write_query = [&](int b) {
       constexpr int kUnits = R / 16;   // 16-byte units per half-warp thread: 36, or 32 without RoPE
+      // All loads in one round trip; in three with the FP8 widen warps
+      // sharing the register file.
+      constexpr int kBatch = kFp8 ? 12 : kUnits;
       const int64_t qrow = int64_t(b) * H + int64_t(g) * kHeadsPerCta + row;
       const bool valid_row = qrow < int64_t(B) * H;
       const uint4* src = reinterpret_cast<const uint4*>(q_cat + (valid_row ? qrow : 0) * R);
-      uint4 v[kUnits];
 #pragma unroll
-      for (int j = 0; j < kUnits; ++j) v[j] = src[2 * j + (lo_half ? 0 : 1)];
-      if (!valid_row) {
+      for (int j0 = 0; j0 < kUnits; j0 += kBatch) {
+        uint4 v[kBatch];
 #pragma unroll
-        for (int j = 0; j < kUnits; ++j) v[j] = make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < kBatch; ++j)
+          v[j] = (valid_row && j0 + j < kUnits) ? src[2 * (j0 + j) + (lo_half ? 0 : 1)]
+                                                : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+          if (j0 + j < kUnits) tmem_st16x2_4<4>(lo_base + kColQ + uint32_t(8 * (j0 + j)), v[j]);
       }
-#pragma unroll
-      for (int j = 0; j < kUnits; ++j) tmem_st16x2_4<4>(lo_base + kColQ + uint32_t(8 * j), v[j]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->q_ready);
@@ -541,17 +668,17 @@ bool make_cache_rows_map_r(CUtensorMap* map, const void* base, uint64_t rows, in
 int decode_tc_head_groups(int H) { return (H + kHeadsPerCta - 1) / kHeadsPerCta; }
 
 namespace {
-template <int kDr>
-cudaError_t launch_decode_tc_t(const CUtensorMap& tm_c, const __nv_bfloat16* q_cat,
-                               const __nv_bfloat16* cache, const PageMap& pm,
-                               const int32_t* seqlens, int B, int H, int64_t cap, float scale,
-                               int W, float* o_part, float* lse_part, int* status,
+template <int kDr, bool kFp8>
+cudaError_t launch_decode_tc_t(const CUtensorMap& tm_c, const CUtensorMap& tm_codes,
+                               const __nv_bfloat16* q_cat, const void* cache, const float* scales,
+                               const PageMap& pm, const int32_t* seqlens, int B, int H, int64_t cap,
+                               float scale, int W, float* o_part, float* lse_part, int* status,
                                uint64_t inject_wait, cudaStream_t stream) {
   static bool attr_done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<kDr>,
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<kDr, kFp8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(kSmemBytes));
     if (e != cudaSuccess) return e;
@@ -559,10 +686,24 @@ cudaError_t launch_decode_tc_t(const CUtensorMap& tm_c, const __nv_bfloat16* q_c
   }
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(decode_tc_head_groups(H), W);
-  decode_tc_kernel<kDr><<<grid, kThreads, kSmemBytes, stream>>>(
-      tm_c, cache, pm, q_cat, seqlens, B, H, cap, scale_log2, W, o_part, lse_part, status,
-      inject_wait);
+  decode_tc_kernel<kDr, kFp8><<<grid, Threads<kFp8>::n, kSmemBytes, stream>>>(
+      tm_c, tm_codes, static_cast<const __nv_bfloat16*>(cache), scales, pm, q_cat, seqlens, B, H,
+      cap, scale_log2, W, o_part, lse_part, status, inject_wait);
   return cudaGetLastError();
+}
+
+// Byte map over FP8 cache rows [rows, 640]: boxes of 128 codes x 64 rows,
+// 128-byte swizzled.
+bool make_code_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(kFp8RowBytes), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(kFp8RowBytes)};
+  const cuuint32_t box[2] = {128, cuuint32_t(kTileKeys)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 }  // namespace
 
@@ -576,10 +717,29 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
   CUtensorMap tm_c;
   if (!make_cache_rows_map_r(&tm_c, cache, uint64_t(pm.total_rows(B)), kDc + d_r))
     return cudaErrorInvalidValue;
-  return d_r == 64 ? launch_decode_tc_t<64>(tm_c, q_cat, cache, pm, seqlens, B, H, cap, scale, W,
-                                            o_part, lse_part, status, inject_wait, stream)
-                   : launch_decode_tc_t<0>(tm_c, q_cat, cache, pm, seqlens, B, H, cap, scale, W,
-                                           o_part, lse_part, status, inject_wait, stream);
+  return d_r == 64 ? launch_decode_tc_t<64, false>(tm_c, tm_c, q_cat, cache, nullptr, pm, seqlens,
+                                                   B, H, cap, scale, W, o_part, lse_part, status,
+                                                   inject_wait, stream)
+                   : launch_decode_tc_t<0, false>(tm_c, tm_c, q_cat, cache, nullptr, pm, seqlens,
+                                                  B, H, cap, scale, W, o_part, lse_part, status,
+                                                  inject_wait, stream);
+}
+
+cudaError_t launch_decode_tc_fp8(const __nv_bfloat16* q_cat, const uint8_t* cache,
+                                 const float* scales, const PageMap& pm, const int32_t* seqlens,
+                                 int B, int H, int64_t cap, float scale, int W, float* o_part,
+                                 float* lse_part, int* status, uint64_t inject_wait,
+                                 cudaStream_t stream) {
+  if (pm.total_rows(B) >= (int64_t(1) << 31) || int64_t(B) * H >= (int64_t(1) << 31))
+    return cudaErrorInvalidValue;
+  // The same rows viewed as bf16 [rows, 320] for the RoPE keys (columns 256..319).
+  CUtensorMap tm_rope, tm_codes;
+  if (!make_cache_rows_map_r(&tm_rope, cache, uint64_t(pm.total_rows(B)), kFp8RowBytes / 2) ||
+      !make_code_rows_map(&tm_codes, cache, uint64_t(pm.total_rows(B))))
+    return cudaErrorInvalidValue;
+  return launch_decode_tc_t<64, true>(tm_rope, tm_codes, q_cat, cache, scales, pm, seqlens, B, H,
+                                      cap, scale, W, o_part, lse_part, status, inject_wait,
+                                      stream);
 }
 
 }  // namespace mla

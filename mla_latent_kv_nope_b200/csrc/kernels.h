@@ -33,6 +33,14 @@ cudaError_t launch_decode_tc(const __nv_bfloat16* q_cat, const __nv_bfloat16* ca
                              int d_r, float scale, int W, float* o_part, float* lse_part,
                              int* status, uint64_t inject_wait, cudaStream_t stream);
 int decode_tc_head_groups(int H);
+// The same over an FP8 latent cache: rows [512 E4M3 codes || 64 bf16 RoPE keys]
+// (640 bytes) addressed through `pm`, and one fp32 scale per row (`scales`,
+// indexed like the rows).
+cudaError_t launch_decode_tc_fp8(const __nv_bfloat16* q_cat, const uint8_t* cache,
+                                 const float* scales, const PageMap& pm, const int32_t* seqlens,
+                                 int B, int H, int64_t cap, float scale, int W, float* o_part,
+                                 float* lse_part, int* status, uint64_t inject_wait,
+                                 cudaStream_t stream);
 // 2D TMA map over the cache viewed as [rows, 576] bf16: 64 x 64 boxes, 128-byte
 // swizzle.  False if the driver entry point is missing or encoding fails.
 bool make_cache_rows_map(CUtensorMap* map, const void* base, uint64_t rows);
@@ -65,6 +73,14 @@ cudaError_t launch_append_finalize(const float* part, int n_parts, const float* 
                                    float rope_base, int B, int d_c, int d_r, int64_t cap,
                                    T* cache, const PageMap& pm, int32_t* seqlens, int* status,
                                    cudaStream_t stream);
+
+// Finalize into an FP8 latent cache: rows of [d_c E4M3 codes || d_r bf16 RoPE
+// keys] (d_c + 2 d_r bytes) and one fp32 power-of-two scale per row.
+cudaError_t launch_append_finalize_fp8(const float* part, int n_parts, const float* gamma,
+                                       float eps, float rope_base, int B, int d_c, int d_r,
+                                       int64_t cap, uint8_t* cache, float* scales,
+                                       const PageMap& pm, int32_t* seqlens, int* status,
+                                       cudaStream_t stream);
 
 // Tensor-core kernels for the bf16 step (d_c = 512, d_r = 64 or 0, d_nope = d_v = 128).
 bool gemm_tc_supported(int d_c, int d_r, int d_n, int d_v);

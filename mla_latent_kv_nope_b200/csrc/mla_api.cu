@@ -340,6 +340,74 @@ int mla_decode_paged(const mla_dims* d, const void* q_cat, const void* cache_poo
 }
 
 // ---------------------------------------------------------------------------
+// FP8 latent cache: rows [d_c E4M3 codes || d_r bf16 RoPE keys] plus one fp32
+// power-of-two scale per row (shape 512 / 64, bf16 weights and queries).
+namespace {
+bool fp8_shape(const mla_dims* d) {
+  return d->dtype == MLA_BF16 && gemm_tc_supported(d->d_c, d->d_r, d->d_nope, d->d_v) &&
+         d->d_r == 64;
+}
+}  // namespace
+
+int64_t mla_cache_fp8_row_bytes(int32_t d_c, int32_t d_r) {
+  return int64_t(d_c) + 2 * int64_t(d_r);
+}
+
+int mla_cache_append_fp8(const mla_dims* d, int32_t hidden, const void* h, const void* W_DKV,
+                         const float* gamma, float eps, float rope_base, void* cache,
+                         float* scales, int32_t* seqlens, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if (!fp8_shape(d)) return MLA_ERR_UNSUPPORTED;
+  if (hidden <= 0 || !h || !W_DKV || !cache || !scales || !seqlens) return MLA_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !(rope_base > 0.f)) return MLA_ERR_INVALID_ARG;
+  if (hidden % 8) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(h) || !aligned16(W_DKV) || !aligned16(cache) || !aligned16(scales) ||
+      !aligned16(seqlens) || (gamma && !aligned16(gamma)) || (workspace && !aligned16(workspace)))
+    return MLA_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < mla_cache_append_workspace_bytes(d, hidden))
+    return MLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* x = static_cast<float*>(workspace);
+  cudaError_t e = launch_append_proj_tc(static_cast<const __nv_bfloat16*>(h),
+                                        static_cast<const __nv_bfloat16*>(W_DKV), d->B,
+                                        d->d_c + d->d_r, hidden, x, status_ptr(), s);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  return cuda_status(launch_append_finalize_fp8(
+      x, append_tc_splits(hidden), gamma, eps, rope_base, d->B, d->d_c, d->d_r,
+      d->cache_capacity, static_cast<uint8_t*>(cache), scales, contiguous_map(d), seqlens,
+      status_ptr(), s));
+}
+
+int mla_decode_fp8(const mla_dims* d, const void* q_cat, const void* cache, const float* scales,
+                   const int32_t* seqlens, float softmax_scale, int num_splits, void* workspace,
+                   size_t workspace_bytes, int* splits_used, void* stream) {
+  int st = check_dims(d);
+  if (st) return st;
+  if (!fp8_shape(d)) return MLA_ERR_UNSUPPORTED;
+  if (int64_t(d->B) * d->cache_capacity >= (int64_t(1) << 31)) return MLA_ERR_UNSUPPORTED;
+  if (!q_cat || !cache || !scales || !seqlens || num_splits < 0 || num_splits > kMaxSplits ||
+      !(softmax_scale >= 0.f) || softmax_scale == INFINITY)
+    return MLA_ERR_INVALID_ARG;
+  softmax_scale = effective_scale(d, softmax_scale);
+  if (!aligned16(q_cat) || !aligned16(cache) || !aligned16(scales) || !aligned16(seqlens) ||
+      (workspace && !aligned16(workspace)))
+    return MLA_ERR_ALIGNMENT;
+  const int W = num_splits > 0 ? num_splits : mla_decode_default_splits(d);
+  if (W <= 0) return MLA_ERR_CUDA;
+  const WsLayout l = ws_layout(d, W);
+  if (!workspace || workspace_bytes < l.total) return MLA_ERR_WORKSPACE;
+  if (splits_used) *splits_used = W;
+  float* o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + l.o_off);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + l.lse_off);
+  return cuda_status(launch_decode_tc_fp8(
+      static_cast<const __nv_bfloat16*>(q_cat), static_cast<const uint8_t*>(cache), scales,
+      contiguous_map(d), seqlens, d->B, d->H, d->cache_capacity, softmax_scale, W, o_part,
+      lse_part, status_ptr(), g_inject_wait_cycles, static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------------------
 int mla_combine(const mla_dims* d, const int32_t* seqlens, const void* workspace,
                 size_t workspace_bytes, int splits_used, float* o_lat, float* lse, void* stream) {
   int st = check_dims(d);

@@ -20,7 +20,8 @@ import numpy as np
 
 # Tensor ids for the per-tensor streams.
 TID = {"q_nope": 1, "q_pe": 2, "W_UK": 3, "W_UV": 4, "cache": 5, "seqlens": 6,
-       "h": 7, "W_DKV": 8, "gamma": 9, "partials_o": 10, "partials_lse": 11}
+       "h": 7, "W_DKV": 8, "gamma": 9, "partials_o": 10, "partials_lse": 11,
+       "fp8_codes": 12, "fp8_scale": 13, "fp8_rope": 14}
 
 
 @dataclass(frozen=True)
@@ -129,6 +130,41 @@ def fill_cache(w: Workload, cache, lens, fill_rest: float | None = None):
         if fill_rest is not None and L < cache.shape[1]:
             cache[b, L:].fill_(fill_rest)
     return cache
+
+
+def fp8_cache_rows(w: Workload, b: int, n: int):
+    """The first n rows of sequence b of an FP8 latent cache, drawn directly
+    in the stored format: (codes [n, d_c] uint8, uniform over the 254 finite
+    E4M3 bytes, i.e. every byte but 0x7F and 0xFF; exponents k [n] int,
+    uniform in [-9, -6], the token's scale being 2^k; RoPE keys [n, d_r]
+    float32 N(0, 1))."""
+    r = _rng(w.seed, TID["fp8_codes"], b)
+    draw = r.integers(0, 254, size=(n, w.d_c))
+    codes = np.where(draw >= 0x7F, draw + 1, draw).astype(np.uint8)
+    k = _rng(w.seed, TID["fp8_scale"], b).integers(-9, -5, size=n)
+    rope = normal((n, w.d_r), 1.0, w.seed, TID["fp8_rope"], b)
+    return codes, k, rope
+
+
+def fill_fp8_cache(w: Workload, cache, scales, lens, fill_rest_byte: int | None = None):
+    """Write rows [0, L_b) of every sequence into an FP8 cache: cache [B,
+    capacity, d_c + 2 d_r] uint8 (codes, then the RoPE keys' bf16 bytes) and
+    scales [B, capacity] float32 (2^k).  Rows from L_b on get
+    ``fill_rest_byte`` in every byte and scale 1 when given (0xFF is an E4M3
+    NaN code, to show that the decode never depends on them)."""
+    import torch
+    for b in range(w.B):
+        L = int(lens[b])
+        if L:
+            codes, k, rope = fp8_cache_rows(w, b, L)
+            cache[b, :L, :w.d_c].copy_(torch.from_numpy(codes))
+            rb = torch.from_numpy(rope).to(torch.bfloat16).view(torch.uint8).reshape(L, 2 * w.d_r)
+            cache[b, :L, w.d_c:].copy_(rb)
+            scales[b, :L].copy_(torch.from_numpy(np.ldexp(np.ones(L, np.float32), k)))
+        if fill_rest_byte is not None and L < cache.shape[1]:
+            cache[b, L:].fill_(fill_rest_byte)
+            scales[b, L:].fill_(1.0)
+    return cache, scales
 
 
 def partials(B: int, H: int, S: int, D: int, seed: int = 0, empty_frac: float = 0.2):
