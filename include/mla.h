@@ -182,6 +182,31 @@ MLA_API int mla_merge_partials(const mla_dims* dims, int n_parts, const float* o
 MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W_UV,
                  void* out, void* stream);
 
+/* --- W^O folded into the value side ---------------------------------------------
+ * [MLA-とは] "Value側の吸収": W^UV_i can be absorbed into the output
+ * projection, B_i = W^O_i W^UV_i in R^{d x d_c}, so the latent-space weighted
+ * sums o_lat go straight to the model width:
+ *   u[b] = sum_i B_i o_lat[b,i]   (= sum_i W^O_i W^UV_i o_lat[b,i])
+ * W_O [d_model, H * d_v] bf16 (column convention: u = W^O o over the heads'
+ * concatenated d_v-wide outputs); W_UV [H, d_v, d_c] bf16 as in mla_out_proj.
+ * mla_fold_output_weights writes W_fold [d_model, H * d_c] bf16 with
+ * W_fold[m, i*d_c + c] = (B_i)[m, c] (fp32 accumulation, rounded once); it
+ * runs once, when the weights are loaded.  mla_out_proj_folded reads o_lat
+ * [B, H, d_c] fp32 (rounded to bf16 for the tensor cores, as in
+ * mla_out_proj) and writes u [B, d_model] bf16, using
+ * mla_out_proj_folded_workspace_bytes(dims, d_model) bytes of scratch (no
+ * initialisation needed).  Shape: bf16, d_c = 512, d_v = 128; the folded
+ * projection needs B <= 64 (MLA_ERR_UNSUPPORTED otherwise).  Per step the
+ * folded weight is H * d * d_c bf16 against H * d_v * (d_c + d) for W^UV and
+ * W^O: more bytes whenever d_c > d_v, so this form pays only when those
+ * weights are not otherwise read. */
+MLA_API int mla_fold_output_weights(const mla_dims* dims, int32_t d_model, const void* W_O,
+                                    const void* W_UV, void* W_fold, void* stream);
+MLA_API size_t mla_out_proj_folded_workspace_bytes(const mla_dims* dims, int32_t d_model);
+MLA_API int mla_out_proj_folded(const mla_dims* dims, int32_t d_model, const float* o_lat,
+                                const void* W_fold, void* u, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* --- FP8 latent cache ------------------------------------------------------------
  * [abeam] "モデル全体でも推論効率が大きく改善した" names KV-cache quantisation as
  * part of the system's serving efficiency, and [yuuk] "未解決の問い" leaves FP8

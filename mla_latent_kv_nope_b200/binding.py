@@ -28,7 +28,8 @@ EXPORTED = (
     "mla_decode", "mla_combine", "mla_out_proj", "mla_get_device_status",
     "mla_status_string", "mla_decode_noalloc", "mla_decode_paged", "mla_cache_append_paged",
     "mla_merge_partials", "mla_debug_inject_wait", "mla_cache_fp8_row_bytes",
-    "mla_cache_append_fp8", "mla_decode_fp8",
+    "mla_cache_append_fp8", "mla_decode_fp8", "mla_fold_output_weights",
+    "mla_out_proj_folded_workspace_bytes", "mla_out_proj_folded",
 )
 
 PAGE_ROWS = 64   # rows per page of a paged latent cache (one decode work tile)
@@ -109,6 +110,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "mla_debug_inject_wait": (ctypes.c_int, [ctypes.c_uint64]),
         "mla_cache_fp8_row_bytes": (I64, [I32, I32]),
+        "mla_fold_output_weights": (ctypes.c_int, [D, I32, P, P, P, P]),
+        "mla_out_proj_folded_workspace_bytes": (SZ, [D, I32]),
+        "mla_out_proj_folded": (ctypes.c_int, [D, I32, P, P, P, P, SZ, P]),
         "mla_cache_append_fp8": (ctypes.c_int, [D, I32, P, P, P, F, F, P, P, P, P, SZ, P]),
         "mla_decode_fp8": (ctypes.c_int, [D, P, P, P, P, F, ctypes.c_int, P, SZ,
                                           ctypes.POINTER(ctypes.c_int), P]),
@@ -373,6 +377,36 @@ def debug_inject_wait(cycles: int) -> None:
     wait ``cycles`` SM cycles on a barrier nothing arrives on and give up
     (MLA_ERR_DEVICE_TIMEOUT in the status word); 0 turns it off."""
     _check("mla_debug_inject_wait", load_library().mla_debug_inject_wait(int(cycles)))
+
+
+def fold_output_weights(dims: Dims, W_O, W_UV, W_fold, stream=None):
+    """mla_fold_output_weights: W_fold [d_model, H*d_c] with
+    W_fold[m, i*d_c + c] = (W^O_i W^UV_i)[m, c]; W_O [d_model, H*d_v]."""
+    d_model = W_O.shape[0]
+    _need(W_O, dims.torch_dtype, (d_model, dims.H * dims.d_v), "W_O")
+    _need(W_UV, dims.torch_dtype, (dims.H, dims.d_v, dims.d_c), "W_UV")
+    _need(W_fold, dims.torch_dtype, (d_model, dims.H * dims.d_c), "W_fold")
+    st = load_library().mla_fold_output_weights(ctypes.byref(dims.c()), d_model, _ptr(W_O),
+                                                _ptr(W_UV), _ptr(W_fold), _stream(stream))
+    _check("mla_fold_output_weights", st)
+
+
+def out_proj_folded_workspace_bytes(dims: Dims, d_model: int) -> int:
+    return int(load_library().mla_out_proj_folded_workspace_bytes(ctypes.byref(dims.c()),
+                                                                  d_model))
+
+
+def out_proj_folded(dims: Dims, o_lat, W_fold, u, workspace, stream=None):
+    """mla_out_proj_folded: u [B, d_model] = sum_i B_i o_lat[:, i] (bf16)."""
+    d_model = W_fold.shape[0]
+    _need(o_lat, torch.float32, (dims.B, dims.H, dims.d_c), "o_lat")
+    _need(W_fold, dims.torch_dtype, (d_model, dims.H * dims.d_c), "W_fold")
+    _need(u, dims.torch_dtype, (dims.B, d_model), "u")
+    _need_ws(workspace)
+    st = load_library().mla_out_proj_folded(
+        ctypes.byref(dims.c()), d_model, _ptr(o_lat), _ptr(W_fold), _ptr(u), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("mla_out_proj_folded", st)
 
 
 def get_device_status(stream=None) -> int:

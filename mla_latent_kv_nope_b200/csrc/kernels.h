@@ -95,4 +95,17 @@ cudaError_t launch_append_proj_tc(const __nv_bfloat16* h, const __nv_bfloat16* W
                                   int R, int hidden, float* part, int* status,
                                   cudaStream_t stream);
 
+// W^O folded into the value side: W_fold [d_model, H * 512] (bf16) with
+// W_fold[m, i*512 + c] = sum_v W_O[m, i*128 + v] W_UV[i, v, c] (d_c = 512,
+// d_v = 128), and the per-step u [B, d_model] = W_fold o_lat (o_lat fp32
+// [B, H * 512], rounded to bf16 for the MMA; B <= kFoldedMaxBatch).
+constexpr int kFoldedMaxBatch = 64;
+cudaError_t launch_fold_weights(const __nv_bfloat16* W_O, const __nv_bfloat16* W_UV, int d_model,
+                                int H, __nv_bfloat16* w_fold, int* status, cudaStream_t stream);
+int folded_proj_splits(int d_model, int H);
+size_t folded_proj_workspace_bytes(int B, int H, int d_model);
+cudaError_t launch_folded_proj(const float* o_lat, const __nv_bfloat16* w_fold, int B, int H,
+                               int d_model, void* workspace, __nv_bfloat16* u, int* status,
+                               cudaStream_t stream);
+
 }  // namespace mla

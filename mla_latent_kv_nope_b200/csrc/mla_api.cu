@@ -408,6 +408,51 @@ int mla_decode_fp8(const mla_dims* d, const void* q_cat, const void* cache, cons
 }
 
 // ---------------------------------------------------------------------------
+// W^O folded into the value side.
+namespace {
+int check_fold(const mla_dims* d, int32_t d_model) {
+  int st = check_dims(d);
+  if (st) return st;
+  if (d->dtype != MLA_BF16 || d->d_c != 512 || d->d_v != 128) return MLA_ERR_UNSUPPORTED;
+  if (d_model <= 0) return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+}  // namespace
+
+int mla_fold_output_weights(const mla_dims* d, int32_t d_model, const void* W_O,
+                            const void* W_UV, void* W_fold, void* stream) {
+  int st = check_fold(d, d_model);
+  if (st) return st;
+  if (!W_O || !W_UV || !W_fold) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(W_O) || !aligned16(W_UV) || !aligned16(W_fold)) return MLA_ERR_ALIGNMENT;
+  return cuda_status(launch_fold_weights(static_cast<const __nv_bfloat16*>(W_O),
+                                         static_cast<const __nv_bfloat16*>(W_UV), d_model, d->H,
+                                         static_cast<__nv_bfloat16*>(W_fold), status_ptr(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_out_proj_folded_workspace_bytes(const mla_dims* d, int32_t d_model) {
+  if (check_fold(d, d_model) != MLA_OK || d->B > kFoldedMaxBatch) return 0;
+  return folded_proj_workspace_bytes(d->B, d->H, d_model);
+}
+
+int mla_out_proj_folded(const mla_dims* d, int32_t d_model, const float* o_lat, const void* W_fold,
+                        void* u, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_fold(d, d_model);
+  if (st) return st;
+  if (d->B > kFoldedMaxBatch) return MLA_ERR_UNSUPPORTED;
+  if (!o_lat || !W_fold || !u) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(o_lat) || !aligned16(W_fold) || !aligned16(u) ||
+      (workspace && !aligned16(workspace)))
+    return MLA_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < folded_proj_workspace_bytes(d->B, d->H, d_model))
+    return MLA_ERR_WORKSPACE;
+  return cuda_status(launch_folded_proj(o_lat, static_cast<const __nv_bfloat16*>(W_fold), d->B,
+                                        d->H, d_model, workspace, static_cast<__nv_bfloat16*>(u),
+                                        status_ptr(), static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------------------
 int mla_combine(const mla_dims* d, const int32_t* seqlens, const void* workspace,
                 size_t workspace_bytes, int splits_used, float* o_lat, float* lse, void* stream) {
   int st = check_dims(d);
