@@ -45,7 +45,7 @@ def _peaks():
 
 def _decode_source_hash():
     h = hashlib.sha256()
-    for name in ("k_decode_tc.cu", "k_decode_pair.cu", "tile_deal.cuh", "common.cuh"):
+    for name in ("k_decode_tc.cu", "tile_deal.cuh", "common.cuh", "sm100.cuh"):
         with open(os.path.join(ROOT, "mla_latent_kv_nope_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -596,6 +596,85 @@ def run_reference(args, rank, world):
     }
 
 
+def run_folded_out_proj(args, rank, world, local_rank):
+    """The W^O fold variant alone ([MLA-とは] "Value側の吸収"): u = sum_i B_i
+    o_lat_i with B_i = W^O_i W^UV_i folded once, d_model = the workload's
+    hidden width.  One launch set per step (bf16 rounding of o_lat, the
+    weight-streaming tcgen05 kernel, the split reduction); the folded weight
+    (H d_model d_c bf16) exceeds L2, so no flush is needed.  Each rank times
+    its own copy (no collective)."""
+    import torch
+
+    import mla_latent_kv_nope_b200 as mla
+    from mla_latent_kv_nope_b200 import dist as mdist
+    from mla_latent_kv_nope_b200 import inputs
+    from mla_latent_kv_nope_b200.build import build
+
+    if rank == 0:
+        build()
+    if world > 1:
+        mdist.barrier(world)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = inputs.WORKLOADS[args.workload]
+    d_model = w.hidden
+    dims = mla.Dims(w.B, w.H, w.d_c, w.d_r, w.d_nope, w.d_v, w.capacity, w.dtype)
+    _, Wuv = inputs.weights(w)
+    W_UV = torch.from_numpy(Wuv).to(dev, torch.bfloat16)
+    W_O = torch.from_numpy(inputs.normal((d_model, w.H * w.d_v), w.w_std, w.seed, 41,
+                                         d_model)).to(dev, torch.bfloat16)
+    o_lat = torch.from_numpy(inputs.normal((w.B, w.H, w.d_c), 0.05, w.seed, 123, 1)).to(dev)
+    W_fold = torch.empty(d_model, w.H * w.d_c, dtype=torch.bfloat16, device=dev)
+    mla.fold_output_weights(dims, W_O, W_UV, W_fold)
+    del W_O
+    u = torch.empty(w.B, d_model, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(mla.out_proj_folded_workspace_bytes(dims, d_model), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        mla.out_proj_folded(dims, o_lat, W_fold, u, ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        mdist.barrier(world)
+        torch.cuda.synchronize()
+        clk.start()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            mla.out_proj_folded(dims, o_lat, W_fold, u, ws)
+        t1.record(stream)
+        clk.poll_until(t1.query)
+        torch.cuda.synchronize()
+        clk.stop()
+        mdist.barrier(world)
+    ms = mdist.max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    if mla.get_device_status() != 0:
+        raise RuntimeError("device status error during timing")
+    if rank != 0:
+        return None
+    hbm, _, _, peak_src = _peaks()
+    byts = w.H * d_model * w.d_c * 2 + w.B * w.H * w.d_c * 4 + w.B * d_model * 2
+    unfolded = w.H * w.d_v * w.d_c * 2 + d_model * w.H * w.d_v * 2
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {
+        "metric": "folded output projection weight-stream GB/s", "value": gbs, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded)",
+        "config": {"workload": f"folded out-proj B={w.B} H={w.H} d_c={w.d_c} d_v={w.d_v} "
+                               f"d_model={d_model}", "l2": "folded weight exceeds L2"},
+        "roofline": {"kernel": "folded_proj_tc_kernel + to_bf16 + split reduction",
+                     "bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "traffic": None, "algorithmic_bytes_per_launch": byts,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
+                                    if peak_src == "measured" else "fallback"},
+        # The unfolded form reads W^UV and W^O instead of the folded weight.
+        "unfolded_weight_bytes": unfolded, "folded_weight_bytes": w.H * d_model * w.d_c * 2,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+
 def _relaunch_per_gpu(n):
     """`--gpus N` (N > 1) started without a launcher: run this same command as
     N ranks, one process per GPU, under torch.distributed.run (rendezvous on
@@ -663,6 +742,9 @@ def main():
                     help="keep the latent cache in shuffled 64-row pages behind a block table")
     ap.add_argument("--eager", action="store_true",
                     help="launch each kernel from the host every step instead of a CUDA graph")
+    ap.add_argument("--kernel", default="step", choices=["step", "folded_out_proj"],
+                    help="step: the whole decode step (default); folded_out_proj: the W^O "
+                         "fold variant of the output projection alone")
     ap.add_argument("--dry-run", action="store_true",
                     help="host-only check of the multi-rank launch and timing (gloo, no GPU)")
     args = ap.parse_args()
@@ -693,7 +775,10 @@ def main():
             torch.cuda.set_device(local_rank)
             dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                     device_id=torch.device("cuda", local_rank))
-        res = run_ours(args, rank, world, local_rank)
+        if args.kernel == "folded_out_proj":
+            res = run_folded_out_proj(args, rank, world, local_rank)
+        else:
+            res = run_ours(args, rank, world, local_rank)
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()

@@ -135,7 +135,7 @@ __global__ void to_bf16_kernel(const float4* __restrict__ x, uint2* __restrict__
 
 // ---------------------------------------------------------------------------
 // Folded projection: stage = A [128 x 128 B] (16 KB) + X [Np x 128 B].
-constexpr int kFpStages = 6;
+constexpr int kFpStages = 4;   // 4 x 24 KB: two CTAs fit on an SM
 
 __host__ __device__ constexpr size_t fp_stage_bytes(int np) { return 16384 + size_t(np) * 128; }
 
@@ -338,7 +338,7 @@ cudaError_t launch_fold_weights(const __nv_bfloat16* W_O, const __nv_bfloat16* W
 int folded_proj_splits(int d_model, int H) {
   const int m_tiles = (d_model + 127) / 128;
   const int64_t k_chunks = int64_t(H) * 512 / 64;
-  int s = (2 * sms() + m_tiles - 1) / m_tiles;    // about two CTAs per SM
+  int s = 2 * sms() / m_tiles;   // one wave of two CTAs per SM
   if (s < 1) s = 1;
   if (s > k_chunks) s = int(k_chunks);
   return s;
