@@ -196,10 +196,10 @@ MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W
  * mla_out_proj) and writes u [B, d_model] bf16, using
  * mla_out_proj_folded_workspace_bytes(dims, d_model) bytes of scratch (no
  * initialisation needed).  Shape: bf16, d_c = 512, d_v = 128; the folded
- * projection needs B <= 64 (MLA_ERR_UNSUPPORTED otherwise).  Per step the
+ * projection needs B <= 64 (MLA_ERR_UNSUPPORTED otherwise).  Per call the
  * folded weight is H * d * d_c bf16 against H * d_v * (d_c + d) for W^UV and
- * W^O: more bytes whenever d_c > d_v, so this form pays only when those
- * weights are not otherwise read. */
+ * W^O unfolded: fewer bytes only when d * (d_c - d_v) < d_v * d_c (d < 171 at
+ * d_c = 512, d_v = 128). */
 MLA_API int mla_fold_output_weights(const mla_dims* dims, int32_t d_model, const void* W_O,
                                     const void* W_UV, void* W_fold, void* stream);
 MLA_API size_t mla_out_proj_folded_workspace_bytes(const mla_dims* dims, int32_t d_model);
