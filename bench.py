@@ -675,6 +675,99 @@ def run_folded_out_proj(args, rank, world, local_rank):
     }
 
 
+def run_prefill(args, rank, world, local_rank):
+    """The materialised prefill alone ([MLA-とは] "実装上のトレードオフ"): one
+    sequence of T = L prompt tokens whose latent rows are already cached, at
+    the workload's head shape; query t at position t.  A step is one
+    mla_prefill call (query rotation, the K^C/V up-projection GEMM, causal
+    attention).  Each rank times its own sequence (no collective)."""
+    import numpy as np
+    import torch
+
+    import mla_latent_kv_nope_b200 as mla
+    from mla_latent_kv_nope_b200 import dist as mdist
+    from mla_latent_kv_nope_b200 import inputs
+    from mla_latent_kv_nope_b200.build import build
+
+    if rank == 0:
+        build()
+    if world > 1:
+        mdist.barrier(world)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    base = inputs.WORKLOADS[args.workload]
+    T = L = args.prefill_tokens
+    w = base.scaled(B=1, N=L, seed=base.seed + rank)
+    dims = mla.Dims(1, w.H, w.d_c, w.d_r, w.d_nope, w.d_v, 1, w.dtype)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev, torch.bfloat16)  # noqa: E731
+    q_nope = bf(inputs.normal((T, w.H, w.d_nope), 1.0, w.seed, 61, T))
+    q_pe = bf(inputs.normal((T, w.H, w.d_r), 1.0, w.seed, 62, T))
+    Wuk, Wuv = inputs.weights(w)
+    W_UK, W_UV = bf(Wuk), bf(Wuv)
+    rows = bf(inputs.cache_rows(w, 0, L))
+    q_pos = torch.arange(T, dtype=torch.int32, device=dev)
+    out = torch.empty(T, w.H, w.d_v, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(T, w.H, dtype=torch.float32, device=dev)
+    ws = torch.empty(mla.prefill_workspace_bytes(dims, T, L), dtype=torch.uint8, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        mla.prefill(dims, q_nope, q_pe, q_pos, W_UK, W_UV, rows, out, ws, lse=lse)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    evs = []
+    with ClockSampler(local_rank) as clk:
+        mdist.barrier(world)
+        torch.cuda.synchronize()
+        clk.start()
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            evs.append((e0, e1))
+        clk.poll_until(evs[-1][1].query)
+        torch.cuda.synchronize()
+        clk.stop()
+        mdist.barrier(world)
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    ms = mdist.max_over_ranks(ms, world, dev)
+    if mla.get_device_status() != 0:
+        raise RuntimeError("device status error during timing")
+    if rank != 0:
+        return None
+    _, tf_burst, tf_sus, peak_src = _peaks()
+    pairs = T * (T + 1) // 2                          # causal (query, row) pairs
+    flops_attn = 2.0 * pairs * w.H * (w.d_nope + w.d_r + w.d_v)
+    flops_kv = 2.0 * L * w.d_c * w.H * (w.d_nope + w.d_v)
+    flops = flops_attn + flops_kv
+    tf = flops / (ms * 1e-3) / 1e12
+    tokens_s = T * world / (ms * 1e-3)
+    return {
+        "metric": "MLA materialised prefill tokens/s and TFLOP/s", "value": tokens_s,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": f"prefill T=L={T} H={w.H} d_c={w.d_c} d_r={w.d_r} "
+                               f"d_nope={w.d_nope} d_v={w.d_v}, causal, q_pos = 0..T-1",
+                   "l2": "L2 flushed between calls"},
+        "roofline": {"kernel": "mla_prefill (q rotation + K/V up-projection + causal attention)",
+                     "bound": "tensor", "achieved": tf, "peak": tf_burst, "unit": "TFLOP/s",
+                     "frac": tf / tf_burst, "frac_sustained": tf / tf_sus, "traffic": None,
+                     "algorithmic_flops_per_launch": flops, "attention_flops": flops_attn,
+                     "kv_projection_flops": flops_kv,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst)"
+                                    if peak_src == "measured" else "fallback"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+
 def _relaunch_per_gpu(n):
     """`--gpus N` (N > 1) started without a launcher: run this same command as
     N ranks, one process per GPU, under torch.distributed.run (rendezvous on
@@ -742,9 +835,12 @@ def main():
                     help="keep the latent cache in shuffled 64-row pages behind a block table")
     ap.add_argument("--eager", action="store_true",
                     help="launch each kernel from the host every step instead of a CUDA graph")
-    ap.add_argument("--kernel", default="step", choices=["step", "folded_out_proj"],
+    ap.add_argument("--kernel", default="step", choices=["step", "folded_out_proj", "prefill"],
                     help="step: the whole decode step (default); folded_out_proj: the W^O "
-                         "fold variant of the output projection alone")
+                         "fold variant of the output projection alone; prefill: the "
+                         "materialised prefill of one sequence")
+    ap.add_argument("--prefill-tokens", type=int, default=4096,
+                    help="prompt length T = L of --kernel prefill")
     ap.add_argument("--dry-run", action="store_true",
                     help="host-only check of the multi-rank launch and timing (gloo, no GPU)")
     args = ap.parse_args()
@@ -777,6 +873,8 @@ def main():
                                     device_id=torch.device("cuda", local_rank))
         if args.kernel == "folded_out_proj":
             res = run_folded_out_proj(args, rank, world, local_rank)
+        elif args.kernel == "prefill":
+            res = run_prefill(args, rank, world, local_rank)
         else:
             res = run_ours(args, rank, world, local_rank)
         if world > 1:

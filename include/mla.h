@@ -182,6 +182,35 @@ MLA_API int mla_merge_partials(const mla_dims* dims, int n_parts, const float* o
 MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W_UV,
                  void* out, void* stream);
 
+/* --- materialised prefill of one sequence -----------------------------------------
+ * [MLA-とは] "実装上のトレードオフ": prefill processes many query tokens at
+ * once and is compute-bound, so the per-head keys and values are formed
+ * explicitly (k^C_i = W^UK_i c_l, v^C_i = W^UV_i c_l for every latent row l)
+ * and the heads run ordinary causal softmax attention with head dim
+ * d_nope + d_r (the key's RoPE part is the row's shared, already rotated k^R)
+ * and value dim d_v:
+ *   q_t,i  = [q_nope[t,i] ; RoPE(q_pe[t,i], q_pos[t])]
+ *   s_tl   = softmax_scale * (q_t,i . [W^UK_i c_l ; k^R_l]),   l <= q_pos[t]
+ *   out[t,i] = sum_l softmax(s_t)_l W^UV_i c_l,   lse[t,i] = log sum_l exp(s_tl)
+ * One sequence per call: rows [L, d_c + d_r] bf16 are its latent cache rows
+ * (the prompt's own rows already appended, e.g. by mla_cache_append, so a
+ * query attends to itself), q_nope [T, H, d_nope], q_pe [T, H, d_r] bf16,
+ * q_pos [T] int32 device positions (any order); query t sees rows
+ * 0 .. min(q_pos[t], L - 1), and nothing if q_pos[t] < 0 (out 0, lse -inf).
+ * out [T, H, d_v] bf16; lse [T, H] fp32 or NULL.  softmax_scale = 0 selects
+ * 1/sqrt(d_nope + d_r); it must be positive.  Only dims->H, d_c, d_r, d_nope,
+ * d_v and dtype are read.  Shape: bf16, d_c = 512, d_nope = d_v = 128, d_r =
+ * 64 or 0, H * L and H * T below 2^31, L >= 1 (T = 0 does nothing).  The
+ * workspace (mla_prefill_workspace_bytes, no initialisation needed) holds the
+ * rotated queries and the materialised K^C and V: about 2 * H * (T * (d_nope
+ * + d_r) + 2 * L * 128) bytes. */
+MLA_API size_t mla_prefill_workspace_bytes(const mla_dims* dims, int32_t T, int64_t L);
+MLA_API int mla_prefill(const mla_dims* dims, int32_t T, int64_t L, const void* q_nope,
+                        const void* q_pe, const int32_t* q_pos, const void* W_UK,
+                        const void* W_UV, const void* rows, float softmax_scale,
+                        float rope_base, void* out, float* lse, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
 /* --- W^O folded into the value side ---------------------------------------------
  * [MLA-とは] "Value側の吸収": W^UV_i can be absorbed into the output
  * projection, B_i = W^O_i W^UV_i in R^{d x d_c}, so the latent-space weighted

@@ -29,7 +29,8 @@ EXPORTED = (
     "mla_status_string", "mla_decode_noalloc", "mla_decode_paged", "mla_cache_append_paged",
     "mla_merge_partials", "mla_debug_inject_wait", "mla_cache_fp8_row_bytes",
     "mla_cache_append_fp8", "mla_decode_fp8", "mla_fold_output_weights",
-    "mla_out_proj_folded_workspace_bytes", "mla_out_proj_folded",
+    "mla_out_proj_folded_workspace_bytes", "mla_out_proj_folded", "mla_prefill_workspace_bytes",
+    "mla_prefill",
 )
 
 PAGE_ROWS = 64   # rows per page of a paged latent cache (one decode work tile)
@@ -111,6 +112,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_debug_inject_wait": (ctypes.c_int, [ctypes.c_uint64]),
         "mla_cache_fp8_row_bytes": (I64, [I32, I32]),
         "mla_fold_output_weights": (ctypes.c_int, [D, I32, P, P, P, P]),
+        "mla_prefill_workspace_bytes": (SZ, [D, I32, I64]),
+        "mla_prefill": (ctypes.c_int, [D, I32, I64, P, P, P, P, P, P, F, F, P, P, P, SZ, P]),
         "mla_out_proj_folded_workspace_bytes": (SZ, [D, I32]),
         "mla_out_proj_folded": (ctypes.c_int, [D, I32, P, P, P, P, SZ, P]),
         "mla_cache_append_fp8": (ctypes.c_int, [D, I32, P, P, P, F, F, P, P, P, P, SZ, P]),
@@ -377,6 +380,35 @@ def debug_inject_wait(cycles: int) -> None:
     wait ``cycles`` SM cycles on a barrier nothing arrives on and give up
     (MLA_ERR_DEVICE_TIMEOUT in the status word); 0 turns it off."""
     _check("mla_debug_inject_wait", load_library().mla_debug_inject_wait(int(cycles)))
+
+
+def prefill_workspace_bytes(dims: Dims, T: int, L: int) -> int:
+    return int(load_library().mla_prefill_workspace_bytes(ctypes.byref(dims.c()), T, L))
+
+
+def prefill(dims: Dims, q_nope, q_pe, q_pos, W_UK, W_UV, rows, out, workspace, lse=None,
+            softmax_scale: float = 0.0, rope_base: float = 10000.0, stream=None):
+    """mla_prefill: materialised causal attention of one sequence's T query
+    tokens over its L latent rows [L, d_c + d_r]; out [T, H, d_v] (+ lse [T, H])."""
+    T, L = q_nope.shape[0], rows.shape[0]
+    dt = dims.torch_dtype
+    _need(q_nope, dt, (T, dims.H, dims.d_nope), "q_nope")
+    if dims.d_r:
+        _need(q_pe, dt, (T, dims.H, dims.d_r), "q_pe")
+    _need(q_pos, torch.int32, (T,), "q_pos")
+    _need(W_UK, dt, (dims.H, dims.d_nope, dims.d_c), "W_UK")
+    _need(W_UV, dt, (dims.H, dims.d_v, dims.d_c), "W_UV")
+    _need(rows, dt, (L, dims.R), "rows")
+    _need(out, dt, (T, dims.H, dims.d_v), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (T, dims.H), "lse")
+    _need_ws(workspace)
+    st = load_library().mla_prefill(
+        ctypes.byref(dims.c()), T, L, _ptr(q_nope), _ptr(q_pe) if dims.d_r else None,
+        _ptr(q_pos), _ptr(W_UK), _ptr(W_UV), _ptr(rows), softmax_scale, rope_base, _ptr(out),
+        _ptr(lse) if lse is not None else None, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("mla_prefill", st)
 
 
 def fold_output_weights(dims: Dims, W_O, W_UV, W_fold, stream=None):

@@ -1,0 +1,606 @@
+// Materialised prefill for one sequence ([MLA-とは] "実装上のトレードオフ":
+// prefill is compute-bound, so the per-head keys and values are formed
+// explicitly and the heads run ordinary causal attention; the absorbed form is
+// the decode's).
+//
+//   prefill_q_kernel      Q_i[t] = [q^C[t,i] ; RoPE(q^R[t,i], q_pos[t])]
+//                         -> q_full [H, T, 128 + d_r] fp16
+//   prefill_kv_tc_kernel  K^C_i[l] = W^UK_i c_l,  V_i[l] = W^UV_i c_l
+//                         -> kc [H, L, 128] fp16, v [H, L, 128] bf16, and
+//                         kr [L, d_r] fp16 (the rows' k^R, converted once)
+//                         one CTA per (128 rows l, head i): A = latent rows
+//                         (K-major, K = d_c = 512), B = [W^UK_i ; W^UV_i]
+//                         (256 rows, K-major), D [128 x 256] fp32 in TMEM
+//   prefill_attn_tc_kernel  causal softmax attention of head i, 128 queries
+//                         per CTA, 128-key tiles; the key of row l is
+//                         [K^C_i[l] ; k^R_l] (k^R read from the latent rows,
+//                         already rotated), head dim 128 + d_r, value dim 128
+//
+// The causal rule: query t sees rows l <= q_pos[t] (clamped to L - 1); a
+// query with q_pos[t] < 0 sees nothing (out 0, lse -inf).
+// Precision: the QK^T operands (queries, K^C, k^R) are fp16 and P, V are
+// bf16, all with fp32 accumulation.  Materialising K adds a rounding that the
+// absorbed decode does not have, and with a peaked softmax bf16 keys and
+// queries alone put the output 3 % off the exact result; fp16's 11-bit
+// significand brings that under 0.5 %.  Queries, keys and k^R must lie within
+// fp16's range (|x| < 65504).
+// Every wait is bounded; on give-up a kernel records MLA_ERR_DEVICE_TIMEOUT,
+// drains what it issued and skips its stores.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tensor_map.cuh"
+
+namespace mla {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kDn = 128;       // d_nope
+constexpr int kDv = 128;       // d_v
+constexpr int kDcP = 512;      // d_c
+constexpr int kTileQ = 128;    // queries per attention CTA
+constexpr int kTileK = 128;    // keys per attention tile
+constexpr int kBox = 16384;    // one [128 rows x 64] bf16 box, 128-byte swizzle
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  const __half2 p = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+// 8 bf16 (one 16-byte unit) -> 8 fp16.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+  uint4 r;
+  uint32_t* o = reinterpret_cast<uint32_t*>(&r);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(b[j]);
+    o[j] = pack_f16x2(f.x, f.y);
+  }
+  return r;
+}
+
+// Block-wide bounded wait (every calling thread polls; no abort flag).
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
+  volatile int no_abort = 0;
+  return mbar_wait(bar, parity, &no_abort, kWaitLimitCycles);
+}
+
+// ---------------------------------------------------------------------------
+// Queries: one thread per (t, i, 16-byte unit of the 128 + d_r output dims).
+__global__ void prefill_q_kernel(const __nv_bfloat16* __restrict__ q_nope,
+                                 const __nv_bfloat16* __restrict__ q_pe,
+                                 const int32_t* __restrict__ q_pos, int T, int H, int d_r,
+                                 float rope_base, __half* __restrict__ q_full) {
+  const int dq = kDn + d_r;
+  const int units = dq / 8;
+  const int64_t n = int64_t(T) * H * units;
+  for (int64_t k = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; k < n;
+       k += int64_t(gridDim.x) * blockDim.x) {
+    const int u = int(k % units);
+    const int64_t ti = k / units;
+    const int i = int(ti % H), t = int(ti / H);
+    uint4 v;
+    if (u < kDn / 8) {
+      v = bf16x8_to_f16x8(*reinterpret_cast<const uint4*>(q_nope + ti * kDn + u * 8));
+    } else {
+      // RoPE pairs (k, k + d_r/2) for the 8 k of this unit's half.
+      const int half = d_r / 2;
+      const int e0 = (u - kDn / 8) * 8;          // first output dim within the RoPE block
+      const bool upper = e0 >= half;
+      const int k0 = upper ? e0 - half : e0;
+      const __nv_bfloat16* src = q_pe + ti * d_r;
+      float y[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float x1 = __bfloat162float(src[k0 + j]);
+        const float x2 = __bfloat162float(src[k0 + j + half]);
+        float c, s;
+        rope_cos_sin(q_pos[t] < 0 ? 0 : q_pos[t], k0 + j, d_r, rope_base, &c, &s);
+        y[j] = upper ? x1 * s + x2 * c : x1 * c - x2 * s;
+      }
+      v = make_uint4(pack_f16x2(y[0], y[1]), pack_f16x2(y[2], y[3]), pack_f16x2(y[4], y[5]),
+                     pack_f16x2(y[6], y[7]));
+    }
+    *reinterpret_cast<uint4*>(q_full + (int64_t(i) * T + t) * dq + u * 8) = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K/V materialisation.  smem: 4 stages x (A [128 x 128 B] | B [256 x 128 B])
+constexpr int kKvStages = 4;
+constexpr int kKvStage = kBox + 2 * kBox;                  // 48 KB
+constexpr size_t kKvSmem = size_t(kKvStages) * kKvStage + 8 * (2 * kKvStages + 1) + 16 + 1024;
+constexpr int kKvThreads = 128;
+
+__global__ void __launch_bounds__(kKvThreads, 1)
+prefill_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_rows,
+                     const __grid_constant__ CUtensorMap tm_wuk,
+                     const __grid_constant__ CUtensorMap tm_wuv, int64_t L, int H, int d_r,
+                     const __nv_bfloat16* __restrict__ rows, __half* __restrict__ kc,
+                     __nv_bfloat16* __restrict__ v, __half* __restrict__ kr,
+                     int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kKvStages * kKvStage);
+  uint64_t* empty = full + kKvStages;
+  uint64_t* done = empty + kKvStages;
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(done + 1);
+  __shared__ int s_abort;
+  const int64_t l0 = int64_t(blockIdx.x) * 128;
+  const int i = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kChunks = kDcP / 64;   // 8
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kKvStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    s_abort = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    tmem_alloc(tbase, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tbase;
+  volatile int* abort_flag = &s_abort;
+  bool ok = true;
+  int issued = 0;
+  if (warp == 1) {
+    if (lane == 0) {
+      for (int c = 0; c < kChunks; ++c) {
+        const int s = c % kKvStages;
+        if (c >= kKvStages &&
+            !(ok = mbar_wait(&empty[s], ((c / kKvStages) - 1) & 1, abort_flag, kWaitLimitCycles)))
+          break;
+        uint8_t* st = sm + s * kKvStage;
+        mbar_arrive_expect_tx(&full[s], kKvStage);
+        tma_load_2d(&tm_rows, &full[s], st, c * 64, int32_t(l0));
+        tma_load_2d(&tm_wuk, &full[s], st + kBox, c * 64, i * 128);
+        tma_load_2d(&tm_wuv, &full[s], st + 2 * kBox, c * 64, i * 128);
+        ++issued;
+      }
+      if (!ok) *abort_flag = 1;
+    }
+  } else if (warp == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, false);
+    for (int c = 0; c < kChunks; ++c) {
+      const int s = c % kKvStages;
+      bool got = mbar_try(&full[s], (c / kKvStages) & 1);
+      if (!__all_sync(0xffffffffu, got)) {
+        got = mbar_wait(&full[s], (c / kKvStages) & 1, abort_flag, kWaitLimitCycles);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          if (lane == 0) *abort_flag = 1;
+          break;
+        }
+      }
+      tc_fence_after();
+      const uint32_t st = smem_u32(sm + s * kKvStage);
+      const uint64_t a0 = smem_desc_sw128(st, 16, 1024);
+      const uint64_t b0 = smem_desc_sw128(st + kBox, 16, 1024);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_bf16_ss_w(tmem, a0 + uint64_t((k * 32) >> 4), b0 + uint64_t((k * 32) >> 4), idesc,
+                      (c | k) != 0);
+      mma_commit_w(&empty[s]);
+    }
+    mma_commit_w(done);
+  }
+  __syncthreads();
+  ok = wait_bar(done, 0) && ok && !*abort_flag;
+  tc_fence_after();
+  // D[r][n]: thread (warp w, lane t) holds row l0 + 32w + t; columns 0-127 are
+  // K^C, 128-255 are V.
+  const int64_t l = l0 + 32 * warp + lane;
+#pragma unroll 1
+  for (int c0 = 0; c0 < 256; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + uint32_t(c0), r);
+    tmem_wait_ld();
+    if (ok && l < L) {
+      const int64_t off = (int64_t(i) * L + l) * 128 + (c0 & 127);
+      const bool is_k = c0 < 128;                       // K^C fp16, V bf16
+      uint4* dst = reinterpret_cast<uint4*>(is_k ? static_cast<void*>(kc + off)
+                                                 : static_cast<void*>(v + off));
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float a = __uint_as_float(r[e + 2 * j]), b = __uint_as_float(r[e + 2 * j + 1]);
+          w[j] = is_k ? pack_f16x2(a, b) : pack_bf16x2(a, b);
+        }
+        dst[e / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+  // The head-0 CTAs also convert their rows' k^R to fp16 (the QK^T operand).
+  if (i == 0 && d_r && ok && l < L) {
+    const uint4* src = reinterpret_cast<const uint4*>(rows + l * (kDcP + d_r) + kDcP);
+    uint4* dst = reinterpret_cast<uint4*>(kr + l * d_r);
+    for (int u = 0; u < d_r / 8; ++u) dst[u] = bf16x8_to_f16x8(src[u]);
+  }
+  if (!ok && threadIdx.x == 0) record_status(status, MLA_ERR_DEVICE_TIMEOUT);
+  // Loads issued but never consumed land before the shared memory is released.
+  if (warp == 1 && lane == 0) {
+    for (int k = issued > kKvStages ? issued - kKvStages : 0; k < issued; ++k)
+      wait_bar(&full[k % kKvStages], (k / kKvStages) & 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Causal attention.  smem: Q 3 x [128 x 128 B] | 2 stages x (K 3 x [128 x 128 B]
+// | V 2 x [128 x 128 B]) | barriers.  Tensor memory (512 columns): O [128 x
+// 128] fp32 at 0, S double buffer 2 x 128 at 128, P (bf16 pairs) 2 x 64 at 384.
+constexpr int kAtStages = 2;
+constexpr int kAtThreads = 192;      // warps 0-3 softmax + epilogue, 4 TMA, 5 MMA
+constexpr int kAtProducer = 4;
+constexpr int kAtMma = 5;
+constexpr int kQBytes = 3 * kBox;
+constexpr int kKBytes = 3 * kBox;
+constexpr int kVBytes = 2 * kBox;
+constexpr int kAtStage = kKBytes + kVBytes;                // 80 KB
+constexpr uint32_t kColO = 0, kColS = 128, kColP = 384;
+constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by > 2^8
+
+struct AttnBars {
+  uint64_t q_full;
+  uint64_t full[kAtStages], empty[kAtStages];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int max_vis;
+};
+constexpr size_t kAtSmem = size_t(kQBytes) + kAtStages * kAtStage + sizeof(AttnBars) + 1024;
+static_assert(kAtSmem <= 232448, "shared memory budget of one CTA");
+
+// Warp-uniform bounded wait that also gives up when another role aborted.
+__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag) {
+  if (__all_sync(0xffffffffu, mbar_try(bar, parity))) return true;
+  const bool ok = mbar_wait(bar, parity, abort_flag, kWaitLimitCycles);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(kAtThreads, 1)
+prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_kc,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_kr,
+                       const int32_t* __restrict__ q_pos, int T, int64_t L, int H, int d_r,
+                       float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                       int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint8_t* sQ = sm;
+  uint8_t* sStage = sm + kQBytes;
+  AttnBars* bars = reinterpret_cast<AttnBars*>(sStage + kAtStages * kAtStage);
+  const int i = blockIdx.x;
+  const int qt = int(gridDim.y) - 1 - int(blockIdx.y);   // the longest query tiles first
+  const int q0 = qt * kTileQ;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nq = (kDn + d_r) / 64;                       // 64-wide chunks of the head dim
+  volatile int* abort_flag = &bars->abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kAtStages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->p_full[b], 128);
+      mbar_init(&bars->pv_done[b], 1);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    bars->max_vis = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kAtMma) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  // Rows this CTA's queries may see: vis = min(q_pos + 1, L), 0 past T or
+  // for a negative position.
+  int64_t vis = 0;
+  if (threadIdx.x < kTileQ) {
+    const int t = q0 + threadIdx.x;
+    const int32_t pos = t < T ? q_pos[t] : -1;
+    vis = pos < 0 ? 0 : (int64_t(pos) + 1 < L ? int64_t(pos) + 1 : L);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < kTileQ && vis > 0) atomicMax(&bars->max_vis, int(vis));
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int n_tiles = int((int64_t(bars->max_vis) + kTileK - 1) / kTileK);
+  bool ok = true;
+
+  if (warp == kAtProducer) {
+    // ---------------------------------------------------------------- TMA
+    int issued = 0;
+    if (lane == 0 && n_tiles > 0) {
+      mbar_arrive_expect_tx(&bars->q_full, uint32_t(nq * kBox));
+      for (int c = 0; c < nq; ++c)
+        tma_load_2d(&tm_q, &bars->q_full, sQ + c * kBox, c * 64, int32_t(int64_t(i) * T + q0));
+      for (int k = 0; k < n_tiles; ++k) {
+        const int s = k % kAtStages;
+        if (k >= kAtStages &&
+            !(ok = mbar_wait(&bars->empty[s], ((k / kAtStages) - 1) & 1, abort_flag,
+                             kWaitLimitCycles)))
+          break;
+        uint8_t* st = sStage + s * kAtStage;
+        const int32_t row = int32_t(int64_t(i) * L + int64_t(k) * kTileK);
+        mbar_arrive_expect_tx(&bars->full[s], uint32_t((nq + 2) * kBox));
+        tma_load_2d(&tm_kc, &bars->full[s], st, 0, row);
+        tma_load_2d(&tm_kc, &bars->full[s], st + kBox, 64, row);
+        if (d_r) tma_load_2d(&tm_kr, &bars->full[s], st + 2 * kBox, 0, k * kTileK);
+        tma_load_2d(&tm_v, &bars->full[s], st + kKBytes, 0, row);
+        tma_load_2d(&tm_v, &bars->full[s], st + kKBytes + kBox, 64, row);
+        ++issued;
+      }
+      if (!ok) *abort_flag = 1;
+      // Every issued load lands before the shared memory is released.
+      wait_bar(&bars->q_full, 0);
+      for (int k = issued > kAtStages ? issued - kAtStages : 0; k < issued; ++k)
+        wait_bar(&bars->full[k % kAtStages], (k / kAtStages) & 1);
+    }
+  } else if (warp == kAtMma) {
+    // ---------------------------------------------------------------- MMA
+    if (n_tiles > 0) {
+      constexpr uint32_t idesc_qk = idesc_f16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+      ok = warp_wait_bar(&bars->q_full, 0, abort_flag);
+      auto issue_pv = [&](int j) -> bool {
+        const int b = j & 1;
+        if (!warp_wait_bar(&bars->p_full[b], (j >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t v0 = smem_desc_sw128(smem_u32(sStage + (j % kAtStages) * kAtStage + kKBytes),
+                                            kBox, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 16; ++kk)
+          mma_bf16_ts_w(tmem + kColO, tmem + kColP + uint32_t(b * 64 + kk * 8),
+                        v0 + uint64_t((kk * 2048) >> 4), idesc_pv, j > 0 || kk > 0);
+        mma_commit_w(&bars->pv_done[b]);
+        mma_commit_w(&bars->empty[j % kAtStages]);
+        return true;
+      };
+      for (int k = 0; ok && k < n_tiles; ++k) {
+        const int s = k % kAtStages;
+        if (!(ok = warp_wait_bar(&bars->full[s], (k / kAtStages) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t sk = smem_u32(sStage + s * kAtStage);
+        const uint32_t d = tmem + kColS + uint32_t((k & 1) * 128);
+        for (int c = 0; c < nq; ++c) {
+          const uint64_t a0 = smem_desc_sw128(smem_u32(sQ + c * kBox), 16, 1024);
+          const uint64_t b0 = smem_desc_sw128(sk + uint32_t(c * kBox), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss_w(d, a0 + uint64_t((kk * 32) >> 4), b0 + uint64_t((kk * 32) >> 4),
+                          idesc_qk, (c | kk) != 0);
+        }
+        mma_commit_w(&bars->s_full[k & 1]);
+        if (k >= 1 && !(ok = issue_pv(k - 1))) break;
+      }
+      if (ok) ok = issue_pv(n_tiles - 1);
+      if (!ok && lane == 0) *abort_flag = 1;
+    }
+    // Every product issued has finished before tensor memory is released.
+    mma_commit_w(&bars->drain);
+    if (lane == 0) wait_bar(&bars->drain, 0);
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- softmax
+    const int r = threadIdx.x;                 // query row q0 + r, tensor-memory lane r
+    const uint32_t lane_base = uint32_t(32 * warp) << 16;
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int k = 0; k < n_tiles; ++k) {
+      const int b = k & 1;
+      if (!(ok = warp_wait_bar(&bars->s_full[b], (k >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      const int64_t nv = vis - int64_t(k) * kTileK;
+      const int nvalid = nv <= 0 ? 0 : (nv >= kTileK ? kTileK : int(nv));
+      const uint32_t s_addr = tmem + lane_base + kColS + uint32_t(b * 128);
+      float mt = -INFINITY;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kTileK; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(s_addr + uint32_t(c0), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (c0 + e < nvalid) mt = fmaxf(mt, __uint_as_float(v[e]));
+      }
+      const float m_new = fmaxf(m_run, mt * scale_log2);
+      const bool rescale = m_run != -INFINITY && m_new > m_run + kRescaleLog2;
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O holds the products up to tile k - 1: wait for the last of them.
+        if (!(ok = warp_wait_bar(&bars->pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort_flag)))
+          break;
+        tc_fence_after();
+        const float f = rescale ? ex2_approx(m_run - m_new) : 1.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kDv; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + kColO + uint32_t(c0), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+          tmem_st32(tmem + lane_base + kColO + uint32_t(c0), v);
+        }
+        tmem_wait_st();
+        if (rescale) {
+          l_run *= f;
+          m_run = m_new;
+        }
+      }
+      if (m_run == -INFINITY) m_run = m_new;
+      // P buffer b was last read by the product of tile k - 2.
+      if (k >= 2 && !(ok = warp_wait_bar(&bars->pv_done[b], ((k - 2) >> 1) & 1, abort_flag)))
+        break;
+      tc_fence_after();
+      const float mu = m_run == -INFINITY ? 0.f : m_run;
+      float sum = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kTileK; c0 += 32) {
+        uint32_t v[32], pk[16];
+        tmem_ld32(s_addr + uint32_t(c0), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = c0 + e < nvalid ? ex2_approx(fmaf(__uint_as_float(v[e]), scale_log2, -mu)) : 0.f;
+          const float p1 =
+              c0 + e + 1 < nvalid ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), scale_log2, -mu)) : 0.f;
+          sum += p0 + p1;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tmem + lane_base + kColP + uint32_t(b * 64 + c0 / 2), pk);
+      }
+      tmem_wait_st();
+      l_run += sum;
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[b]);
+    }
+    if (!ok) {
+      bars->abort_flag = 1;
+    } else if (n_tiles > 0) {
+      ok = warp_wait_bar(&bars->pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag);
+      tc_fence_after();
+    }
+    const int t = q0 + r;
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kDv; c0 += 32) {
+      uint32_t v[32];
+      if (n_tiles > 0) {
+        tmem_ld32(tmem + lane_base + kColO + uint32_t(c0), v);
+        tmem_wait_ld();
+      }
+      if (ok && t < T) {
+        __nv_bfloat16* dst = out + (int64_t(t) * H + i) * kDv + c0;
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          float x[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) x[j] = n_tiles > 0 ? __uint_as_float(v[e + j]) * inv : 0.f;
+          *reinterpret_cast<uint4*>(dst + e) =
+              make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                         pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+        }
+      }
+    }
+    if (ok && t < T && lse)
+      lse[int64_t(t) * H + i] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f
+                                            : -INFINITY;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && bars->abort_flag) record_status(status, MLA_ERR_DEVICE_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kAtMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <typename K>
+cudaError_t set_smem_once(K kernel, size_t bytes) {
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (done[dev]) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
+size_t round1k(size_t x) { return (x + 1023) / 1024 * 1024; }
+
+}  // namespace
+
+size_t prefill_workspace_bytes(int T, int64_t L, int H, int d_r) {
+  return round1k(size_t(H) * T * (kDn + d_r) * 2) + 2 * round1k(size_t(H) * L * 128 * 2) +
+         round1k(size_t(L) * d_r * 2);
+}
+
+cudaError_t launch_prefill(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_pe,
+                           const int32_t* q_pos, const __nv_bfloat16* W_UK,
+                           const __nv_bfloat16* W_UV, const __nv_bfloat16* rows, int T, int64_t L,
+                           int H, int d_r, float scale, float rope_base, __nv_bfloat16* out,
+                           float* lse, void* workspace, int* status, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  const int dq = kDn + d_r;
+  const int R = kDcP + d_r;
+  // Workspace: q_full [H, T, dq] fp16 | kc [H, L, 128] fp16 | v [H, L, 128]
+  // bf16 | kr [L, d_r] fp16, each rounded up to 1 KB.
+  uint8_t* p = static_cast<uint8_t*>(workspace);
+  __half* q_full = reinterpret_cast<__half*>(p);
+  p += round1k(size_t(H) * T * dq * 2);
+  __half* kc = reinterpret_cast<__half*>(p);
+  p += round1k(size_t(H) * L * 128 * 2);
+  __nv_bfloat16* v = reinterpret_cast<__nv_bfloat16*>(p);
+  p += round1k(size_t(H) * L * 128 * 2);
+  __half* kr = reinterpret_cast<__half*>(p);
+  const int64_t nq_units = int64_t(T) * H * (dq / 8);
+  const int qb = int((nq_units + 255) / 256 < 4096 ? (nq_units + 255) / 256 : 4096);
+  prefill_q_kernel<<<qb, 256, 0, stream>>>(q_nope, q_pe, q_pos, T, H, d_r, rope_base, q_full);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap tm_rows, tm_wuk, tm_wuv, tm_q, tm_kc, tm_v, tm_kr;
+  if (!make_map16(&tm_rows, rows, uint64_t(L), uint64_t(R), uint64_t(R), 128) ||
+      !make_map16(&tm_wuk, W_UK, uint64_t(H) * 128, kDcP, kDcP, 128) ||
+      !make_map16(&tm_wuv, W_UV, uint64_t(H) * 128, kDcP, kDcP, 128) ||
+      !make_map16(&tm_q, q_full, uint64_t(H) * T, uint64_t(dq), uint64_t(dq), 128) ||
+      !make_map16(&tm_kc, kc, uint64_t(H) * L, 128, 128, 128) ||
+      !make_map16(&tm_v, v, uint64_t(H) * L, 128, 128, 128))
+    return cudaErrorInvalidValue;
+  // Without RoPE the k^R map is never read; it is built over kc instead.
+  if (!(d_r ? make_map16(&tm_kr, kr, uint64_t(L), uint64_t(d_r), uint64_t(d_r), 128)
+            : make_map16(&tm_kr, kc, uint64_t(H) * L, 128, 128, 128)))
+    return cudaErrorInvalidValue;
+
+  if ((e = set_smem_once(prefill_kv_tc_kernel, kKvSmem)) != cudaSuccess) return e;
+  prefill_kv_tc_kernel<<<dim3(unsigned((L + 127) / 128), H), kKvThreads, kKvSmem, stream>>>(
+      tm_rows, tm_wuk, tm_wuv, L, H, d_r, rows, kc, v, kr, status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  if ((e = set_smem_once(prefill_attn_tc_kernel, kAtSmem)) != cudaSuccess) return e;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  prefill_attn_tc_kernel<<<dim3(H, unsigned((T + kTileQ - 1) / kTileQ)), kAtThreads, kAtSmem,
+                           stream>>>(tm_q, tm_kc, tm_v, tm_kr, q_pos, T, L, H, d_r, scale_log2,
+                                     out, lse, status);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -108,4 +108,15 @@ cudaError_t launch_folded_proj(const float* o_lat, const __nv_bfloat16* w_fold, 
                                int d_model, void* workspace, __nv_bfloat16* u, int* status,
                                cudaStream_t stream);
 
+// Materialised prefill of one sequence (bf16, d_c = 512, d_nope = d_v = 128,
+// d_r = 64 or 0): q_nope [T, H, 128], q_pe [T, H, d_r], q_pos [T], rows
+// [L, 512 + d_r] -> out [T, H, 128] bf16, lse [T, H] fp32 (nullable).  The
+// workspace holds the rotated queries and the materialised K^C and V.
+size_t prefill_workspace_bytes(int T, int64_t L, int H, int d_r);
+cudaError_t launch_prefill(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_pe,
+                           const int32_t* q_pos, const __nv_bfloat16* W_UK,
+                           const __nv_bfloat16* W_UV, const __nv_bfloat16* rows, int T, int64_t L,
+                           int H, int d_r, float scale, float rope_base, __nv_bfloat16* out,
+                           float* lse, void* workspace, int* status, cudaStream_t stream);
+
 }  // namespace mla

@@ -408,6 +408,52 @@ int mla_decode_fp8(const mla_dims* d, const void* q_cat, const void* cache, cons
 }
 
 // ---------------------------------------------------------------------------
+// Materialised prefill of one sequence.
+namespace {
+int check_prefill(const mla_dims* d, int32_t T, int64_t L) {
+  if (!d) return MLA_ERR_INVALID_ARG;
+  if (d->H <= 0 || T < 0 || L <= 0) return MLA_ERR_INVALID_ARG;
+  if (d->dtype != MLA_BF16 || d->d_c != 512 || d->d_nope != 128 || d->d_v != 128 ||
+      (d->d_r != 64 && d->d_r != 0) || d->H > 65535)
+    return MLA_ERR_UNSUPPORTED;
+  // 32-bit TMA row coordinates over [H * L] and [H * T] matrices.
+  if (int64_t(d->H) * L >= (int64_t(1) << 31) || int64_t(d->H) * T >= (int64_t(1) << 31))
+    return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+}  // namespace
+
+size_t mla_prefill_workspace_bytes(const mla_dims* d, int32_t T, int64_t L) {
+  if (check_prefill(d, T, L) != MLA_OK) return 0;
+  return prefill_workspace_bytes(T, L, d->H, d->d_r);
+}
+
+int mla_prefill(const mla_dims* d, int32_t T, int64_t L, const void* q_nope, const void* q_pe,
+                const int32_t* q_pos, const void* W_UK, const void* W_UV, const void* rows,
+                float softmax_scale, float rope_base, void* out, float* lse, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  int st = check_prefill(d, T, L);
+  if (st) return st;
+  if (T == 0) return MLA_OK;
+  if (!q_nope || (d->d_r && !q_pe) || !q_pos || !W_UK || !W_UV || !rows || !out)
+    return MLA_ERR_INVALID_ARG;
+  softmax_scale = effective_scale(d, softmax_scale);
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale) || !(rope_base > 0.f))
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || (q_pe && !aligned16(q_pe)) || !aligned16(W_UK) ||
+      !aligned16(W_UV) || !aligned16(rows) || !aligned16(out) || (workspace && !aligned16(workspace)))
+    return MLA_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < prefill_workspace_bytes(T, L, d->H, d->d_r))
+    return MLA_ERR_WORKSPACE;
+  return cuda_status(launch_prefill(
+      static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_pe), q_pos,
+      static_cast<const __nv_bfloat16*>(W_UK), static_cast<const __nv_bfloat16*>(W_UV),
+      static_cast<const __nv_bfloat16*>(rows), T, L, d->H, d->d_r, softmax_scale, rope_base,
+      static_cast<__nv_bfloat16*>(out), lse, workspace, status_ptr(),
+      static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------------------
 // W^O folded into the value side.
 namespace {
 int check_fold(const mla_dims* d, int32_t d_model) {

@@ -154,6 +154,61 @@ def test_other_entry_point_errors(lib):
     assert ap(ws=None) == WS
 
 
+def test_prefill_entry_point_errors(lib):
+    d = _dims(H=8)
+    need = lib.mla_prefill_workspace_bytes(ctypes.byref(d), 100, 300)
+    # q_full [H, T, 192] + K^C and V [H, L, 128] + k^R [L, 64], each rounded
+    # up to 1 KB.
+    r1k = lambda x: (x + 1023) // 1024 * 1024  # noqa: E731
+    assert need == r1k(8 * 100 * 192 * 2) + 2 * r1k(8 * 300 * 128 * 2) + r1k(300 * 64 * 2)
+    pf = lambda T=100, L=300, qn=GOOD, qpe=GOOD, pos=GOOD, scale=0.0, base=1e4, out=GOOD2, \
+        ws=GOOD2, n=need, dims=d: lib.mla_prefill(  # noqa: E731
+            ctypes.byref(dims), T, L, qn, qpe, pos, GOOD, GOOD, GOOD, scale, base, out, None,
+            ws, n, None)
+    assert pf(T=0) == OK                     # nothing to do, nothing launched
+    assert pf(T=-1) == INVALID
+    assert pf(L=0) == INVALID
+    assert pf(qn=None) == INVALID
+    assert pf(pos=None) == INVALID
+    assert pf(qpe=None) == INVALID           # d_r = 64 needs q_pe
+    assert pf(scale=-0.1) == INVALID
+    assert pf(base=0.0) == INVALID
+    assert pf(out=BAD) == ALIGN
+    assert pf(n=need - 1) == WS
+    assert pf(ws=None) == WS
+    for bad in (dict(dtype=bd.MLA_F32), dict(d_c=256), dict(d_r=32), dict(d_v=64)):
+        dd = _dims(H=8, **bad)
+        assert pf(dims=dd) == UNSUP
+        assert lib.mla_prefill_workspace_bytes(ctypes.byref(dd), 100, 300) == 0
+    assert pf(L=1 << 28) == UNSUP            # H * L beyond a 32-bit TMA row coordinate
+    d0 = _dims(H=8, d_r=0)
+    need0 = lib.mla_prefill_workspace_bytes(ctypes.byref(d0), 100, 300)
+    assert need0 == r1k(8 * 100 * 128 * 2) + 2 * r1k(8 * 300 * 128 * 2)
+    assert pf(dims=d0, qpe=None, n=need0 - 1) == WS   # NoPE: q_pe may be NULL
+
+
+def test_fold_entry_point_errors(lib):
+    d = _dims(B=32, H=8)
+    fw = lambda dm=300, wo=GOOD, dims=d: lib.mla_fold_output_weights(  # noqa: E731
+        ctypes.byref(dims), dm, wo, GOOD, GOOD2, None)
+    assert fw(dm=0) == INVALID
+    assert fw(wo=None) == INVALID
+    assert fw(wo=BAD) == ALIGN
+    assert fw(dims=_dims(B=32, H=8, dtype=bd.MLA_F32)) == UNSUP
+    assert fw(dims=_dims(B=32, H=8, d_v=64)) == UNSUP
+    need = lib.mla_out_proj_folded_workspace_bytes(ctypes.byref(d), 300)
+    assert need > 0
+    fp = lambda dims=d, ws=GOOD2, n=need, x=GOOD: lib.mla_out_proj_folded(  # noqa: E731
+        ctypes.byref(dims), 300, x, GOOD, GOOD, ws, n, None)
+    assert fp(x=None) == INVALID
+    assert fp(x=BAD) == ALIGN
+    assert fp(n=need - 1) == WS
+    assert fp(ws=None) == WS
+    big = _dims(B=65, H=8)
+    assert lib.mla_out_proj_folded_workspace_bytes(ctypes.byref(big), 300) == 0
+    assert fp(dims=big) == UNSUP
+
+
 def test_paged_entry_point_errors(lib):
     d = _dims(cache_capacity=4096)          # 64 pages of 64 rows per sequence at most
     need = lib.mla_decode_workspace_bytes(ctypes.byref(d), 8)
