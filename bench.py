@@ -332,53 +332,21 @@ def run_ours(args, rank, world, local_rank):
                 h_out.copy_(step.out, non_blocking=True)
                 seq.copy_(seq0)
     else:
-        # Pipelined: two device input sets, each with a graph of the step; the
-        # copy stream brings step k+1's inputs in and takes step k's output
-        # out while step k computes.  Every step still copies its own inputs
-        # from pinned host memory and its result back to it.
-        copy_stream = torch.cuda.Stream(device=dev)
-        sets = []
-        for _ in range(2):
-            d_in = [t.clone() for t in (q_nope, q_pe, q_pos, hh)]
-            stage = torch.empty_like(step.out)
-
-            def after(stage=stage):
-                if flush is not None:
-                    flush.zero_()
-                stage.copy_(step.out)
-                seq.copy_(seq0)
-            g = step.capture(d_in[0], d_in[1], d_in[2], cache, seq, h=d_in[3], after=after,
-                             block_table=table, scales=scales)
-            sets.append((d_in, stage, g))
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        ev_out = [torch.cuda.Event() for _ in range(2)]
-
-        def load_inputs(c):
-            for d_t, h_t in zip(sets[c][0], host_in):
-                d_t.copy_(h_t, non_blocking=True)
-            ev_in[c].record(copy_stream)
+        # Pipelined through DecodeStep.host_pipeline: one graph launch per
+        # step runs the step on one device input set while a copy stream
+        # brings the next step's inputs in from pinned host memory and takes
+        # the previous step's output out; every step still copies its own
+        # inputs and result.
+        def after():
+            if flush is not None:
+                flush.zero_()
+            seq.copy_(seq0)
+        pipe = step.host_pipeline(host_in, h_out, cache, seq, after=after, block_table=table,
+                                  scales=scales)
+        assert pipe.bytes_per_step() == (bi, bo)
 
         def e2e_run(n):
-            copy_stream.wait_stream(stream)
-            with torch.cuda.stream(copy_stream):
-                load_inputs(0)
-            for k in range(n):
-                c = k % 2
-                stream.wait_event(ev_in[c])
-                if k >= 2:
-                    stream.wait_event(ev_out[c])     # step k-2's result has left `stage`
-                sets[c][2].replay()
-                ev_done[c].record(stream)
-                with torch.cuda.stream(copy_stream):
-                    if k + 1 < n:
-                        if k >= 1:
-                            copy_stream.wait_event(ev_done[1 - c])  # step k-1 read that set
-                        load_inputs(1 - c)
-                    copy_stream.wait_event(ev_done[c])
-                    h_out.copy_(sets[c][1], non_blocking=True)
-                    ev_out[c].record(copy_stream)
-            stream.wait_stream(copy_stream)
+            pipe.run(n)
 
     e2e_run(3)
     torch.cuda.synchronize()

@@ -533,6 +533,23 @@ class DecodeStep:
         main.wait_stream(self._side)
         return self._attend_latent(cache, seqlens, block_table, scales)
 
+    def host_pipeline(self, host_inputs, host_out, cache, seqlens, after=None,
+                      block_table=None, scales=None):
+        """Steps fed from pinned host memory with the copies overlapped.
+
+        ``host_inputs`` = (q_nope, q_pe, q_pos[, h]) pinned host tensors,
+        ``host_out`` a pinned host tensor shaped like ``self.out``.  Two device
+        input sets and two output stages alternate; each is served by one CUDA
+        graph that runs a step on set c while a forked copy stream brings the
+        next step's inputs into set 1 - c and takes the previous step's
+        output from stage 1 - c to ``host_out``.  So every step still copies
+        its own inputs in and its result out, but one graph launch per step
+        does it.  ``run(n)`` performs n steps, with the first step's inputs
+        copied in before and the last result copied out after; ``host_out``
+        holds the last step's result once the stream has finished."""
+        return _HostPipeline(self, host_inputs, host_out, cache, seqlens, after, block_table,
+                             scales)
+
     def capture(self, q_nope, q_pe, q_pos, cache, seqlens, h=None, before=None, after=None,
                 block_table=None, scales=None):
         """Record one step into a CUDA graph; ``before``/``after`` are optional
@@ -547,3 +564,54 @@ class DecodeStep:
             if after is not None:
                 after()
         return g
+
+
+class _HostPipeline:
+    """See DecodeStep.host_pipeline."""
+
+    def __init__(self, step, host_inputs, host_out, cache, seqlens, after, block_table, scales):
+        for t in (*host_inputs, host_out):
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError("host_pipeline needs pinned host tensors")
+        self.step, self.host_in, self.host_out = step, tuple(host_inputs), host_out
+        dev = step.out.device
+        self.sets = [[torch.empty_like(t, device=dev) for t in self.host_in] for _ in range(2)]
+        self.stages = [torch.empty_like(step.out) for _ in range(2)]
+        # Host->device and device->host copies on separate streams, so the two
+        # directions overlap each other as well as the step.
+        self.in_stream = torch.cuda.Stream(device=dev)
+        self.out_stream = torch.cuda.Stream(device=dev)
+        self.graphs = []
+        for c in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                main = torch.cuda.current_stream()
+                self.in_stream.wait_stream(main)
+                self.out_stream.wait_stream(main)
+                with torch.cuda.stream(self.in_stream):
+                    for d_t, h_t in zip(self.sets[1 - c], self.host_in):
+                        d_t.copy_(h_t, non_blocking=True)
+                with torch.cuda.stream(self.out_stream):
+                    self.host_out.copy_(self.stages[1 - c], non_blocking=True)
+                x = self.sets[c]
+                step(x[0], x[1], x[2], cache, seqlens, h=x[3] if len(x) > 3 else None,
+                     block_table=block_table, scales=scales)
+                self.stages[c].copy_(step.out)
+                if after is not None:
+                    after()
+                main.wait_stream(self.in_stream)
+                main.wait_stream(self.out_stream)
+            self.graphs.append(g)
+
+    def run(self, n: int):
+        for d_t, h_t in zip(self.sets[0], self.host_in):
+            d_t.copy_(h_t, non_blocking=True)
+        for k in range(n):
+            self.graphs[k % 2].replay()
+        if n:
+            self.host_out.copy_(self.stages[(n - 1) % 2], non_blocking=True)
+
+    def bytes_per_step(self):
+        """(host->device, device->host) bytes each step copies."""
+        return (sum(t.numel() * t.element_size() for t in self.host_in),
+                self.host_out.numel() * self.host_out.element_size())

@@ -79,26 +79,35 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------------------
-// Queries: one thread per (t, i, 16-byte unit of the 128 + d_r output dims).
-__global__ void prefill_q_kernel(const __nv_bfloat16* __restrict__ q_nope,
-                                 const __nv_bfloat16* __restrict__ q_pe,
-                                 const int32_t* __restrict__ q_pos, int T, int H, int d_r,
-                                 float rope_base, __half* __restrict__ q_full) {
+// Queries: one block per token t.  The rotation angles depend on (t, pair)
+// only, so the block forms the d_r/2 (cos, sin) pairs once and every head
+// uses them; each thread then writes 16-byte units of the H rows.
+constexpr int kQThreads = 256;
+
+__global__ void __launch_bounds__(kQThreads)
+prefill_q_kernel(const __nv_bfloat16* __restrict__ q_nope, const __nv_bfloat16* __restrict__ q_pe,
+                 const int32_t* __restrict__ q_pos, int T, int H, int d_r, float rope_base,
+                 __half* __restrict__ q_full) {
+  __shared__ float s_cos[32], s_sin[32];
+  const int t = blockIdx.x;
+  const int half = d_r / 2;
+  if (threadIdx.x < half) {
+    const int32_t pos = q_pos[t];
+    rope_cos_sin(pos < 0 ? 0 : pos, threadIdx.x, d_r, rope_base, &s_cos[threadIdx.x],
+                 &s_sin[threadIdx.x]);
+  }
+  __syncthreads();
   const int dq = kDn + d_r;
   const int units = dq / 8;
-  const int64_t n = int64_t(T) * H * units;
-  for (int64_t k = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; k < n;
-       k += int64_t(gridDim.x) * blockDim.x) {
-    const int u = int(k % units);
-    const int64_t ti = k / units;
-    const int i = int(ti % H), t = int(ti / H);
+  for (int k = threadIdx.x; k < H * units; k += kQThreads) {
+    const int u = k % units, i = k / units;
+    const int64_t ti = int64_t(t) * H + i;
     uint4 v;
     if (u < kDn / 8) {
       v = bf16x8_to_f16x8(*reinterpret_cast<const uint4*>(q_nope + ti * kDn + u * 8));
     } else {
-      // RoPE pairs (k, k + d_r/2) for the 8 k of this unit's half.
-      const int half = d_r / 2;
-      const int e0 = (u - kDn / 8) * 8;          // first output dim within the RoPE block
+      // Output dims e0 .. e0+7 of the RoPE block: pairs (k, k + d_r/2).
+      const int e0 = (u - kDn / 8) * 8;
       const bool upper = e0 >= half;
       const int k0 = upper ? e0 - half : e0;
       const __nv_bfloat16* src = q_pe + ti * d_r;
@@ -107,9 +116,8 @@ __global__ void prefill_q_kernel(const __nv_bfloat16* __restrict__ q_nope,
       for (int j = 0; j < 8; ++j) {
         const float x1 = __bfloat162float(src[k0 + j]);
         const float x2 = __bfloat162float(src[k0 + j + half]);
-        float c, s;
-        rope_cos_sin(q_pos[t] < 0 ? 0 : q_pos[t], k0 + j, d_r, rope_base, &c, &s);
-        y[j] = upper ? x1 * s + x2 * c : x1 * c - x2 * s;
+        const float c = s_cos[k0 + j], sn = s_sin[k0 + j];
+        y[j] = upper ? x1 * sn + x2 * c : x1 * c - x2 * sn;
       }
       v = make_uint4(pack_f16x2(y[0], y[1]), pack_f16x2(y[2], y[3]), pack_f16x2(y[4], y[5]),
                      pack_f16x2(y[6], y[7]));
@@ -258,9 +266,12 @@ prefill_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_rows,
 // | V 2 x [128 x 128 B]) | barriers.  Tensor memory (512 columns): O [128 x
 // 128] fp32 at 0, S double buffer 2 x 128 at 128, P (bf16 pairs) 2 x 64 at 384.
 constexpr int kAtStages = 2;
-constexpr int kAtThreads = 192;      // warps 0-3 softmax + epilogue, 4 TMA, 5 MMA
-constexpr int kAtProducer = 4;
-constexpr int kAtMma = 5;
+// Warps 0-7 softmax + epilogue (warp w: rows 32 (w % 4) .., key/value
+// columns 64 (w / 4) ..: two threads per query row), 8 TMA, 9 MMA.
+constexpr int kAtSoftmaxThreads = 256;
+constexpr int kAtThreads = 320;
+constexpr int kAtProducer = 8;
+constexpr int kAtMma = 9;
 constexpr int kQBytes = 3 * kBox;
 constexpr int kKBytes = 3 * kBox;
 constexpr int kVBytes = 2 * kBox;
@@ -276,6 +287,8 @@ struct AttnBars {
   uint32_t tmem_base;
   int abort_flag;
   int max_vis;
+  float row_max[2][2][kTileQ];   // [tile parity][column half][row]: the halves' maxima
+  float row_sum[2][kTileQ];      // [column half][row]: the halves' sums, at the end
 };
 constexpr size_t kAtSmem = size_t(kQBytes) + kAtStages * kAtStage + sizeof(AttnBars) + 1024;
 static_assert(kAtSmem <= 232448, "shared memory budget of one CTA");
@@ -301,8 +314,10 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* sQ = sm;
   uint8_t* sStage = sm + kQBytes;
   AttnBars* bars = reinterpret_cast<AttnBars*>(sStage + kAtStages * kAtStage);
-  const int i = blockIdx.x;
-  const int qt = int(gridDim.y) - 1 - int(blockIdx.y);   // the longest query tiles first
+  // Query tiles vary fastest, so the CTAs in flight share a few heads' K and
+  // V through L2; within a head the longest query tiles start first.
+  const int i = blockIdx.y;
+  const int qt = int(gridDim.x) - 1 - int(blockIdx.x);
   const int q0 = qt * kTileQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nq = (kDn + d_r) / 64;                       // 64-wide chunks of the head dim
@@ -315,7 +330,7 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], 128);
+      mbar_init(&bars->p_full[b], kAtSoftmaxThreads);
       mbar_init(&bars->pv_done[b], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -331,8 +346,8 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   // Rows this CTA's queries may see: vis = min(q_pos + 1, L), 0 past T or
   // for a negative position.
   int64_t vis = 0;
-  if (threadIdx.x < kTileQ) {
-    const int t = q0 + threadIdx.x;
+  if (threadIdx.x < kAtSoftmaxThreads) {
+    const int t = q0 + (threadIdx.x & (kTileQ - 1));
     const int32_t pos = t < T ? q_pos[t] : -1;
     vis = pos < 0 ? 0 : (int64_t(pos) + 1 < L ? int64_t(pos) + 1 : L);
   }
@@ -420,42 +435,66 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax
-    const int r = threadIdx.x;                 // query row q0 + r, tensor-memory lane r
-    const uint32_t lane_base = uint32_t(32 * warp) << 16;
+    // Thread (warp w, lane) owns row r = 32 (w % 4) + lane, columns
+    // [64 h, 64 h + 64) with h = w / 4, of S, P and O.  The two halves of a row
+    // swap their maxima through shared memory once per tile (a 64-thread named
+    // barrier per lane quadrant) and apply the same rescales, so their partial
+    // sums add up at the end.
+    const int quad = warp & 3, h = warp >> 2;
+    const int r = 32 * quad + lane;
+    const uint32_t lane_base = uint32_t(32 * quad) << 16;
+    const int cb = 64 * h;
     float m_run = -INFINITY, l_run = 0.f;
+    // Both halves of a row run every iteration up to the named barrier, even
+    // after a give-up (then with no work), so the barrier never waits for a
+    // thread that left the loop.
     for (int k = 0; k < n_tiles; ++k) {
       const int b = k & 1;
-      if (!(ok = warp_wait_bar(&bars->s_full[b], (k >> 1) & 1, abort_flag))) break;
-      tc_fence_after();
-      const int64_t nv = vis - int64_t(k) * kTileK;
-      const int nvalid = nv <= 0 ? 0 : (nv >= kTileK ? kTileK : int(nv));
-      const uint32_t s_addr = tmem + lane_base + kColS + uint32_t(b * 128);
+      if (!ok) bars->abort_flag = 1;   // the other roles stop waiting for this warp
+      if (ok) ok = warp_wait_bar(&bars->s_full[b], (k >> 1) & 1, abort_flag);
+      const int64_t nv = vis - int64_t(k) * kTileK - cb;   // visible columns of this half
+      const int nvalid = nv <= 0 ? 0 : (nv >= 64 ? 64 : int(nv));
+      uint32_t va[32], vb[32];
       float mt = -INFINITY;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kTileK; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(s_addr + uint32_t(c0), v);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t s_addr = tmem + lane_base + kColS + uint32_t(b * 128 + cb);
+        tmem_ld32(s_addr, va);
+        tmem_ld32(s_addr + 32, vb);
         tmem_wait_ld();
+        if (nvalid == 64) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (c0 + e < nvalid) mt = fmaxf(mt, __uint_as_float(v[e]));
+          for (int e = 0; e < 32; ++e)
+            mt = fmaxf(mt, fmaxf(__uint_as_float(va[e]), __uint_as_float(vb[e])));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (e < nvalid) mt = fmaxf(mt, __uint_as_float(va[e]));
+            if (e + 32 < nvalid) mt = fmaxf(mt, __uint_as_float(vb[e]));
+          }
+        }
       }
+      bars->row_max[b][h][r] = mt;
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+      if (!ok) continue;
+      mt = fmaxf(mt, bars->row_max[b][1 - h][r]);
       const float m_new = fmaxf(m_run, mt * scale_log2);
       const bool rescale = m_run != -INFINITY && m_new > m_run + kRescaleLog2;
       if (__any_sync(0xffffffffu, rescale)) {
         // O holds the products up to tile k - 1: wait for the last of them.
         if (!(ok = warp_wait_bar(&bars->pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, abort_flag)))
-          break;
+          continue;
         tc_fence_after();
         const float f = rescale ? ex2_approx(m_run - m_new) : 1.f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kDv; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + kColO + uint32_t(c0), v);
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          uint32_t o[32];
+          const uint32_t oa = tmem + lane_base + kColO + uint32_t(cb + c0);
+          tmem_ld32(oa, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-          tmem_st32(tmem + lane_base + kColO + uint32_t(c0), v);
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+          tmem_st32(oa, o);
         }
         tmem_wait_st();
         if (rescale) {
@@ -466,25 +505,30 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (m_run == -INFINITY) m_run = m_new;
       // P buffer b was last read by the product of tile k - 2.
       if (k >= 2 && !(ok = warp_wait_bar(&bars->pv_done[b], ((k - 2) >> 1) & 1, abort_flag)))
-        break;
+        continue;
       tc_fence_after();
       const float mu = m_run == -INFINITY ? 0.f : m_run;
       float sum = 0.f;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kTileK; c0 += 32) {
-        uint32_t v[32], pk[16];
-        tmem_ld32(s_addr + uint32_t(c0), v);
-        tmem_wait_ld();
+      uint32_t pa[16], pb[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = c0 + e < nvalid ? ex2_approx(fmaf(__uint_as_float(v[e]), scale_log2, -mu)) : 0.f;
-          const float p1 =
-              c0 + e + 1 < nvalid ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), scale_log2, -mu)) : 0.f;
-          sum += p0 + p1;
-          pk[e / 2] = pack_bf16x2(p0, p1);
+      for (int e = 0; e < 32; e += 2) {
+        float p0 = ex2_approx(fmaf(__uint_as_float(va[e]), scale_log2, -mu));
+        float p1 = ex2_approx(fmaf(__uint_as_float(va[e + 1]), scale_log2, -mu));
+        float p2 = ex2_approx(fmaf(__uint_as_float(vb[e]), scale_log2, -mu));
+        float p3 = ex2_approx(fmaf(__uint_as_float(vb[e + 1]), scale_log2, -mu));
+        if (nvalid < 64) {
+          p0 = e < nvalid ? p0 : 0.f;
+          p1 = e + 1 < nvalid ? p1 : 0.f;
+          p2 = e + 32 < nvalid ? p2 : 0.f;
+          p3 = e + 33 < nvalid ? p3 : 0.f;
         }
-        tmem_st16(tmem + lane_base + kColP + uint32_t(b * 64 + c0 / 2), pk);
+        sum += (p0 + p1) + (p2 + p3);
+        pa[e / 2] = pack_bf16x2(p0, p1);
+        pb[e / 2] = pack_bf16x2(p2, p3);
       }
+      const uint32_t p_addr = tmem + lane_base + kColP + uint32_t(b * 64 + cb / 2);
+      tmem_st16(p_addr, pa);
+      tmem_st16(p_addr + 16, pb);
       tmem_wait_st();
       l_run += sum;
       tc_fence_before();
@@ -496,30 +540,35 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       ok = warp_wait_bar(&bars->pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag);
       tc_fence_after();
     }
+    // Row sum of both halves.  Both threads of a row reach this barrier
+    // whatever happened above (an abort only skips stores).
+    bars->row_sum[h][r] = l_run;
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+    const float l_row = bars->row_sum[0][r] + bars->row_sum[1][r];
     const int t = q0 + r;
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
 #pragma unroll 1
-    for (int c0 = 0; c0 < kDv; c0 += 32) {
-      uint32_t v[32];
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+      uint32_t o[32];
       if (n_tiles > 0) {
-        tmem_ld32(tmem + lane_base + kColO + uint32_t(c0), v);
+        tmem_ld32(tmem + lane_base + kColO + uint32_t(cb + c0), o);
         tmem_wait_ld();
       }
       if (ok && t < T) {
-        __nv_bfloat16* dst = out + (int64_t(t) * H + i) * kDv + c0;
+        __nv_bfloat16* dst = out + (int64_t(t) * H + i) * kDv + cb + c0;
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
           float x[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) x[j] = n_tiles > 0 ? __uint_as_float(v[e + j]) * inv : 0.f;
+          for (int j = 0; j < 8; ++j) x[j] = n_tiles > 0 ? __uint_as_float(o[e + j]) * inv : 0.f;
           *reinterpret_cast<uint4*>(dst + e) =
               make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
                          pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
         }
       }
     }
-    if (ok && t < T && lse)
-      lse[int64_t(t) * H + i] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f
+    if (h == 0 && ok && t < T && lse)
+      lse[int64_t(t) * H + i] = l_row > 0.f ? (m_run + __log2f(l_row)) * 0.69314718055994531f
                                             : -INFINITY;
   }
   __syncthreads();
@@ -571,9 +620,8 @@ cudaError_t launch_prefill(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_p
   __nv_bfloat16* v = reinterpret_cast<__nv_bfloat16*>(p);
   p += round1k(size_t(H) * L * 128 * 2);
   __half* kr = reinterpret_cast<__half*>(p);
-  const int64_t nq_units = int64_t(T) * H * (dq / 8);
-  const int qb = int((nq_units + 255) / 256 < 4096 ? (nq_units + 255) / 256 : 4096);
-  prefill_q_kernel<<<qb, 256, 0, stream>>>(q_nope, q_pe, q_pos, T, H, d_r, rope_base, q_full);
+  prefill_q_kernel<<<T, kQThreads, 0, stream>>>(q_nope, q_pe, q_pos, T, H, d_r, rope_base,
+                                                 q_full);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
@@ -597,7 +645,7 @@ cudaError_t launch_prefill(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_p
 
   if ((e = set_smem_once(prefill_attn_tc_kernel, kAtSmem)) != cudaSuccess) return e;
   const float scale_log2 = scale * 1.4426950408889634f;
-  prefill_attn_tc_kernel<<<dim3(H, unsigned((T + kTileQ - 1) / kTileQ)), kAtThreads, kAtSmem,
+  prefill_attn_tc_kernel<<<dim3(unsigned((T + kTileQ - 1) / kTileQ), H), kAtThreads, kAtSmem,
                            stream>>>(tm_q, tm_kc, tm_v, tm_kr, q_pos, T, L, H, d_r, scale_log2,
                                      out, lse, status);
   return cudaGetLastError();

@@ -461,6 +461,40 @@ def test_decode_step_streams_and_graph(w):
         assert torch.equal(l, outs[0][1])
 
 
+def test_host_pipeline_matches_step():
+    """DecodeStep.host_pipeline (inputs from pinned host memory, copies
+    overlapped with the previous step) returns, in host memory, exactly the
+    output of the plain step on the same inputs, for runs of 1, 2 and 5
+    steps (both graphs, and the prologue and epilogue copies)."""
+    w = W["v3_bf16"].scaled(B=3, N=300, append=True, hidden=512)
+    lens = inputs.seqlens(w)
+    d = dims_of(w)
+    qn, qp = inputs.query(w)
+    Wuk, Wuv = inputs.weights(w)
+    h, Wdkv = inputs.append_inputs(w)
+    cache = device_cache(w, lens)
+    seq0 = torch.from_numpy(lens).cuda()
+    seq = seq0.clone()
+    step = mla.DecodeStep(d, dev(Wuk, w), dev(Wuv, w), dev(Wdkv, w))
+    pos = torch.from_numpy(lens.astype(np.int32))
+    host = [dev(qn, w).cpu().pin_memory(), dev(qp, w).cpu().pin_memory(), pos.pin_memory(),
+            dev(h, w).cpu().pin_memory()]
+    step(*[t.cuda() for t in host[:3]], cache, seq, h=host[3].cuda())
+    seq.copy_(seq0)
+    torch.cuda.synchronize()
+    ref = step.out.cpu()
+    out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    pipe = step.host_pipeline(host, out, cache, seq, after=lambda: seq.copy_(seq0))
+    for n in (1, 2, 5):
+        out.zero_()
+        pipe.run(n)
+        torch.cuda.synchronize()
+        assert mla.get_device_status() == 0
+        assert torch.equal(out, ref)
+    assert pipe.bytes_per_step() == (sum(t.numel() * t.element_size() for t in host),
+                                     out.numel() * out.element_size())
+
+
 def _sample(w, n_seq, heads, seed=0):
     r = np.random.default_rng(seed)
     seqs = sorted(set([0, w.B - 1] + list(r.choice(w.B, size=min(n_seq, w.B), replace=False))))
