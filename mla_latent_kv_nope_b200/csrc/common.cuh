@@ -13,6 +13,34 @@ namespace mla {
 // kernel agree on this unit.
 constexpr int kTileKeys = 64;
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl may start
+// while the previous kernel in its stream is still running; pdl_wait() blocks
+// until that kernel has finished and its writes are visible, so every read of
+// a predecessor's output comes after it (without the launch attribute it
+// returns at once).  pdl_trigger() lets the next kernel be scheduled; it is
+// issued after the caller's own tensor-memory allocation, so a dependent
+// that holds tensor memory never waits on a primary that still needs some.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Device code records the first error it meets (bounds, timeout) in the
 // per-device status word whose address the host passes to the kernel;
 // mla_get_device_status reads and clears it.

@@ -77,6 +77,8 @@ append_finalize_kernel(const float* __restrict__ part, int n_parts,
                        const float* __restrict__ gamma, float eps, float rope_base, int d_c,
                        int d_r, int64_t cap, T* __restrict__ cache, const PageMap pm,
                        int32_t* __restrict__ seqlens, int* __restrict__ status) {
+  pdl_wait();   // the projection sums come from the kernel launched just before
+  pdl_trigger();
   const int b = blockIdx.x;
   const int B = gridDim.x;
   const int R = d_c + d_r;
@@ -148,6 +150,8 @@ append_finalize_fp8_kernel(const float* __restrict__ part, int n_parts,
                            int d_r, int64_t cap, uint8_t* __restrict__ cache,
                            float* __restrict__ scales, const PageMap pm,
                            int32_t* __restrict__ seqlens, int* __restrict__ status) {
+  pdl_wait();   // the projection sums come from the kernel launched just before
+  pdl_trigger();
   const int b = blockIdx.x;
   const int B = gridDim.x;
   const int R = d_c + d_r;
@@ -241,10 +245,9 @@ cudaError_t launch_append_finalize_fp8(const float* part, int n_parts, const flo
                                        cudaStream_t stream) {
   const size_t smem = sizeof(float) * size_t(d_c + d_r);
   const int threads = min(1024, (d_c + d_r + 31) / 32 * 32);
-  append_finalize_fp8_kernel<<<B, threads, smem, stream>>>(part, n_parts, gamma, eps, rope_base,
-                                                           d_c, d_r, cap, cache, scales, pm,
-                                                           seqlens, status);
-  return cudaGetLastError();
+  return launch_pdl(append_finalize_fp8_kernel, dim3(B), dim3(threads), smem, stream, part,
+                    n_parts, gamma, eps, rope_base, d_c, d_r, cap, cache, scales, pm, seqlens,
+                    status);
 }
 
 template <typename T>
@@ -268,10 +271,8 @@ cudaError_t launch_append_finalize(const float* part, int n_parts, const float* 
                                    cudaStream_t stream) {
   const size_t smem = sizeof(float) * size_t(d_c + d_r);
   const int threads = min(1024, (d_c + d_r + 31) / 32 * 32);
-  append_finalize_kernel<T><<<B, threads, smem, stream>>>(part, n_parts, gamma, eps, rope_base,
-                                                             d_c, d_r, cap, cache, pm, seqlens,
-                                                             status);
-  return cudaGetLastError();
+  return launch_pdl(append_finalize_kernel<T>, dim3(B), dim3(threads), smem, stream, part,
+                    n_parts, gamma, eps, rope_base, d_c, d_r, cap, cache, pm, seqlens, status);
 }
 
 template cudaError_t launch_append_finalize<float>(const float*, int, const float*, float, float,

@@ -171,6 +171,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
 
   // Tile prefix of the batch (all threads load lengths in parallel; warp 0
   // scans 32 at a time with shuffles).
+  pdl_wait();   // lengths, queries and the appended rows come from earlier kernels
   TilePrefix tp;
   const int64_t n_tiles = build_tile_prefix(smem + kOffPrefix, seqlens, B, cap, &tp);
   if (n_tiles == 0) return;
@@ -212,6 +213,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
   uint32_t n_issued = 0;   // loads issued by the producer (lane 0 of its warp)
@@ -686,10 +688,9 @@ cudaError_t launch_decode_tc_t(const CUtensorMap& tm_c, const CUtensorMap& tm_co
   }
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(decode_tc_head_groups(H), W);
-  decode_tc_kernel<kDr, kFp8><<<grid, Threads<kFp8>::n, kSmemBytes, stream>>>(
-      tm_c, tm_codes, static_cast<const __nv_bfloat16*>(cache), scales, pm, q_cat, seqlens, B, H,
-      cap, scale_log2, W, o_part, lse_part, status, inject_wait);
-  return cudaGetLastError();
+  return launch_pdl(decode_tc_kernel<kDr, kFp8>, grid, dim3(Threads<kFp8>::n), kSmemBytes, stream,
+                    tm_c, tm_codes, static_cast<const __nv_bfloat16*>(cache), scales, pm, q_cat,
+                    seqlens, B, H, cap, scale_log2, W, o_part, lse_part, status, inject_wait);
 }
 
 // Byte map over FP8 cache rows [rows, 640]: boxes of 128 codes x 64 rows,

@@ -85,6 +85,9 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __rest
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tbase;
+  // The weight block is already on its way; o_lat comes from the combine.
+  pdl_wait();
+  pdl_trigger();
   bool ok = true;
   constexpr uint32_t idesc = idesc_bf16_f32(128, kOpN, false, false);
   int pass = 0;
@@ -348,6 +351,7 @@ append_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_con
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();   // the finalize may be scheduled; it waits for this grid's sums
   const uint32_t tmem = *tbase;
   bool ok = block_wait(&bars[0], 0);
   if (warp == 0) {
@@ -445,8 +449,8 @@ cudaError_t launch_out_proj_tc(const float* o_lat, const __nv_bfloat16* W_UV, in
   if (!make_map(&tm, W_UV, uint64_t(H) * 128, 512, 128)) return cudaErrorInvalidValue;
   cudaError_t e = set_smem(out_proj_tc_kernel, kOpSmem);
   if (e != cudaSuccess) return e;
-  out_proj_tc_kernel<<<H, kThreadsG, kOpSmem, stream>>>(tm, o_lat, B, H, out, status);
-  return cudaGetLastError();
+  return launch_pdl(out_proj_tc_kernel, dim3(H), dim3(kThreadsG), kOpSmem, stream, tm, o_lat, B,
+                    H, out, status);
 }
 
 cudaError_t launch_absorb_q_tc(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_pe,

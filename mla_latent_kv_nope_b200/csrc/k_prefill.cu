@@ -89,6 +89,7 @@ prefill_q_kernel(const __nv_bfloat16* __restrict__ q_nope, const __nv_bfloat16* 
                  const int32_t* __restrict__ q_pos, int T, int H, int d_r, float rope_base,
                  __half* __restrict__ q_full) {
   __shared__ float s_cos[32], s_sin[32];
+  pdl_trigger();   // the K/V projection does not read the queries: let it start
   const int t = blockIdx.x;
   const int half = d_r / 2;
   if (threadIdx.x < half) {
@@ -168,6 +169,7 @@ prefill_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_rows,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_trigger();
   const uint32_t tmem = *tbase;
   volatile int* abort_flag = &s_abort;
   bool ok = true;
@@ -259,6 +261,10 @@ prefill_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_rows,
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
+  // This kernel reads only inputs and may run beside the query kernel before
+  // it; it finishes only after that kernel, so the attention kernel, which
+  // waits for this one, also sees the rotated queries.
+  pdl_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -322,6 +328,7 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nq = (kDn + d_r) / 64;                       // 64-wide chunks of the head dim
   volatile int* abort_flag = &bars->abort_flag;
+  pdl_wait();   // queries, K^C, V and k^R come from the two kernels before
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < kAtStages; ++s) {
@@ -639,16 +646,16 @@ cudaError_t launch_prefill(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_p
     return cudaErrorInvalidValue;
 
   if ((e = set_smem_once(prefill_kv_tc_kernel, kKvSmem)) != cudaSuccess) return e;
-  prefill_kv_tc_kernel<<<dim3(unsigned((L + 127) / 128), H), kKvThreads, kKvSmem, stream>>>(
-      tm_rows, tm_wuk, tm_wuv, L, H, d_r, rows, kc, v, kr, status);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_pdl(prefill_kv_tc_kernel, dim3(unsigned((L + 127) / 128), H), dim3(kKvThreads),
+                      kKvSmem, stream, tm_rows, tm_wuk, tm_wuv, L, H, d_r, rows, kc, v, kr,
+                      status)) != cudaSuccess)
+    return e;
 
   if ((e = set_smem_once(prefill_attn_tc_kernel, kAtSmem)) != cudaSuccess) return e;
   const float scale_log2 = scale * 1.4426950408889634f;
-  prefill_attn_tc_kernel<<<dim3(unsigned((T + kTileQ - 1) / kTileQ), H), kAtThreads, kAtSmem,
-                           stream>>>(tm_q, tm_kc, tm_v, tm_kr, q_pos, T, L, H, d_r, scale_log2,
-                                     out, lse, status);
-  return cudaGetLastError();
+  return launch_pdl(prefill_attn_tc_kernel, dim3(unsigned((T + kTileQ - 1) / kTileQ), H),
+                    dim3(kAtThreads), kAtSmem, stream, tm_q, tm_kc, tm_v, tm_kr, q_pos, T, L, H,
+                    d_r, scale_log2, out, lse, status);
 }
 
 }  // namespace mla
