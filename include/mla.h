@@ -202,8 +202,10 @@ MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W
  * d_v and dtype are read.  Shape: bf16, d_c = 512, d_nope = d_v = 128, d_r =
  * 64 or 0, H * L and H * T below 2^31, L >= 1 (T = 0 does nothing).  The
  * workspace (mla_prefill_workspace_bytes, no initialisation needed) holds the
- * rotated queries and the materialised K^C and V: about 2 * H * (T * (d_nope
- * + d_r) + 2 * L * 128) bytes. */
+ * materialised K^C and V and a 16-bit copy of k^R: about 4 * H * L * 128 +
+ * 2 * L * d_r bytes.  Precision: the QK^T operands (queries, K^C, k^R) are
+ * rounded to fp16 and P, V to bf16, with fp32 accumulation, so queries and
+ * keys must lie within fp16's range (|x| < 65504). */
 MLA_API size_t mla_prefill_workspace_bytes(const mla_dims* dims, int32_t T, int64_t L);
 MLA_API int mla_prefill(const mla_dims* dims, int32_t T, int64_t L, const void* q_nope,
                         const void* q_pe, const int32_t* q_pos, const void* W_UK,

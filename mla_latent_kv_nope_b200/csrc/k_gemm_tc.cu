@@ -69,6 +69,9 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __rest
   uint32_t* tbase = reinterpret_cast<uint32_t*>(bars + 2);
   const int i = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Nothing is read before the kernel in front (the combine) has finished:
+  // the weight could have been written by stream work before this call too.
+  pdl_wait();
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
@@ -84,10 +87,8 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __rest
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tbase;
-  // The weight block is already on its way; o_lat comes from the combine.
-  pdl_wait();
   pdl_trigger();
+  const uint32_t tmem = *tbase;
   bool ok = true;
   constexpr uint32_t idesc = idesc_bf16_f32(128, kOpN, false, false);
   int pass = 0;

@@ -3,8 +3,6 @@
 // explicitly and the heads run ordinary causal attention; the absorbed form is
 // the decode's).
 //
-//   prefill_q_kernel      Q_i[t] = [q^C[t,i] ; RoPE(q^R[t,i], q_pos[t])]
-//                         -> q_full [H, T, 128 + d_r] fp16
 //   prefill_kv_tc_kernel  K^C_i[l] = W^UK_i c_l,  V_i[l] = W^UV_i c_l
 //                         -> kc [H, L, 128] fp16, v [H, L, 128] bf16, and
 //                         kr [L, d_r] fp16 (the rows' k^R, converted once)
@@ -12,9 +10,11 @@
 //                         (K-major, K = d_c = 512), B = [W^UK_i ; W^UV_i]
 //                         (256 rows, K-major), D [128 x 256] fp32 in TMEM
 //   prefill_attn_tc_kernel  causal softmax attention of head i, 128 queries
-//                         per CTA, 128-key tiles; the key of row l is
-//                         [K^C_i[l] ; k^R_l] (k^R read from the latent rows,
-//                         already rotated), head dim 128 + d_r, value dim 128
+//                         per CTA, 128-key tiles; the query row is
+//                         Q_i[t] = [q^C[t,i] ; RoPE(q^R[t,i], q_pos[t])], formed
+//                         by the CTA straight into tensor memory; the key of
+//                         row l is [K^C_i[l] ; k^R_l] (k^R already rotated),
+//                         head dim 128 + d_r, value dim 128
 //
 // The causal rule: query t sees rows l <= q_pos[t] (clamped to L - 1); a
 // query with q_pos[t] < 0 sees nothing (out 0, lse -inf).
@@ -79,51 +79,20 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------------------
-// Queries: one block per token t.  The rotation angles depend on (t, pair)
-// only, so the block forms the d_r/2 (cos, sin) pairs once and every head
-// uses them; each thread then writes 16-byte units of the H rows.
-constexpr int kQThreads = 256;
-
-__global__ void __launch_bounds__(kQThreads)
-prefill_q_kernel(const __nv_bfloat16* __restrict__ q_nope, const __nv_bfloat16* __restrict__ q_pe,
-                 const int32_t* __restrict__ q_pos, int T, int H, int d_r, float rope_base,
-                 __half* __restrict__ q_full) {
-  __shared__ float s_cos[32], s_sin[32];
-  pdl_trigger();   // the K/V projection does not read the queries: let it start
-  const int t = blockIdx.x;
+// RoPE angles of the queries: cs[t][k] = (cos, sin) of q_pos[t] * base^(-2k/d_r)
+// for the d_r/2 pairs, formed once per token (every head uses them).
+__global__ void prefill_rope_table_kernel(const int32_t* __restrict__ q_pos, int T, int d_r,
+                                          float rope_base, float2* __restrict__ cs) {
+  pdl_trigger();   // the K/V projection does not read the table: let it start
   const int half = d_r / 2;
-  if (threadIdx.x < half) {
+  const int64_t n = int64_t(T) * half;
+  for (int64_t u = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; u < n;
+       u += int64_t(gridDim.x) * blockDim.x) {
+    const int t = int(u / half), k = int(u % half);
     const int32_t pos = q_pos[t];
-    rope_cos_sin(pos < 0 ? 0 : pos, threadIdx.x, d_r, rope_base, &s_cos[threadIdx.x],
-                 &s_sin[threadIdx.x]);
-  }
-  __syncthreads();
-  const int dq = kDn + d_r;
-  const int units = dq / 8;
-  for (int k = threadIdx.x; k < H * units; k += kQThreads) {
-    const int u = k % units, i = k / units;
-    const int64_t ti = int64_t(t) * H + i;
-    uint4 v;
-    if (u < kDn / 8) {
-      v = bf16x8_to_f16x8(*reinterpret_cast<const uint4*>(q_nope + ti * kDn + u * 8));
-    } else {
-      // Output dims e0 .. e0+7 of the RoPE block: pairs (k, k + d_r/2).
-      const int e0 = (u - kDn / 8) * 8;
-      const bool upper = e0 >= half;
-      const int k0 = upper ? e0 - half : e0;
-      const __nv_bfloat16* src = q_pe + ti * d_r;
-      float y[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float x1 = __bfloat162float(src[k0 + j]);
-        const float x2 = __bfloat162float(src[k0 + j + half]);
-        const float c = s_cos[k0 + j], sn = s_sin[k0 + j];
-        y[j] = upper ? x1 * sn + x2 * c : x1 * c - x2 * sn;
-      }
-      v = make_uint4(pack_f16x2(y[0], y[1]), pack_f16x2(y[2], y[3]), pack_f16x2(y[4], y[5]),
-                     pack_f16x2(y[6], y[7]));
-    }
-    *reinterpret_cast<uint4*>(q_full + (int64_t(i) * T + t) * dq + u * 8) = v;
+    float c, sn;
+    rope_cos_sin(pos < 0 ? 0 : pos, k, d_r, rope_base, &c, &sn);
+    cs[u] = make_float2(c, sn);
   }
 }
 
@@ -261,34 +230,37 @@ prefill_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_rows,
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
-  // This kernel reads only inputs and may run beside the query kernel before
-  // it; it finishes only after that kernel, so the attention kernel, which
-  // waits for this one, also sees the rotated queries.
-  pdl_wait();
+  pdl_wait();   // the kernel before (the query angles) has finished too
 }
 
 // ---------------------------------------------------------------------------
-// Causal attention.  smem: Q 3 x [128 x 128 B] | 2 stages x (K 3 x [128 x 128 B]
-// | V 2 x [128 x 128 B]) | barriers.  Tensor memory (512 columns): O [128 x
-// 128] fp32 at 0, S double buffer 2 x 128 at 128, P (bf16 pairs) 2 x 64 at 384.
-constexpr int kAtStages = 2;
-// Warps 0-7 softmax + epilogue (warp w: rows 32 (w % 4) .., key/value
-// columns 64 (w / 4) ..: two threads per query row), 8 TMA, 9 MMA.
+// Causal attention: one CTA per (128 queries, head).
+// Tensor memory (512 columns): O [128 x 128] fp32 at 0; S double buffer
+// 2 x 128 at 128, whose first 64 columns receive P (bf16 pairs) once both
+// threads of a row have read their S; Q (fp16 pairs: 96 columns, 64 without
+// RoPE) at 384, the tensor-memory A operand of QK^T.  Shared memory: a
+// 3-stage K ring (K^C boxes and the k^R box of 128 keys) and a 2-stage V ring,
+// with separate barriers, so a K stage is refilled as soon as its QK^T is
+// done and the load of key tile k + 3 overlaps tiles k + 1 and k + 2.
+// Warps 0-7: query rows into tensor memory, softmax, epilogue (warp w: rows
+// 32 (w % 4) .., columns 64 (w / 4) .. of S, P and O, so two threads per
+// row); warp 8: K loads; warp 9: MMA issue; warp 10: V loads.
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kKStage = 3 * kBox;                         // 48 KB
+constexpr int kVStage = 2 * kBox;                         // 32 KB
 constexpr int kAtSoftmaxThreads = 256;
-constexpr int kAtThreads = 320;
-constexpr int kAtProducer = 8;
+constexpr int kAtKLoad = 8;
 constexpr int kAtMma = 9;
-constexpr int kQBytes = 3 * kBox;
-constexpr int kKBytes = 3 * kBox;
-constexpr int kVBytes = 2 * kBox;
-constexpr int kAtStage = kKBytes + kVBytes;                // 80 KB
-constexpr uint32_t kColO = 0, kColS = 128, kColP = 384;
+constexpr int kAtVLoad = 10;
+constexpr int kAtThreads = 352;
+constexpr uint32_t kColO = 0, kColS = 128, kColQ = 384;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by > 2^8
 
 struct AttnBars {
-  uint64_t q_full;
-  uint64_t full[kAtStages], empty[kAtStages];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t q_ready, s_full[2], p_full[2], pv_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -296,7 +268,8 @@ struct AttnBars {
   float row_max[2][2][kTileQ];   // [tile parity][column half][row]: the halves' maxima
   float row_sum[2][kTileQ];      // [column half][row]: the halves' sums, at the end
 };
-constexpr size_t kAtSmem = size_t(kQBytes) + kAtStages * kAtStage + sizeof(AttnBars) + 1024;
+constexpr size_t kAtSmem =
+    size_t(kKStages) * kKStage + size_t(kVStages) * kVStage + sizeof(AttnBars) + 1024;
 static_assert(kAtSmem <= 232448, "shared memory budget of one CTA");
 
 // Warp-uniform bounded wait that also gives up when another role aborted.
@@ -307,19 +280,79 @@ __device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// One arrival per warp on a barrier that counts warps: every lane's tensor-
+// memory stores are complete and ordered before lane 0 arrives.
+__device__ __forceinline__ void warp_arrive_after_tmem_st(uint64_t* bar) {
+  tmem_wait_st();
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// Query row t of head i, fp16 dims [32 j, 32 j + 32) as 16 packed columns:
+// q^C for j < 4, then RoPE(q^R, pos) (pairs (k, k + d_r/2)).  Rows past T are zero.
+__device__ __forceinline__ void query_chunk(const __nv_bfloat16* __restrict__ q_nope,
+                                            const __nv_bfloat16* __restrict__ q_pe, bool valid,
+                                            int64_t row, int d_r, int j,
+                                            const float2* __restrict__ cs_row, uint32_t (&out)[16]) {
+  if (!valid) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) out[e] = 0u;
+    return;
+  }
+  if (j < kDn / 32) {
+    const uint4* src = reinterpret_cast<const uint4*>(q_nope + row * kDn + 32 * j);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint4 h = bf16x8_to_f16x8(src[u]);
+      out[4 * u] = h.x;
+      out[4 * u + 1] = h.y;
+      out[4 * u + 2] = h.z;
+      out[4 * u + 3] = h.w;
+    }
+    return;
+  }
+  // RoPE chunk: the whole q^R row (64 bf16) and the 32 angle pairs come in
+  // with 16-byte loads; output dims e0 .. e0 + 31 of the rotated block.
+  const int e0 = 32 * (j - kDn / 32);
+  const bool upper = e0 >= 32;               // d_r = 64: dims 32..63 are the k + 32 halves
+  float x[64];
+  const uint4* src = reinterpret_cast<const uint4*>(q_pe + row * d_r);
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const uint4 w = src[u];
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(p2[q]);
+      x[8 * u + 2 * q] = f.x;
+      x[8 * u + 2 * q + 1] = f.y;
+    }
+  }
+  const float4* cs4 = reinterpret_cast<const float4*>(cs_row);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float4 a = cs4[e / 2];               // (cos, sin) of pairs e and e + 1
+    const float y0 = upper ? x[e] * a.y + x[e + 32] * a.x : x[e] * a.x - x[e + 32] * a.y;
+    const float y1 = upper ? x[e + 1] * a.w + x[e + 33] * a.z : x[e + 1] * a.z - x[e + 33] * a.w;
+    out[e / 2] = pack_f16x2(y0, y1);
+  }
+}
+
 __global__ void __launch_bounds__(kAtThreads, 1)
-prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_kc,
+prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc,
                        const __grid_constant__ CUtensorMap tm_v,
                        const __grid_constant__ CUtensorMap tm_kr,
+                       const __nv_bfloat16* __restrict__ q_nope,
+                       const __nv_bfloat16* __restrict__ q_pe, const float2* __restrict__ cs,
                        const int32_t* __restrict__ q_pos, int T, int64_t L, int H, int d_r,
-                       float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                       int* __restrict__ status) {
+                       float scale_log2, __nv_bfloat16* __restrict__ out,
+                       float* __restrict__ lse, int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  uint8_t* sQ = sm;
-  uint8_t* sStage = sm + kQBytes;
-  AttnBars* bars = reinterpret_cast<AttnBars*>(sStage + kAtStages * kAtStage);
+  uint8_t* sK = sm;
+  uint8_t* sV = sm + kKStages * kKStage;
+  AttnBars* bars = reinterpret_cast<AttnBars*>(sV + kVStages * kVStage);
   // Query tiles vary fastest, so the CTAs in flight share a few heads' K and
   // V through L2; within a head the longest query tiles start first.
   const int i = blockIdx.y;
@@ -328,16 +361,20 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nq = (kDn + d_r) / 64;                       // 64-wide chunks of the head dim
   volatile int* abort_flag = &bars->abort_flag;
-  pdl_wait();   // queries, K^C, V and k^R come from the two kernels before
+  pdl_wait();   // K^C, V, k^R and the query angles come from the kernels before
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kAtStages; ++s) {
-      mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->empty[s], 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
     }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    mbar_init(&bars->q_ready, kAtSoftmaxThreads / 32);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], kAtSoftmaxThreads);
+      mbar_init(&bars->p_full[b], kAtSoftmaxThreads / 32);
       mbar_init(&bars->pv_done[b], 1);
     }
     mbar_init(&bars->drain, 1);
@@ -353,9 +390,10 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   // Rows this CTA's queries may see: vis = min(q_pos + 1, L), 0 past T or
   // for a negative position.
   int64_t vis = 0;
+  int32_t pos = 0;
   if (threadIdx.x < kAtSoftmaxThreads) {
     const int t = q0 + (threadIdx.x & (kTileQ - 1));
-    const int32_t pos = t < T ? q_pos[t] : -1;
+    pos = t < T ? q_pos[t] : -1;
     vis = pos < 0 ? 0 : (int64_t(pos) + 1 < L ? int64_t(pos) + 1 : L);
   }
   tc_fence_before();
@@ -367,70 +405,76 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int n_tiles = int((int64_t(bars->max_vis) + kTileK - 1) / kTileK);
   bool ok = true;
 
-  if (warp == kAtProducer) {
+  if (warp == kAtKLoad || warp == kAtVLoad) {
     // ---------------------------------------------------------------- TMA
+    const bool is_k = warp == kAtKLoad;
+    const int stages = is_k ? kKStages : kVStages;
+    uint64_t* full = is_k ? bars->k_full : bars->v_full;
+    uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
     int issued = 0;
     if (lane == 0 && n_tiles > 0) {
-      mbar_arrive_expect_tx(&bars->q_full, uint32_t(nq * kBox));
-      for (int c = 0; c < nq; ++c)
-        tma_load_2d(&tm_q, &bars->q_full, sQ + c * kBox, c * 64, int32_t(int64_t(i) * T + q0));
       for (int k = 0; k < n_tiles; ++k) {
-        const int s = k % kAtStages;
-        if (k >= kAtStages &&
-            !(ok = mbar_wait(&bars->empty[s], ((k / kAtStages) - 1) & 1, abort_flag,
-                             kWaitLimitCycles)))
+        const int s = k % stages;
+        if (k >= stages &&
+            !(ok = mbar_wait(&empty[s], ((k / stages) - 1) & 1, abort_flag, kWaitLimitCycles)))
           break;
-        uint8_t* st = sStage + s * kAtStage;
         const int32_t row = int32_t(int64_t(i) * L + int64_t(k) * kTileK);
-        mbar_arrive_expect_tx(&bars->full[s], uint32_t((nq + 2) * kBox));
-        tma_load_2d(&tm_kc, &bars->full[s], st, 0, row);
-        tma_load_2d(&tm_kc, &bars->full[s], st + kBox, 64, row);
-        if (d_r) tma_load_2d(&tm_kr, &bars->full[s], st + 2 * kBox, 0, k * kTileK);
-        tma_load_2d(&tm_v, &bars->full[s], st + kKBytes, 0, row);
-        tma_load_2d(&tm_v, &bars->full[s], st + kKBytes + kBox, 64, row);
+        if (is_k) {
+          uint8_t* st = sK + s * kKStage;
+          mbar_arrive_expect_tx(&full[s], uint32_t(nq * kBox));
+          tma_load_2d(&tm_kc, &full[s], st, 0, row);
+          tma_load_2d(&tm_kc, &full[s], st + kBox, 64, row);
+          if (d_r) tma_load_2d(&tm_kr, &full[s], st + 2 * kBox, 0, k * kTileK);
+        } else {
+          uint8_t* st = sV + s * kVStage;
+          mbar_arrive_expect_tx(&full[s], uint32_t(2 * kBox));
+          tma_load_2d(&tm_v, &full[s], st, 0, row);
+          tma_load_2d(&tm_v, &full[s], st + kBox, 64, row);
+        }
         ++issued;
       }
       if (!ok) *abort_flag = 1;
       // Every issued load lands before the shared memory is released.
-      wait_bar(&bars->q_full, 0);
-      for (int k = issued > kAtStages ? issued - kAtStages : 0; k < issued; ++k)
-        wait_bar(&bars->full[k % kAtStages], (k / kAtStages) & 1);
+      for (int k = issued > stages ? issued - stages : 0; k < issued; ++k)
+        wait_bar(&full[k % stages], (k / stages) & 1);
     }
   } else if (warp == kAtMma) {
     // ---------------------------------------------------------------- MMA
     if (n_tiles > 0) {
+      // kind::f16 MMAs: the instruction descriptor names the operand type (fp16 for
+      // QK^T, bf16 for P.V).
       constexpr uint32_t idesc_qk = idesc_f16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
-      ok = warp_wait_bar(&bars->q_full, 0, abort_flag);
+      ok = warp_wait_bar(&bars->q_ready, 0, abort_flag);
       auto issue_pv = [&](int j) -> bool {
-        const int b = j & 1;
+        const int b = j & 1, sv = j % kVStages;
         if (!warp_wait_bar(&bars->p_full[b], (j >> 1) & 1, abort_flag)) return false;
+        if (!warp_wait_bar(&bars->v_full[sv], (j / kVStages) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint64_t v0 = smem_desc_sw128(smem_u32(sStage + (j % kAtStages) * kAtStage + kKBytes),
-                                            kBox, 1024);
+        const uint64_t v0 = smem_desc_sw128(smem_u32(sV + sv * kVStage), kBox, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk)
-          mma_bf16_ts_w(tmem + kColO, tmem + kColP + uint32_t(b * 64 + kk * 8),
+          mma_bf16_ts_w(tmem + kColO, tmem + kColS + uint32_t(b * 128 + kk * 8),
                         v0 + uint64_t((kk * 2048) >> 4), idesc_pv, j > 0 || kk > 0);
         mma_commit_w(&bars->pv_done[b]);
-        mma_commit_w(&bars->empty[j % kAtStages]);
+        mma_commit_w(&bars->v_empty[sv]);
         return true;
       };
       for (int k = 0; ok && k < n_tiles; ++k) {
-        const int s = k % kAtStages;
-        if (!(ok = warp_wait_bar(&bars->full[s], (k / kAtStages) & 1, abort_flag))) break;
+        const int sk = k % kKStages;
+        if (!(ok = warp_wait_bar(&bars->k_full[sk], (k / kKStages) & 1, abort_flag))) break;
         tc_fence_after();
-        const uint32_t sk = smem_u32(sStage + s * kAtStage);
+        const uint32_t kb = smem_u32(sK + sk * kKStage);
         const uint32_t d = tmem + kColS + uint32_t((k & 1) * 128);
         for (int c = 0; c < nq; ++c) {
-          const uint64_t a0 = smem_desc_sw128(smem_u32(sQ + c * kBox), 16, 1024);
-          const uint64_t b0 = smem_desc_sw128(sk + uint32_t(c * kBox), 16, 1024);
+          const uint64_t b0 = smem_desc_sw128(kb + uint32_t(c * kBox), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss_w(d, a0 + uint64_t((kk * 32) >> 4), b0 + uint64_t((kk * 32) >> 4),
-                          idesc_qk, (c | kk) != 0);
+            mma_bf16_ts_w(d, tmem + kColQ + uint32_t(c * 32 + kk * 8),
+                         b0 + uint64_t((kk * 32) >> 4), idesc_qk, (c | kk) != 0);
         }
         mma_commit_w(&bars->s_full[k & 1]);
+        mma_commit_w(&bars->k_empty[sk]);
         if (k >= 1 && !(ok = issue_pv(k - 1))) break;
       }
       if (ok) ok = issue_pv(n_tiles - 1);
@@ -440,7 +484,7 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     mma_commit_w(&bars->drain);
     if (lane == 0) wait_bar(&bars->drain, 0);
     __syncwarp();
-  } else {
+  } else if (warp < kAtSoftmaxThreads / 32) {
     // ---------------------------------------------------------------- softmax
     // Thread (warp w, lane) owns row r = 32 (w % 4) + lane, columns
     // [64 h, 64 h + 64) with h = w / 4, of S, P and O.  The two halves of a row
@@ -451,6 +495,18 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int r = 32 * quad + lane;
     const uint32_t lane_base = uint32_t(32 * quad) << 16;
     const int cb = 64 * h;
+    // The query row into tensor memory: this half writes chunks [nc/2 h, nc/2 (h+1)).
+    {
+      const int t = q0 + r;
+      const int nc = (kDn + d_r) / 32;
+      const int64_t row = int64_t(t) * H + i;
+      for (int j = h * nc / 2; j < (h + 1) * nc / 2; ++j) {
+        uint32_t v[16];
+        query_chunk(q_nope, q_pe, t < T, row, d_r, j, cs + int64_t(t < T ? t : 0) * (d_r / 2), v);
+        tmem_st16(tmem + lane_base + kColQ + uint32_t(16 * j), v);
+      }
+      warp_arrive_after_tmem_st(&bars->q_ready);
+    }
     float m_run = -INFINITY, l_run = 0.f;
     // Both halves of a row run every iteration up to the named barrier, even
     // after a give-up (then with no work), so the barrier never waits for a
@@ -461,13 +517,13 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (ok) ok = warp_wait_bar(&bars->s_full[b], (k >> 1) & 1, abort_flag);
       const int64_t nv = vis - int64_t(k) * kTileK - cb;   // visible columns of this half
       const int nvalid = nv <= 0 ? 0 : (nv >= 64 ? 64 : int(nv));
+      const uint32_t s_addr = tmem + lane_base + kColS + uint32_t(b * 128);
       uint32_t va[32], vb[32];
       float mt = -INFINITY;
       if (ok) {
         tc_fence_after();
-        const uint32_t s_addr = tmem + lane_base + kColS + uint32_t(b * 128 + cb);
-        tmem_ld32(s_addr, va);
-        tmem_ld32(s_addr + 32, vb);
+        tmem_ld32(s_addr + uint32_t(cb), va);
+        tmem_ld32(s_addr + uint32_t(cb + 32), vb);
         tmem_wait_ld();
         if (nvalid == 64) {
 #pragma unroll
@@ -482,6 +538,8 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
       bars->row_max[b][h][r] = mt;
+      // Both halves have their S in registers past this barrier, so P may
+      // overwrite the S columns.
       asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
       if (!ok) continue;
       mt = fmaxf(mt, bars->row_max[b][1 - h][r]);
@@ -510,10 +568,6 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
       if (m_run == -INFINITY) m_run = m_new;
-      // P buffer b was last read by the product of tile k - 2.
-      if (k >= 2 && !(ok = warp_wait_bar(&bars->pv_done[b], ((k - 2) >> 1) & 1, abort_flag)))
-        continue;
-      tc_fence_after();
       const float mu = m_run == -INFINITY ? 0.f : m_run;
       float sum = 0.f;
       uint32_t pa[16], pb[16];
@@ -533,13 +587,11 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
         pa[e / 2] = pack_bf16x2(p0, p1);
         pb[e / 2] = pack_bf16x2(p2, p3);
       }
-      const uint32_t p_addr = tmem + lane_base + kColP + uint32_t(b * 64 + cb / 2);
-      tmem_st16(p_addr, pa);
-      tmem_st16(p_addr + 16, pb);
-      tmem_wait_st();
+      // P of keys [64 h, 64 h + 64) into columns [32 h, 32 h + 32) of the S buffer.
+      tmem_st16(s_addr + uint32_t(cb / 2), pa);
+      tmem_st16(s_addr + uint32_t(cb / 2 + 16), pb);
       l_run += sum;
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[b]);
+      warp_arrive_after_tmem_st(&bars->p_full[b]);
     }
     if (!ok) {
       bars->abort_flag = 1;
@@ -605,8 +657,8 @@ size_t round1k(size_t x) { return (x + 1023) / 1024 * 1024; }
 }  // namespace
 
 size_t prefill_workspace_bytes(int T, int64_t L, int H, int d_r) {
-  return round1k(size_t(H) * T * (kDn + d_r) * 2) + 2 * round1k(size_t(H) * L * 128 * 2) +
-         round1k(size_t(L) * d_r * 2);
+  return 2 * round1k(size_t(H) * L * 128 * 2) + round1k(size_t(L) * d_r * 2) +
+         round1k(size_t(T) * (d_r / 2) * 8);
 }
 
 cudaError_t launch_prefill(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_pe,
@@ -615,28 +667,22 @@ cudaError_t launch_prefill(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_p
                            int H, int d_r, float scale, float rope_base, __nv_bfloat16* out,
                            float* lse, void* workspace, int* status, cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
-  const int dq = kDn + d_r;
   const int R = kDcP + d_r;
-  // Workspace: q_full [H, T, dq] fp16 | kc [H, L, 128] fp16 | v [H, L, 128]
-  // bf16 | kr [L, d_r] fp16, each rounded up to 1 KB.
+  // Workspace: kc [H, L, 128] fp16 | v [H, L, 128] bf16 | kr [L, d_r] fp16 |
+  // cs [T, d_r/2] float2, each rounded up to 1 KB.
   uint8_t* p = static_cast<uint8_t*>(workspace);
-  __half* q_full = reinterpret_cast<__half*>(p);
-  p += round1k(size_t(H) * T * dq * 2);
   __half* kc = reinterpret_cast<__half*>(p);
   p += round1k(size_t(H) * L * 128 * 2);
   __nv_bfloat16* v = reinterpret_cast<__nv_bfloat16*>(p);
   p += round1k(size_t(H) * L * 128 * 2);
   __half* kr = reinterpret_cast<__half*>(p);
-  prefill_q_kernel<<<T, kQThreads, 0, stream>>>(q_nope, q_pe, q_pos, T, H, d_r, rope_base,
-                                                 q_full);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  p += round1k(size_t(L) * d_r * 2);
+  float2* cs = reinterpret_cast<float2*>(p);
 
-  CUtensorMap tm_rows, tm_wuk, tm_wuv, tm_q, tm_kc, tm_v, tm_kr;
+  CUtensorMap tm_rows, tm_wuk, tm_wuv, tm_kc, tm_v, tm_kr;
   if (!make_map16(&tm_rows, rows, uint64_t(L), uint64_t(R), uint64_t(R), 128) ||
       !make_map16(&tm_wuk, W_UK, uint64_t(H) * 128, kDcP, kDcP, 128) ||
       !make_map16(&tm_wuv, W_UV, uint64_t(H) * 128, kDcP, kDcP, 128) ||
-      !make_map16(&tm_q, q_full, uint64_t(H) * T, uint64_t(dq), uint64_t(dq), 128) ||
       !make_map16(&tm_kc, kc, uint64_t(H) * L, 128, 128, 128) ||
       !make_map16(&tm_v, v, uint64_t(H) * L, 128, 128, 128))
     return cudaErrorInvalidValue;
@@ -645,17 +691,36 @@ cudaError_t launch_prefill(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_p
             : make_map16(&tm_kr, kc, uint64_t(H) * L, 128, 128, 128)))
     return cudaErrorInvalidValue;
 
+  cudaError_t e;
+  if (d_r) {
+    const int64_t n = int64_t(T) * (d_r / 2);
+    prefill_rope_table_kernel<<<int((n + 255) / 256 < 2048 ? (n + 255) / 256 : 2048), 256, 0,
+                                stream>>>(q_pos, T, d_r, rope_base, cs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // With RoPE the projection may start beside the angle kernel: that kernel
+  // itself started only after all earlier work in the stream, and the
+  // projection reads only inputs.  It waits for the angle kernel before it
+  // finishes, so the attention kernel, which waits for the projection, sees
+  // the table.  Without RoPE it is an ordinary launch.
   if ((e = set_smem_once(prefill_kv_tc_kernel, kKvSmem)) != cudaSuccess) return e;
-  if ((e = launch_pdl(prefill_kv_tc_kernel, dim3(unsigned((L + 127) / 128), H), dim3(kKvThreads),
-                      kKvSmem, stream, tm_rows, tm_wuk, tm_wuv, L, H, d_r, rows, kc, v, kr,
-                      status)) != cudaSuccess)
-    return e;
+  const dim3 kv_grid(unsigned((L + 127) / 128), H);
+  if (d_r) {
+    e = launch_pdl(prefill_kv_tc_kernel, kv_grid, dim3(kKvThreads), kKvSmem, stream, tm_rows,
+                   tm_wuk, tm_wuv, L, H, d_r, rows, kc, v, kr, status);
+  } else {
+    prefill_kv_tc_kernel<<<kv_grid, kKvThreads, kKvSmem, stream>>>(tm_rows, tm_wuk, tm_wuv, L, H,
+                                                                   d_r, rows, kc, v, kr, status);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return e;
 
   if ((e = set_smem_once(prefill_attn_tc_kernel, kAtSmem)) != cudaSuccess) return e;
   const float scale_log2 = scale * 1.4426950408889634f;
   return launch_pdl(prefill_attn_tc_kernel, dim3(unsigned((T + kTileQ - 1) / kTileQ), H),
-                    dim3(kAtThreads), kAtSmem, stream, tm_q, tm_kc, tm_v, tm_kr, q_pos, T, L, H,
-                    d_r, scale_log2, out, lse, status);
+                    dim3(kAtThreads), kAtSmem, stream, tm_kc, tm_v, tm_kr, q_nope, q_pe,
+                    static_cast<const float2*>(cs), q_pos, T, L, H, d_r, scale_log2, out, lse,
+                    status);
 }
 
 }  // namespace mla

@@ -157,10 +157,10 @@ def test_other_entry_point_errors(lib):
 def test_prefill_entry_point_errors(lib):
     d = _dims(H=8)
     need = lib.mla_prefill_workspace_bytes(ctypes.byref(d), 100, 300)
-    # q_full [H, T, 192] + K^C and V [H, L, 128] + k^R [L, 64], each rounded
-    # up to 1 KB.
+    # K^C and V [H, L, 128] + k^R [L, 64], 16-bit, and the queries' RoPE
+    # angles [T, 32] (cos, sin) in fp32, each rounded up to 1 KB.
     r1k = lambda x: (x + 1023) // 1024 * 1024  # noqa: E731
-    assert need == r1k(8 * 100 * 192 * 2) + 2 * r1k(8 * 300 * 128 * 2) + r1k(300 * 64 * 2)
+    assert need == 2 * r1k(8 * 300 * 128 * 2) + r1k(300 * 64 * 2) + r1k(100 * 32 * 8)
     pf = lambda T=100, L=300, qn=GOOD, qpe=GOOD, pos=GOOD, scale=0.0, base=1e4, out=GOOD2, \
         ws=GOOD2, n=need, dims=d: lib.mla_prefill(  # noqa: E731
             ctypes.byref(dims), T, L, qn, qpe, pos, GOOD, GOOD, GOOD, scale, base, out, None,
@@ -183,7 +183,7 @@ def test_prefill_entry_point_errors(lib):
     assert pf(L=1 << 28) == UNSUP            # H * L beyond a 32-bit TMA row coordinate
     d0 = _dims(H=8, d_r=0)
     need0 = lib.mla_prefill_workspace_bytes(ctypes.byref(d0), 100, 300)
-    assert need0 == r1k(8 * 100 * 128 * 2) + 2 * r1k(8 * 300 * 128 * 2)
+    assert need0 == 2 * r1k(8 * 300 * 128 * 2)
     assert pf(dims=d0, qpe=None, n=need0 - 1) == WS   # NoPE: q_pe may be NULL
 
 
