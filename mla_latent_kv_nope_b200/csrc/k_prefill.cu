@@ -289,39 +289,48 @@ __device__ __forceinline__ void warp_arrive_after_tmem_st(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-// Query row t of head i, fp16 dims [32 j, 32 j + 32) as 16 packed columns:
-// q^C for j < 4, then RoPE(q^R, pos) (pairs (k, k + d_r/2)).  Rows past T are zero.
-__device__ __forceinline__ void query_chunk(const __nv_bfloat16* __restrict__ q_nope,
-                                            const __nv_bfloat16* __restrict__ q_pe, bool valid,
-                                            int64_t row, int d_r, int j,
-                                            const float2* __restrict__ cs_row, uint32_t (&out)[16]) {
-  if (!valid) {
+// The query row Q_i[t] = [q^C ; RoPE(q^R, pos)] in fp16 pairs, written to
+// tensor memory by the two threads of the row: half 0 takes q^C dims 0-127
+// (dims 0-63 without RoPE), half 1 the RoPE block (dims 64-127 of q^C
+// without RoPE).  Every global load of a thread is issued before the first
+// use, so the row costs one memory round trip.  Rows past T are zero.
+__device__ __forceinline__ void nope_to_tmem(const uint4* __restrict__ src, bool valid, int j0,
+                                             int j1, uint32_t taddr) {
+  uint4 raw[16];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) out[e] = 0u;
-    return;
-  }
-  if (j < kDn / 32) {
-    const uint4* src = reinterpret_cast<const uint4*>(q_nope + row * kDn + 32 * j);
+  for (int u = 0; u < 16; ++u)
+    raw[u] = (valid && u < 4 * (j1 - j0)) ? src[4 * j0 + u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (j >= j1 - j0) break;
+    uint32_t v[16];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const uint4 h = bf16x8_to_f16x8(src[u]);
-      out[4 * u] = h.x;
-      out[4 * u + 1] = h.y;
-      out[4 * u + 2] = h.z;
-      out[4 * u + 3] = h.w;
+      const uint4 hq = bf16x8_to_f16x8(raw[4 * j + u]);
+      v[4 * u] = hq.x;
+      v[4 * u + 1] = hq.y;
+      v[4 * u + 2] = hq.z;
+      v[4 * u + 3] = hq.w;
     }
-    return;
+    tmem_st16(taddr + uint32_t(16 * (j0 + j)), v);
   }
-  // RoPE chunk: the whole q^R row (64 bf16) and the 32 angle pairs come in
-  // with 16-byte loads; output dims e0 .. e0 + 31 of the rotated block.
-  const int e0 = 32 * (j - kDn / 32);
-  const bool upper = e0 >= 32;               // d_r = 64: dims 32..63 are the k + 32 halves
+}
+
+// RoPE block (d_r = 64): y[k] = x[k] c_k - x[k+32] s_k, y[k+32] = x[k] s_k +
+// x[k+32] c_k, with (c_k, s_k) from the angle table; 32 packed columns.
+__device__ __forceinline__ void rope_to_tmem(const uint4* __restrict__ src,
+                                             const float4* __restrict__ cs4, bool valid,
+                                             uint32_t taddr) {
+  uint4 xr[8];
+  float4 a[16];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) xr[u] = valid ? src[u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int u = 0; u < 16; ++u) a[u] = valid ? cs4[u] : make_float4(1.f, 0.f, 1.f, 0.f);
   float x[64];
-  const uint4* src = reinterpret_cast<const uint4*>(q_pe + row * d_r);
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    const uint4 w = src[u];
-    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&xr[u]);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float2 f = __bfloat1622float2(p2[q]);
@@ -329,14 +338,14 @@ __device__ __forceinline__ void query_chunk(const __nv_bfloat16* __restrict__ q_
       x[8 * u + 2 * q + 1] = f.y;
     }
   }
-  const float4* cs4 = reinterpret_cast<const float4*>(cs_row);
+  uint32_t v[32];
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    const float4 a = cs4[e / 2];               // (cos, sin) of pairs e and e + 1
-    const float y0 = upper ? x[e] * a.y + x[e + 32] * a.x : x[e] * a.x - x[e + 32] * a.y;
-    const float y1 = upper ? x[e + 1] * a.w + x[e + 33] * a.z : x[e + 1] * a.z - x[e + 33] * a.w;
-    out[e / 2] = pack_f16x2(y0, y1);
+    const float4 c = a[e / 2];                 // (cos, sin) of pairs e and e + 1
+    v[e / 2] = pack_f16x2(x[e] * c.x - x[e + 32] * c.y, x[e + 1] * c.z - x[e + 33] * c.w);
+    v[16 + e / 2] = pack_f16x2(x[e] * c.y + x[e + 32] * c.x, x[e + 1] * c.w + x[e + 33] * c.z);
   }
+  tmem_st32(taddr, v);
 }
 
 __global__ void __launch_bounds__(kAtThreads, 1)
@@ -495,15 +504,21 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kc,
     const int r = 32 * quad + lane;
     const uint32_t lane_base = uint32_t(32 * quad) << 16;
     const int cb = 64 * h;
-    // The query row into tensor memory: this half writes chunks [nc/2 h, nc/2 (h+1)).
+    // The query row into tensor memory (see nope_to_tmem / rope_to_tmem).
     {
       const int t = q0 + r;
-      const int nc = (kDn + d_r) / 32;
-      const int64_t row = int64_t(t) * H + i;
-      for (int j = h * nc / 2; j < (h + 1) * nc / 2; ++j) {
-        uint32_t v[16];
-        query_chunk(q_nope, q_pe, t < T, row, d_r, j, cs + int64_t(t < T ? t : 0) * (d_r / 2), v);
-        tmem_st16(tmem + lane_base + kColQ + uint32_t(16 * j), v);
+      const bool valid = t < T;
+      const int64_t row = int64_t(valid ? t : 0) * H + i;
+      const uint4* src = reinterpret_cast<const uint4*>(q_nope + row * kDn);
+      const uint32_t qa = tmem + lane_base + kColQ;
+      if (h == 0) {
+        nope_to_tmem(src, valid, 0, d_r ? 4 : 2, qa);
+      } else if (d_r) {
+        rope_to_tmem(reinterpret_cast<const uint4*>(q_pe + row * d_r),
+                     reinterpret_cast<const float4*>(cs + int64_t(valid ? t : 0) * (d_r / 2)),
+                     valid, qa + 64);
+      } else {
+        nope_to_tmem(src, valid, 2, 4, qa);
       }
       warp_arrive_after_tmem_st(&bars->q_ready);
     }
