@@ -523,18 +523,16 @@ class DecodeStep:
                 self.append(h, cache, seqlens, block_table, scales)
             return self.attend(q_nope, q_pe, q_pos, cache, seqlens, block_table, scales)
         main = torch.cuda.current_stream()
-        # Fork point: the side stream starts after everything issued so far
-        # (the previous step's decode has finished reading q_cat).  The append
-        # is launched first: its projection CTAs are the larger ones, so they
-        # take their SMs before absorb_q's smaller CTAs fill the space left
-        # beside them, and the two run side by side.
-        fork = torch.cuda.Event()
-        fork.record(main)
-        if h is not None:
-            self.append(h, cache, seqlens, block_table, scales)
-        self._side.wait_event(fork)
+        # Fork: the side stream starts after everything issued so far (the
+        # previous step's decode has finished reading q_cat).  absorb_q is
+        # launched first: measured in a graph on B200 the pair takes 14.9 us
+        # this way and 20.6 us with the append launched first (each alone
+        # about 12.3 us).
+        self._side.wait_stream(main)
         with torch.cuda.stream(self._side):
             self.absorb(q_nope, q_pe, q_pos)
+        if h is not None:
+            self.append(h, cache, seqlens, block_table, scales)
         main.wait_stream(self._side)
         return self._attend_latent(cache, seqlens, block_table, scales)
 
