@@ -29,23 +29,49 @@ def _load(name):
 # The draw order and shapes are fixed by the page; the arithmetic below goes
 # through the oracle's functions.
 # ---------------------------------------------------------------------------
+# The seeded inputs of [MLA-とは] "数値検証" and its RoPE follow-ups, as data:
+# (name, kind, shape, fan-in divisor) in the order the page draws them from
+# default_rng(0).  "normal" draws are scaled by 1/sqrt(fan-in); "attn" is a
+# uniform draw normalised over the key axis.  The order is an interface (it
+# decides every printed value); the arithmetic after it goes through the
+# oracle.
+_PAGE_DIMS = dict(d=256, d_c=64, d_cq=96, d_h=32, n_h=4, T=6, d_r=16)
+_PAGE_DRAWS = (
+    ("hid", "normal", ("T", "d"), None),
+    ("w_dkv", "normal", ("d", "d_c"), "d"),
+    ("w_uk", "normal", ("d_c", "n_h*d_h"), "d_c"),
+    ("w_dq", "normal", ("d", "d_cq"), "d"),
+    ("w_uq", "normal", ("d_cq", "n_h*d_h"), "d_cq"),
+    ("w_uv", "normal", ("d_c", "n_h*d_h"), "d_c"),
+    ("w_o", "normal", ("n_h*d_h", "d"), "n_h*d_h"),
+    ("attn", "attn", ("T", "T", "n_h"), None),
+    ("w_qr", "normal", ("d_cq", "n_h*d_r"), "d_cq"),
+    ("w_kr", "normal", ("d", "d_r"), "d"),
+)
+
+
+def _size(expr):
+    out = 1
+    for f in expr.split("*"):
+        out *= _PAGE_DIMS[f]
+    return out
+
+
 def _pages_inputs():
     g = np.random.default_rng(0)
-    d, d_c, d_cq, d_h, n_h, T, d_r = 256, 64, 96, 32, 4, 6, 16
     x = {}
-    x["hid"] = g.normal(size=(T, d))
-    x["w_dkv"] = g.normal(size=(d, d_c)) / np.sqrt(d)
-    x["w_uk"] = g.normal(size=(d_c, n_h * d_h)) / np.sqrt(d_c)
-    x["w_dq"] = g.normal(size=(d, d_cq)) / np.sqrt(d)
-    x["w_uq"] = g.normal(size=(d_cq, n_h * d_h)) / np.sqrt(d_cq)
-    x["w_uv"] = g.normal(size=(d_c, n_h * d_h)) / np.sqrt(d_c)
-    x["w_o"] = g.normal(size=(n_h * d_h, d)) / np.sqrt(n_h * d_h)
-    attn = g.random((T, T, n_h))
-    x["attn"] = attn / attn.sum(axis=1, keepdims=True)
-    x["w_qr"] = g.normal(size=(d_cq, n_h * d_r)) / np.sqrt(d_cq)
-    x["w_kr"] = g.normal(size=(d, d_r)) / np.sqrt(d)
+    for name, kind, shape, fan_in in _PAGE_DRAWS:
+        dims = tuple(_size(e) for e in shape)
+        if kind == "attn":
+            a = g.random(dims)
+            x[name] = a / a.sum(axis=1, keepdims=True)
+        else:
+            a = g.normal(size=dims)
+            x[name] = a / np.sqrt(_size(fan_in)) if fan_in else a
+    d, d_c, d_cq, d_h, n_h, T, d_r = (_PAGE_DIMS[k]
+                                      for k in ("d", "d_c", "d_cq", "d_h", "n_h", "T", "d_r"))
     x["dims"] = (d, d_c, d_cq, d_h, n_h, T, d_r)
-    # Row-vector weights of the snippets -> the oracle's column convention.
+    # Row-vector weights of the page's checks -> the oracle's column convention.
     x["W_UK"] = x["w_uk"].reshape(d_c, n_h, d_h).transpose(1, 2, 0)
     x["W_UV"] = x["w_uv"].reshape(d_c, n_h, d_h).transpose(1, 2, 0)
     x["c_kv"] = O.down_project(x["hid"], x["w_dkv"].T)
