@@ -236,6 +236,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
                                         : min(int64_t(kTileKeys), cap - t * kTileKeys);
           bulk_prefetch_l2(cache_bytes + r * kRowBytes, uint32_t(rows * kRowBytes));
         };
+        int64_t pf = lo + kStages;   // next tile to prefetch into L2
         for (int64_t t = lo; t < hi; ++t, ++i) {
           const int s = i % kStages;
           // The tile's first row (a page-table read when paged) is looked up
@@ -263,10 +264,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
             for (int c = 0; c < kLoadChunks; ++c)
               tma_load_2d(&tm_c, &bars->full[s], dst + c * kChunkBytes, c * kChunkElems, crow);
           }
-          // Loads of the first tiles go out before any prefetch.
-          if (t == lo)
-            for (int64_t u = t + kStages; u < t + kPrefetchTiles; ++u) prefetch(u);
-          prefetch(t + kPrefetchTiles);
+          // Prefetch up to kPrefetchTiles ahead; the kernel's first stage loads
+          // all go out before any prefetch (at start-up every CTA asks for its
+          // first tiles and query block at once, and those are what the first
+          // QK^T waits for).
+          if (t == lo) pf = t + kStages;
+          if (i >= kStages - 1)
+            for (; pf <= t + kPrefetchTiles; ++pf) prefetch(pf);
         }
         return true;
       });
