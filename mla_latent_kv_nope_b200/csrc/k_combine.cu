@@ -38,6 +38,7 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
   constexpr int kBatch = 1;   // partials per round past the first four
   __shared__ float4 s_rows[kCombineHeads][kQuadsPerBlock + 1];
   __shared__ int64_t s_red[2][kCombineWarps];
+  pdl_wait();   // the partials come from the decode launched just before
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h0 = blockIdx.y * kCombineHeads;
@@ -208,6 +209,7 @@ combine_many_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int
   __shared__ float4 s_acc[kCombineWarps][kCombineHeads][kManyQuads];
   __shared__ float s_red[kCombineWarps][kCombineHeads];
   __shared__ int64_t s_pre[2][kCombineWarps];
+  pdl_wait();   // the partials come from the decode launched just before
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h0 = blockIdx.y * kCombineHeads;
@@ -341,16 +343,16 @@ cudaError_t launch_combine(const int32_t* seqlens, int64_t cap, int B, int H, in
   const int nq = d_c / 4;
   const int hb = (H + kCombineHeads - 1) / kCombineHeads;
   // Many partials per sequence on average (few long sequences): the warps
-  // split the partials.  Launched without programmatic overlap: measured on
-  // B200, letting it start beside the decode's last CTAs made the pair slower.
-  if (int64_t(B) + W - 1 > int64_t(kFastParts) * B) {
-    combine_many_kernel<<<dim3(B, hb, (nq + kManyQuads - 1) / kManyQuads), kCombineThreads, 0,
-                          stream>>>(seqlens, cap, B, H, d_c, W, o_part, lse_part, o_lat, lse);
-    return cudaGetLastError();
-  }
-  combine_kernel<<<dim3(B, hb, (nq + kQuadsPerBlock - 1) / kQuadsPerBlock), kCombineThreads, 0,
-                   stream>>>(seqlens, cap, B, H, d_c, W, o_part, lse_part, o_lat, lse);
-  return cudaGetLastError();
+  // split the partials.  Both are launched with programmatic overlap; the
+  // decode before them triggers only by finishing, so the combine's launch
+  // overlaps the decode's drain and nothing more.
+  if (int64_t(B) + W - 1 > int64_t(kFastParts) * B)
+    return launch_pdl(combine_many_kernel, dim3(B, hb, (nq + kManyQuads - 1) / kManyQuads),
+                      dim3(kCombineThreads), 0, stream, seqlens, cap, B, H, d_c, W, o_part,
+                      lse_part, o_lat, lse);
+  return launch_pdl(combine_kernel, dim3(B, hb, (nq + kQuadsPerBlock - 1) / kQuadsPerBlock),
+                    dim3(kCombineThreads), 0, stream, seqlens, cap, B, H, d_c, W, o_part, lse_part,
+                    o_lat, lse);
 }
 
 }  // namespace mla

@@ -213,7 +213,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_trigger();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
   uint32_t n_issued = 0;   // loads issued by the producer (lane 0 of its warp)
