@@ -772,6 +772,99 @@ def run_prefill(args, rank, world, local_rank):
     }
 
 
+def run_seqshard(args, rank, world, local_rank):
+    """Long-context sequence sharding: every rank holds one contiguous token
+    range of every sequence (dist.token_ranges) and runs absorb + decode +
+    combine on it; the per-range (o_lat, lse) are all-gathered (NCCL), merged
+    by log-sum-exp (mla_merge_partials) and projected by W^UV.  The batch is
+    the same on every rank, so total work is fixed as N grows (strong
+    scaling).  Timed on the device, max over ranks; the collective is inside
+    the timed region."""
+    import numpy as np
+    import torch
+
+    import mla_latent_kv_nope_b200 as mla
+    from mla_latent_kv_nope_b200 import dist as mdist
+    from mla_latent_kv_nope_b200 import inputs
+    from mla_latent_kv_nope_b200.build import build
+
+    if rank == 0:
+        build()
+    if world > 1:
+        mdist.barrier(world)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = inputs.WORKLOADS[args.workload]
+    lens = inputs.seqlens(w)
+    ranges = mdist.token_ranges(lens, world)[rank]
+    loc = (ranges[:, 1] - ranges[:, 0]).astype(np.int32)
+    cap = max(int(loc.max()), 1)
+    cap = (cap + 63) // 64 * 64
+    dims = mla.Dims(w.B, w.H, w.d_c, w.d_r, w.d_nope, w.d_v, cap, w.dtype)
+    cache = torch.zeros(w.B, cap, w.R, dtype=torch.bfloat16, device=dev)
+    for b in range(w.B):
+        lo, hi = int(ranges[b, 0]), int(ranges[b, 1])
+        if hi > lo:
+            cache[b, :hi - lo].copy_(torch.from_numpy(inputs.cache_rows(w, b, hi)[lo:hi]))
+    local_seq = torch.from_numpy(loc).to(dev)
+    qn, qp = inputs.query(w)
+    Wuk, Wuv = inputs.weights(w)
+    T = lambda a: torch.from_numpy(a).to(dev, torch.bfloat16)  # noqa: E731
+    q_nope, q_pe, W_UK, W_UV = map(T, (qn, qp, Wuk, Wuv))
+    q_pos = torch.from_numpy((lens - 1).astype(np.int32)).to(dev)
+    step = mla.DecodeStep(dims, W_UK, W_UV, None, num_splits=args.splits)
+    stream = torch.cuda.current_stream()
+
+    def one():
+        mdist.sequence_sharded_attend(step, q_nope, q_pe, q_pos, cache, local_seq, world)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    if mla.get_device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+    with ClockSampler(local_rank) as clk:
+        mdist.barrier(world)
+        torch.cuda.synchronize()
+        clk.start()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            one()
+        t1.record(stream)
+        clk.poll_until(t1.query)
+        torch.cuda.synchronize()
+        clk.stop()
+        mdist.barrier(world)
+    ms = mdist.max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    if mla.get_device_status() != 0:
+        raise RuntimeError("device status error during timing")
+    if rank != 0:
+        return None
+    hbm, _, _, peak_src = _peaks()
+    byts = int(lens.sum()) * w.R * 2
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {
+        "metric": METRIC + " (sequence-sharded)", "value": w.B / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded)",
+        "config": {"workload": _workload_desc(w) + f", each rank a token range (<= {cap} rows)",
+                   "global_batch": w.B, "seq_len": int(lens.max()),
+                   "parallelism": f"seq{world}", "launch": "eager",
+                   "l2": "inputs exceed L2" if byts > 2 * L2_BYTES else "per-rank cache may fit L2"},
+        "roofline": {"kernel": "whole sharded attend (absorb, decode, combine, all-gather, merge, "
+                               "out_proj) over the whole job's cache bytes",
+                     "bound": "hbm", "achieved": gbs * 1.0, "peak": hbm * world, "unit": "GB/s",
+                     "frac": gbs / (hbm * world), "traffic": None,
+                     "algorithmic_bytes_per_step": byts,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json, x n_gpus)"
+                                    if peak_src == "measured" else "fallback x n_gpus"},
+        "gpu_launches": (6 if world > 1 else 4) * args.steps,
+        "clocks": clk.summary(),
+    }
+
+
 def _relaunch_per_gpu(n):
     """`--gpus N` (N > 1) started without a launcher: run this same command as
     N ranks, one process per GPU, under torch.distributed.run (rendezvous on
@@ -839,10 +932,13 @@ def main():
                     help="keep the latent cache in shuffled 64-row pages behind a block table")
     ap.add_argument("--eager", action="store_true",
                     help="launch each kernel from the host every step instead of a CUDA graph")
-    ap.add_argument("--kernel", default="step", choices=["step", "folded_out_proj", "prefill"],
+    ap.add_argument("--kernel", default="step",
+                    choices=["step", "folded_out_proj", "prefill", "seqshard"],
                     help="step: the whole decode step (default); folded_out_proj: the W^O "
                          "fold variant of the output projection alone; prefill: the "
-                         "materialised prefill of one sequence")
+                         "materialised prefill of one sequence; seqshard: attention with the "
+                         "cache split by token range over the ranks (use with "
+                         "--workload longctx_bf16)")
     ap.add_argument("--prefill-tokens", type=int, default=4096,
                     help="prompt length T = L of --kernel prefill")
     ap.add_argument("--dry-run", action="store_true",
@@ -879,6 +975,8 @@ def main():
             res = run_folded_out_proj(args, rank, world, local_rank)
         elif args.kernel == "prefill":
             res = run_prefill(args, rank, world, local_rank)
+        elif args.kernel == "seqshard":
+            res = run_seqshard(args, rank, world, local_rank)
         else:
             res = run_ours(args, rank, world, local_rank)
         if world > 1:
