@@ -4,8 +4,9 @@
 //   o_lat[b,i] = sum_s exp(lse_s - lse[b,i]) * o_s
 //
 // The partials of sequence b live in slots (b + w) for every non-empty worker
-// w whose tile range meets b's tiles; the block recomputes that set from the
-// sequence lengths exactly as the decode kernels dealt the tiles.
+// w whose unit range meets b's tiles; the block recomputes that set from the
+// sequence lengths exactly as the decode kernels dealt the work units (each
+// sequence's kSwitchUnits start-up units, then its tiles).
 // Partials are stored as o_part[slot][d_c / 4][H][4] (see combine_kernel).
 #include "common.cuh"
 #include "kernels.h"
@@ -50,9 +51,9 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
   const int nh = min(kCombineHeads, H - h0);
   int64_t pre = 0, tot = 0;
   for (int bb = threadIdx.x; bb < B; bb += kCombineThreads) {
-    const int64_t nt = tiles_of(clamp_len(seqlens[bb], cap));
-    tot += nt;
-    if (bb < b) pre += nt;
+    const int64_t nu = units_of(clamp_len(seqlens[bb], cap));
+    tot += nu;
+    if (bb < b) pre += nu;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -80,8 +81,9 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
     if (blockIdx.z == 0 && warp == 0 && head_ok && lse_out) lse_out[int64_t(b) * H + i] = -INFINITY;
     return;
   }
-  const int w_first = int(worker_of_tile(pre, T, W));
-  const int w_last = int(worker_of_tile(pre + nt - 1, T, W));
+  // The sequence's tiles are units [pre + kSwitchUnits, + nt) of the deal.
+  const int w_first = int(worker_of_tile(pre + kSwitchUnits, T, W));
+  const int w_last = int(worker_of_tile(pre + kSwitchUnits + nt - 1, T, W));
   auto live = [&](int w) { return worker_tile_begin(w, T, W) != worker_tile_begin(w + 1, T, W); };
   // Column groups of this thread: q_base + warp + 8 j, j < 4.
   const float4* src0 = reinterpret_cast<const float4*>(o_part) + int64_t(q_base + warp) * H + i;
@@ -221,9 +223,9 @@ combine_many_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int
   const int nh = min(kCombineHeads, H - h0);
   int64_t pre = 0, tot = 0;
   for (int bb = threadIdx.x; bb < B; bb += kCombineThreads) {
-    const int64_t nt = tiles_of(clamp_len(seqlens[bb], cap));
-    tot += nt;
-    if (bb < b) pre += nt;
+    const int64_t nu = units_of(clamp_len(seqlens[bb], cap));
+    tot += nu;
+    if (bb < b) pre += nu;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -251,8 +253,9 @@ combine_many_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int
     if (blockIdx.z == 0 && warp == 0 && head_ok && lse_out) lse_out[int64_t(b) * H + i] = -INFINITY;
     return;
   }
-  const int w_first = int(worker_of_tile(pre, T, W));
-  const int w_last = int(worker_of_tile(pre + nt - 1, T, W));
+  // The sequence's tiles are units [pre + kSwitchUnits, + nt) of the deal.
+  const int w_first = int(worker_of_tile(pre + kSwitchUnits, T, W));
+  const int w_last = int(worker_of_tile(pre + kSwitchUnits + nt - 1, T, W));
   // This warp's partials: w_first + warp + 8 j.  Their lse values, up to 8
   // per warp in registers (64 partials per sequence), the rest reloaded.
   auto lse_of = [&](int w) {

@@ -38,10 +38,11 @@ decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache, con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = h0 + warp;
 
-  // Total tiles T and this worker's tile range.
+  // Total work units T (tiles plus each sequence's start-up units, as the
+  // tensor-core kernels deal them) and this worker's unit range.
   int64_t n_tiles = 0;
   for (int b = 0; b < B; ++b) {
-    n_tiles += tiles_of(clamp_len(seqlens[b], cap));
+    n_tiles += units_of(clamp_len(seqlens[b], cap));
     if (w == 0 && blockIdx.y == 0 && threadIdx.x == 0 && int64_t(seqlens[b]) > cap)
       record_status(status, MLA_ERR_BOUNDS);
   }
@@ -50,15 +51,16 @@ decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache, con
   const int64_t t_end = worker_tile_begin(w + 1, n_tiles, W);
   if (t_begin >= t_end) return;
 
-  // Walk the sequences overlapping [t_begin, t_end).
+  // Walk the sequences whose tiles overlap [t_begin, t_end).
   int64_t prefix = 0;
   for (int b = 0; b < B && prefix < t_end; ++b) {
     const int64_t L = clamp_len(seqlens[b], cap);
     const int64_t nt = tiles_of(L);
-    const int64_t lo_t = max(prefix, t_begin), hi_t = min(prefix + nt, t_end);
-    if (lo_t < hi_t) {
-      const int64_t key_lo = (lo_t - prefix) * kTileKeys;
-      const int64_t key_hi = min((hi_t - prefix) * int64_t(kTileKeys), L);
+    const int64_t r0 = prefix + kSwitchUnits;   // this sequence's first tile
+    const int64_t lo_t = max(r0, t_begin), hi_t = min(r0 + nt, t_end);
+    if (nt > 0 && lo_t < hi_t) {
+      const int64_t key_lo = (lo_t - r0) * kTileKeys;
+      const int64_t key_hi = min((hi_t - r0) * int64_t(kTileKeys), L);
 
       // Stage this block's queries.
       __syncthreads();
@@ -120,7 +122,7 @@ decode_simt_kernel(const T* __restrict__ q_cat, const T* __restrict__ cache, con
         if (lane == 0) lse_part[int64_t(slot) * H + head] = m + logf(l);
       }
     }
-    prefix += nt;
+    prefix += units_of(L);
   }
 }
 

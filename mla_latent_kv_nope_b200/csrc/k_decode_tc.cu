@@ -391,7 +391,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
     float next_scale = 0.f;
     {
       const int b0 = tp.next_sequence(-1, t_begin, t_end);
-      if (b0 >= 0) next_scale = load_scale(b0, max(tp.at(b0), t_begin) - tp.at(b0));
+      if (b0 >= 0) next_scale = load_scale(b0, max(tp.tile0(b0), t_begin) - tp.tile0(b0));
     }
     for_each_segment(tp, t_begin, t_end, [&](int b, int64_t lo, int64_t hi, int64_t) {
       for (int64_t t = lo; t < hi; ++t, ++i) {

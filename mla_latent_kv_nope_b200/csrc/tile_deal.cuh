@@ -1,10 +1,12 @@
 // The split-KV work list shared by the tensor-core decode kernels.
 //
-// The key space of all sequences, cut into tiles of kTileKeys rows and
-// concatenated in batch order (T tiles), is dealt into W contiguous ranges;
-// worker w takes tiles [floor(wT/W), floor((w+1)T/W)) and walks the
-// sequences that overlap its range ("segments").  Every role of a CTA walks
-// the same segments in the same order, so their barrier phases agree.
+// The key space of all sequences, cut into tiles of kTileKeys rows, is laid
+// out in batch order as work units: each sequence with tiles takes
+// kSwitchUnits units (its start-up cost) and then one unit per tile (T units
+// in all).  The units are dealt into W contiguous ranges: worker w takes
+// units [floor(wT/W), floor((w+1)T/W)) and walks the sequences whose tiles
+// overlap its range ("segments").  Every role of a CTA walks the same
+// segments in the same order, so their barrier phases agree.
 #pragma once
 
 #include "common.cuh"
@@ -17,8 +19,9 @@ namespace mla {
 constexpr int kMaxSeqSmem = 1024;
 constexpr size_t kTilePrefixSmemBytes = sizeof(int32_t) * (2 * kMaxSeqSmem + 1);
 
-// Tile prefix of the batch: prefix(b) = sum of tiles of sequences < b, from
-// shared memory when the batch fits, else recomputed from the lengths.
+// Unit prefix of the batch: at(b) = sum of the units of sequences < b, from
+// shared memory when the batch fits, else recomputed from the lengths; the
+// tiles of b are units [tile0(b), tile0(b) + tiles).
 struct TilePrefix {
   const int32_t* sp;       // shared prefix [B + 1] or nullptr
   const int32_t* sl;       // shared clamped lengths [B] or nullptr
@@ -28,16 +31,17 @@ struct TilePrefix {
   __device__ int64_t at(int b) const {
     if (sp) return sp[b];
     int64_t p = 0;
-    for (int k = 0; k < b; ++k) p += tiles_of(clamp_len(seqlens[k], cap));
+    for (int k = 0; k < b; ++k) p += units_of(clamp_len(seqlens[k], cap));
     return p;
   }
+  __device__ int64_t tile0(int b) const { return at(b) + kSwitchUnits; }
   __device__ int64_t len(int b) const { return sl ? sl[b] : clamp_len(seqlens[b], cap); }
-  // First sequence whose tiles end after tile t (binary search on the prefix).
+  // First sequence whose units end after unit t (binary search on the prefix).
   __device__ int first_after(int64_t t) const {
     if (!sp) {
       int64_t p = 0;
       for (int b = 0; b < B; ++b) {
-        p += tiles_of(len(b));
+        p += units_of(len(b));
         if (p > t) return b;
       }
       return B;
@@ -49,21 +53,22 @@ struct TilePrefix {
     }
     return lo;
   }
-  // The sequence of the range [t_begin, t_end) that follows sequence `after`
-  // (-1 for the first), or -1 if there is none.
+  // The sequence with tiles in the unit range [t_begin, t_end) that follows
+  // sequence `after` (-1 for the first), or -1 if there is none.
   __device__ int next_sequence(int after, int64_t t_begin, int64_t t_end) const {
     for (int bb = (after < 0 ? first_after(t_begin) : after + 1); bb < B; ++bb) {
       const int64_t pre = at(bb);
       if (pre >= t_end) return -1;
       const int64_t nt = tiles_of(len(bb));
-      if (nt > 0 && pre + nt > t_begin) return bb;
+      const int64_t r0 = pre + kSwitchUnits;
+      if (nt > 0 && max(r0, t_begin) < min(r0 + nt, t_end)) return bb;
     }
     return -1;
   }
 };
 
 // Builds the shared prefix (all threads of the block take part; two block
-// barriers) and returns the total tile count.  `smem` holds
+// barriers) and returns the total unit count.  `smem` holds
 // kTilePrefixSmemBytes.
 __device__ __forceinline__ int64_t build_tile_prefix(uint8_t* smem, const int32_t* seqlens,
                                                      int B, int64_t cap, TilePrefix* tp) {
@@ -76,7 +81,7 @@ __device__ __forceinline__ int64_t build_tile_prefix(uint8_t* smem, const int32_
     for (int b = threadIdx.x; b < B; b += blockDim.x) {
       const int64_t L = clamp_len(seqlens[b], cap);
       s_lens[b] = int32_t(L);
-      s_prefix[b + 1] = int32_t(tiles_of(L));
+      s_prefix[b + 1] = int32_t(units_of(L));
     }
     __syncthreads();
     if (warp == 0) {
@@ -96,14 +101,14 @@ __device__ __forceinline__ int64_t build_tile_prefix(uint8_t* smem, const int32_
     __syncthreads();
     n_tiles = s_prefix[B];
   } else {
-    for (int b = 0; b < B; ++b) n_tiles += tiles_of(clamp_len(seqlens[b], cap));
+    for (int b = 0; b < B; ++b) n_tiles += units_of(clamp_len(seqlens[b], cap));
   }
   *tp = TilePrefix{in_smem ? s_prefix : nullptr, in_smem ? s_lens : nullptr, seqlens, B, cap};
   return n_tiles;
 }
 
-// Sequences overlapping the tile range [t_begin, t_end) are visited in
-// order; the callback gets (b, first tile, end tile (both local to b),
+// Sequences whose tiles overlap the unit range [t_begin, t_end) are visited
+// in order; the callback gets (b, first tile, end tile (both local to b),
 // length) and returns false to stop.
 template <typename F>
 __device__ __forceinline__ void for_each_segment(const TilePrefix& tp, int64_t t_begin,
@@ -113,8 +118,9 @@ __device__ __forceinline__ void for_each_segment(const TilePrefix& tp, int64_t t
     if (pre >= t_end) return;
     const int64_t L = tp.len(b);
     const int64_t nt = tiles_of(L);
-    const int64_t lo = max(pre, t_begin), hi = min(pre + nt, t_end);
-    if (lo < hi && !f(b, lo - pre, hi - pre, L)) return;
+    const int64_t r0 = pre + kSwitchUnits;
+    const int64_t lo = max(r0, t_begin), hi = min(r0 + nt, t_end);
+    if (lo < hi && !f(b, lo - r0, hi - r0, L)) return;
   }
 }
 

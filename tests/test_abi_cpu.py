@@ -232,19 +232,25 @@ def test_paged_entry_point_errors(lib):
     assert used.value == -1
 
 
+SWITCH_UNITS = 4   # start-up units ahead of each sequence's tiles in the deal
+
+
 def _deal(lens, W, tile=64):
-    """Host restatement of the documented split-KV dealing: worker w takes
-    tiles [w*T//W, (w+1)*T//W) of the concatenated per-sequence tiles."""
-    nt = [(L + tile - 1) // tile for L in lens]
-    T = sum(nt)
-    pre = [sum(nt[:b]) for b in range(len(lens))]
+    """Host restatement of the documented split-KV dealing: each sequence with
+    tiles takes SWITCH_UNITS units and then one unit per tile, in batch order
+    (T units); worker w takes units [w*T//W, (w+1)*T//W).  Returns T, the
+    owner of each unit, and the (worker, sequence) pairs that share tiles."""
+    nt = [(L + tile - 1) // tile if L > 0 else 0 for L in lens]
+    units = [n + SWITCH_UNITS if n else 0 for n in nt]
+    T = sum(units)
+    pre = [sum(units[:b]) for b in range(len(lens))]
     owner = {}
     for w in range(W):
         for t in range(w * T // W, (w + 1) * T // W):
             owner[t] = w
     pairs = set()
     for b, (p, n) in enumerate(zip(pre, nt)):
-        for t in range(p, p + n):
+        for t in range(p + SWITCH_UNITS, p + SWITCH_UNITS + n):
             pairs.add((owner[t], b))
     return T, owner, pairs
 
@@ -253,9 +259,9 @@ def _deal(lens, W, tile=64):
                                     ([5, 0, 0, 7], 16), ([131072] * 4, 148),
                                     ([0, 0], 3)])
 def test_split_dealing_slots_unique(lens, W):
-    """Every tile has exactly one worker; the partial slots b + w of the
+    """Every work unit has exactly one worker; the partial slots b + w of the
     (worker, sequence) pairs are distinct and below B + W - 1; the owner of
-    tile t is ((t+1)*W - 1) // T, the closed form the kernels use."""
+    unit t is ((t+1)*W - 1) // T, the closed form the kernels use."""
     T, owner, pairs = _deal(lens, W)
     assert len(owner) == T
     slots = [b + w for (w, b) in pairs]

@@ -318,9 +318,12 @@ def test_combine_alone():
     lens = np.array([300, 0, 64, 1000, 1], dtype=np.int32)
     w = SMALL_BF16.scaled(B=B)
     d = dims_of(w, capacity=1000)
+    # The documented deal: each non-empty sequence takes 4 start-up units,
+    # then one unit per 64-key tile; worker w takes units [wT/W, (w+1)T/W).
     nt = [(L + 63) // 64 for L in lens]
-    T = sum(nt)
-    pre = np.concatenate([[0], np.cumsum(nt)])
+    units = [n + 4 if n else 0 for n in nt]
+    T = sum(units)
+    pre = np.concatenate([[0], np.cumsum(units)])
     slots = B + Wn - 1
     o_all, l_all = inputs.partials(1, H, slots, d_c, seed=3, empty_frac=0.0)
     ws = torch.full((mla.decode_workspace_bytes(d, Wn) // 4,), float("nan"), device="cuda")
@@ -337,7 +340,7 @@ def test_combine_alone():
         if nt[b] == 0:
             assert torch.all(o_lat[b] == 0) and torch.all(torch.isneginf(lse[b]))
             continue
-        ws_ = sorted({w_ for t in range(pre[b], pre[b + 1]) for w_ in range(Wn)
+        ws_ = sorted({w_ for t in range(pre[b] + 4, pre[b + 1]) for w_ in range(Wn)
                       if w_ * T // Wn <= t < (w_ + 1) * T // Wn})
         sl = [b + w_ for w_ in ws_]
         ref_o, ref_l = O.combine_partials(o_all[0][:, sl].astype(np.float64),
