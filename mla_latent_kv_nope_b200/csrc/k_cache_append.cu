@@ -22,7 +22,7 @@ namespace {
 constexpr int kApRows = 4;
 constexpr int kApBatch = 16;
 constexpr int kApThreads = 256;
-constexpr int kFinBatch = 16;       // partial sums loaded together in the finalize
+constexpr int kFinBatch = 32;       // partial sums loaded together in the finalize
 
 template <typename T>
 __global__ void __launch_bounds__(kApThreads)
@@ -86,6 +86,8 @@ append_finalize_kernel(const float* __restrict__ part, int n_parts,
   __shared__ float s_part[32];
   __shared__ int32_t s_L;
   if (threadIdx.x == 0) s_L = seqlens[b];
+  // The thread's first gain, loaded with the partial sums (one round trip).
+  const float g_first = (gamma && int(threadIdx.x) < d_c) ? gamma[threadIdx.x] : 1.f;
   // Sum the partials in a fixed order (deterministic) with up to
   // kFinBatch loads in flight per thread; one column per thread when the
   // block covers the row.
@@ -125,7 +127,7 @@ append_finalize_kernel(const float* __restrict__ part, int n_parts,
   }
   T* row = cache + r * R;
   for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
-    const float g = gamma ? gamma[c] : 1.f;
+    const float g = c == int(threadIdx.x) ? g_first : gamma ? gamma[c] : 1.f;
     row[c] = Storage<T>::from_f(xb[c] * inv * g);
   }
   const int half = d_r / 2;
@@ -160,6 +162,7 @@ append_finalize_fp8_kernel(const float* __restrict__ part, int n_parts,
   __shared__ float s_part[32];
   __shared__ int32_t s_L;
   if (threadIdx.x == 0) s_L = seqlens[b];
+  const float g_first = (gamma && int(threadIdx.x) < d_c) ? gamma[threadIdx.x] : 1.f;
   for (int c = threadIdx.x; c < R; c += blockDim.x) {
     const float* src = part + int64_t(b) * R + c;
     const int64_t stride = int64_t(B) * R;
@@ -197,7 +200,7 @@ append_finalize_fp8_kernel(const float* __restrict__ part, int n_parts,
   // The normalised latent (fp32) and its largest magnitude.
   float amax = 0.f;
   for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
-    const float v = s_x[c] * inv * (gamma ? gamma[c] : 1.f);
+    const float v = s_x[c] * inv * (c == int(threadIdx.x) ? g_first : gamma ? gamma[c] : 1.f);
     s_x[c] = v;
     amax = fmaxf(amax, fabsf(v));
   }
