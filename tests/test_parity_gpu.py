@@ -171,6 +171,12 @@ DECODE_CASES = [
     ("bf16-H128-W1", W["v3_bf16"].scaled(B=3, N=300), [300, 1, 100], 1, 1.0),
     ("bf16-H128-Wbig", W["v3_bf16"].scaled(B=2, N=2000), [2000, 3], 300, 1.0),
     ("bf16-H128-peaked-long", W["v3_bf16"].scaled(B=1, N=3000), [3000], 2, 10.0),
+    # Many partials per sequence with a peaked softmax: the combine's running
+    # maximum jumps between rounds of partials (one sequence over 74 workers,
+    # some of them with empty ranges; one long sequence among 31 short ones)
+    ("bf16-H128-peaked-manysplits", W["v3_bf16"].scaled(B=1, N=3000), [3000], 0, 10.0),
+    ("bf16-H128-one-long-many-short", W["v3_bf16"].scaled(B=25, N=4000),
+     [4000] + [64] * 23 + [1], 0, 10.0),
     ("bf16-H100", W["v3_bf16"].scaled(B=3, H=100, N=300), [300, 65, 0], 0, 1.0),
     ("bf16-H192", W["v3_bf16"].scaled(B=2, H=192, N=200), [200, 64], 0, 1.0),
     # NoPE ([yuuk] 横断的知見: MLA layers without RoPE): d_r = 0, rows are c^KV alone
