@@ -90,7 +90,7 @@ struct Barriers {
   uint64_t o_free;
   uint64_t mma_drain, pv_drain;
   uint64_t never;                 // injected test wait: nothing ever arrives on it
-  uint64_t widened[kStages];      // FP8 cache: the stage holds bf16 latent rows
+  uint64_t widened[kStages];      // FP8 cache: the stage holds fp16 latent rows
   uint64_t wsync[kStages];        // FP8 cache: every widen thread has read its codes
   uint32_t tmem_base;
   int abort_flag;
@@ -104,6 +104,10 @@ static_assert(kSmemBytes <= 232448, "shared memory budget of one CTA");
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256, false, true);
+// FP8 cache: both products in fp16 (the widened codes, the query, the scaled
+// RoPE keys and P are fp16 operands).
+constexpr uint32_t kIdescQK16 = idesc_f16_f32(64, 64, false, false);
+constexpr uint32_t kIdescPV16 = idesc_f16_f32(64, 256, false, true);
 
 __device__ __forceinline__ void raise_abort(Barriers* bars, int* status) {
   bars->abort_flag = 1;
@@ -127,20 +131,35 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// 8 E4M3 codes (little-endian in `c`) times the row's power-of-two scale, as
-// 8 bf16 (exact: an E4M3 value has 4 significant bits and scale * value stays
-// in range for the scales the append produces).
-__device__ __forceinline__ uint4 widen_e4m3x8(uint2 c, float scale) {
+// 8 E4M3 codes (little-endian in `c`) times the token's power-of-two scale
+// (`s2`, the scale as fp16 in both halves), as 8 fp16: the code converts
+// exactly (every finite E4M3 value is an fp16 value) and the product is one
+// fp16 multiply, exact while it is a normal fp16 (|c| >= 2^-14) and rounded
+// once below that.  fp16 holds every latent value of magnitude below 65504
+// and every power-of-two scale from 2^-24 to 2^15.
+__device__ __forceinline__ uint4 e4m3x8_to_f16(uint2 c, __half2 s2) {
   uint32_t out[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const uint32_t word = p < 2 ? c.x : c.y;
     const __nv_fp8x2_storage_t pair = __nv_fp8x2_storage_t((word >> (16 * (p & 1))) & 0xFFFFu);
-    const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
-    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
-    out[p] = *reinterpret_cast<const uint32_t*>(&b);
+    const __half2 v = __hmul2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)), s2);
+    out[p] = *reinterpret_cast<const uint32_t*>(&v);
   }
   return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// 8 bf16 as 8 fp16, rounded to nearest (exact for |x| in fp16's normal
+// range with at most 11 significant bits, which every bf16 value has).
+__device__ __forceinline__ uint4 bf16x8_to_f16(uint4 v) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(w[p] << 16),
+                                        __uint_as_float(w[p] & 0xFFFF0000u));
+    w[p] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 template <int kDr, bool kFp8>
@@ -290,8 +309,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_bf16_ts_w(d, a0 + uint32_t(c * 4 + k) * 8u,
-                          b0 + uint64_t((c * kChunkBytes + k * 32) >> 4), kIdescQK,
-                          (c | k) != 0);
+                          b0 + uint64_t((c * kChunkBytes + k * 32) >> 4),
+                          kFp8 ? kIdescQK16 : kIdescQK, (c | k) != 0);
         }
         mma_commit_w(&bars->s_full[sb]);
       }
@@ -328,8 +347,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
 #pragma unroll
           for (int h = 0; h < 2; ++h)
             mma_bf16_ss_w(tmem + kHiLanes + uint32_t(h) * 256u, a0 + uint64_t((k * 32) >> 4),
-                          b0 + uint64_t((4 * h * kChunkBytes + k * 2048) >> 4), kIdescPV,
-                          !(first && k == 0));
+                          b0 + uint64_t((4 * h * kChunkBytes + k * 2048) >> 4),
+                          kFp8 ? kIdescPV16 : kIdescPV, !(first && k == 0));
         }
         mma_commit_w(&bars->empty[st]);
       }
@@ -343,28 +362,31 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
   } else if (kFp8 && warp >= kWidenWarp0) {
     // ------------------------------------------------------------ widen (FP8 cache)
     // Thread (r, hh) expands row r of code boxes hh and 2 + hh: box c holds
-    // latent columns [128c, 128c + 128), i.e. bf16 chunks 2c and 2c + 1.
+    // latent columns [128c, 128c + 128), i.e. fp16 chunks 2c and 2c + 1.
     // Boxes 0-1 (chunks 4-5) are widened into chunks 0-3; boxes 2-3 are read
     // into registers, every widen thread meets at `wsync` (so chunks 4-7 have
-    // been read by all), then written into chunks 4-7.
+    // been read by all), then written into chunks 4-7.  Both products run in
+    // fp16, so the row's RoPE keys (chunk 8, bf16) are rewritten in place as
+    // fp16 too.
     const int wt = threadIdx.x - 32 * kWidenWarp0;
     const int r = wt >> 1, hh = wt & 1;
     uint32_t i = 0;
     bool ok = true;
     auto store_units = [&](uint8_t* stage, int box, int v, uint4 lo, uint4 hi_) {
-      // 16 codes -> dims [128 box + 16 v, +16): bf16 units 2(v%4), 2(v%4)+1 of
+      // 16 codes -> dims [128 box + 16 v, +16): fp16 units 2(v%4), 2(v%4)+1 of
       // chunk 2 box + v / 4, 128-byte swizzled.
       uint8_t* chunk = stage + (2 * box + v / 4) * kChunkBytes + r * 128;
       const int u0 = 2 * (v % 4);
       *reinterpret_cast<uint4*>(chunk + ((u0 ^ (r & 7)) * 16)) = lo;
       *reinterpret_cast<uint4*>(chunk + (((u0 + 1) ^ (r & 7)) * 16)) = hi_;
     };
-    // The row's scale for tile t of sequence b; rows past the capacity get 0
-    // (their keys are masked and their rows zeroed before P.C).
+    // The row's scale for tile t of sequence b; rows past the sequence's
+    // length get 0 (their keys are masked and their rows zeroed before P.C;
+    // their stored scales may hold anything).
     auto load_scale = [&](int b, int64_t t) {
       if (b < 0) return 0.f;
       const int64_t key = t * kTileKeys + r;
-      const int64_t prow = key < cap ? pm.row(b, key) : -1;
+      const int64_t prow = key < tp.len(b) ? pm.row(b, key) : -1;
       return prow >= 0 ? scales[prow] : 0.f;
     };
     // Scales are read one tile ahead of their use (a global load per row
@@ -384,6 +406,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
         else next_scale = load_scale(tp.next_sequence(b, t_begin, t_end), 0);
         if (!(ok = warp_wait(&bars->full[s], (i / kStages) & 1, abort_flag))) return false;
         uint8_t* stage = sStage + s * kStageBytes;
+        const __half2 s2 = __float2half2_rn(scale);
         // Code boxes arrive 128-byte swizzled like the bf16 chunks: unit v
         // (16 codes) of row r sits at 16 (v ^ (r % 8)), so the rows a warp
         // reads together fall in different banks.
@@ -394,8 +417,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           const uint4 c = code_unit(hh, v);
-          store_units(stage, hh, v, widen_e4m3x8(make_uint2(c.x, c.y), scale),
-                      widen_e4m3x8(make_uint2(c.z, c.w), scale));
+          store_units(stage, hh, v, e4m3x8_to_f16(make_uint2(c.x, c.y), s2),
+                      e4m3x8_to_f16(make_uint2(c.z, c.w), s2));
         }
         uint4 c2[8];
 #pragma unroll
@@ -404,8 +427,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
         if (!(ok = warp_wait(&bars->wsync[s], (i / kStages) & 1, abort_flag))) return false;
 #pragma unroll
         for (int v = 0; v < 8; ++v)
-          store_units(stage, 2 + hh, v, widen_e4m3x8(make_uint2(c2[v].x, c2[v].y), scale),
-                      widen_e4m3x8(make_uint2(c2[v].z, c2[v].w), scale));
+          store_units(stage, 2 + hh, v, e4m3x8_to_f16(make_uint2(c2[v].x, c2[v].y), s2),
+                      e4m3x8_to_f16(make_uint2(c2[v].z, c2[v].w), s2));
+        // RoPE keys: units 4 hh .. 4 hh + 3 of the row, as fp16.
+        {
+          uint8_t* rrow = stage + kRopeChunk * kChunkBytes + r * 128;
+#pragma unroll
+          for (int u = 4 * hh; u < 4 * hh + 4; ++u) {
+            uint4* unit = reinterpret_cast<uint4*>(rrow + ((u ^ (r & 7)) * 16));
+            *unit = bf16x8_to_f16(*unit);
+          }
+        }
         fence_proxy_async_smem();
         mbar_arrive(&bars->widened[s]);
       }
@@ -426,7 +458,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
     bool ok = true;
 
     // Query block of sequence b into tensor memory (lo lanes, K-major pairs of
-    // bf16 per 32-bit column).  A row is 72 16-byte units; the two half-warps
+    // bf16 per 32-bit column; fp16 with the FP8 cache).  A row is 72 16-byte units; the two half-warps
     // take alternate units of the same 16 rows, so each warp load reads one
     // 32-byte sector per row, and a 16x32bx2 store with a 4-column split puts
     // unit 2j at columns [8j, 8j+4) and unit 2j+1 at [8j+4, 8j+8).  All 36
@@ -448,7 +480,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
                                                 : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int j = 0; j < kBatch; ++j)
-          if (j0 + j < kUnits) tmem_st16x2_4<4>(lo_base + kColQ + uint32_t(8 * (j0 + j)), v[j]);
+          if (j0 + j < kUnits)
+            tmem_st16x2_4<4>(lo_base + kColQ + uint32_t(8 * (j0 + j)),
+                             kFp8 ? bf16x8_to_f16(v[j]) : v[j]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -529,9 +563,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
             for (int e = 0; e < 4; ++e) {
               const float p0 = ex2_approx(__uint_as_float(xs[8 * uu + 2 * e]) - m_ref);
               const float p1 = ex2_approx(__uint_as_float(xs[8 * uu + 2 * e + 1]) - m_ref);
-              const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
-              sum += __low2float(pp) + __high2float(pp);
-              pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+              if (kFp8) {   // fp16 operands for P.C with the FP8 cache
+                const __half2 pp = __floats2half2_rn(p0, p1);
+                sum += __low2float(pp) + __high2float(pp);
+                pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+              } else {
+                const __nv_bfloat162 pp = __floats2bfloat162_rn(p0, p1);
+                sum += __low2float(pp) + __high2float(pp);
+                pk[e] = *reinterpret_cast<const uint32_t*>(&pp);
+              }
             }
             const int u = (kofs >> 3) + uu;
             *reinterpret_cast<uint4*>(prow + ((u ^ (row & 7)) * 16)) =

@@ -4,8 +4,9 @@
 The cache is drawn in its stored format (E4M3 codes, power-of-two scales,
 bf16 RoPE keys), so the decode is compared with the oracle's attention over
 the exactly dequantised rows at the bf16 tolerance (dequantisation adds no
-rounding), and with the bf16 decode over the same rows written as bf16: the
-two must be bit-identical.  The append is compared code by code with the
+rounding), and with the bf16 decode over the same rows written as bf16, at
+the same tolerance (the FP8 path multiplies fp16 operands: unscaled codes,
+the query, the RoPE keys over the token's scale and P times it).  The append is compared code by code with the
 oracle's quantisation of its own float64 latent; a code may differ by one
 step only where the oracle's value lies within float32 accumulation error of
 a rounding midpoint (the GPU forms the latent in fp32, in another order)."""
@@ -89,7 +90,7 @@ def test_decode_fp8(name, w, lens, nsplit, boost):
     assert np.array_equal(np.isneginf(got_l), np.isneginf(ref_l))
     assert np.max(np.abs(got_l[fin] - ref_l[fin])) < tol(w)
     # The same rows in a bf16 cache (exact: code x 2^k has 4 significant
-    # bits): the bf16 decode gives the same bits.
+    # bits): the bf16 decode agrees within the bf16 bar.
     bf = torch.zeros(w.B, cap, w.R, dtype=torch.bfloat16, device="cuda")
     for b, r in rows.items():
         if len(r):
@@ -101,7 +102,8 @@ def test_decode_fp8(name, w, lens, nsplit, boost):
     o2 = torch.empty_like(o_lat)
     l2 = torch.empty_like(lse)
     mla.combine(d, seq, ws2, used2, o2, l2)
-    assert torch.equal(o2, o_lat) and torch.equal(l2, lse)
+    assert rel_l2(f64(o2)[nz], got_o[nz]) < tol(w)
+    assert np.max(np.abs(f64(l2)[fin] - got_l[fin])) < tol(w)
 
 
 def _near_midpoint(x, rel=2e-5):
