@@ -255,7 +255,13 @@ MLA_API int mla_out_proj_folded(const mla_dims* dims, int32_t d_model, const flo
  * 640 bytes] and scales[b, L_b].  mla_decode_fp8 is mla_decode over the
  * dequantised rows [c~ || k^R] (same q_cat, seqlens, scale, splits,
  * workspace, partial layout; mla_combine merges as usual).  Rows past L_b
- * may hold anything. */
+ * (codes and scales) may hold anything.
+ * Precision: its tensor-core products take fp16 operands (fp32 accumulation):
+ * c~ (the code times its power-of-two scale, exact while |c~| >= 2^-14), the
+ * query and k^R (converted from bf16; exact for |x| in [2^-14, 65504)) and
+ * the probabilities.  So q_cat and k^R must stay below 65504 in magnitude
+ * (as for mla_prefill's fp16 scores), and scales must lie in [2^-24, 2^15]
+ * (every row the append writes from a normalised latent does). */
 MLA_API int64_t mla_cache_fp8_row_bytes(int32_t d_c, int32_t d_r);
 MLA_API int mla_cache_append_fp8(const mla_dims* dims, int32_t hidden, const void* h,
                                  const void* W_DKV, const float* gamma, float eps,

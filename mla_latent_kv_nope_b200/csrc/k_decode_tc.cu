@@ -1,5 +1,6 @@
 // Tensor-core split-KV latent decode for sm_100a (bf16, d_c = 512, d_r = 64,
-// or d_r = 0 for MLA without the decoupled RoPE part).
+// or d_r = 0 for MLA without the decoupled RoPE part; or an FP8 latent cache,
+// widened in shared memory to fp16 operands).
 //
 // What it computes ([MLA-とは] "実装上のトレードオフ": after absorption the
 // decode is MQA with head dim d_c + d_r = 576 -- one latent row per cached
