@@ -585,26 +585,34 @@ class _HostPipeline:
         self.in_stream = torch.cuda.Stream(device=dev)
         self.out_stream = torch.cuda.Stream(device=dev)
         self.graphs = []
-        for c in range(2):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                main = torch.cuda.current_stream()
-                self.in_stream.wait_stream(main)
-                self.out_stream.wait_stream(main)
-                with torch.cuda.stream(self.in_stream):
-                    for d_t, h_t in zip(self.sets[1 - c], self.host_in):
-                        d_t.copy_(h_t, non_blocking=True)
-                with torch.cuda.stream(self.out_stream):
-                    self.host_out.copy_(self.stages[1 - c], non_blocking=True)
-                x = self.sets[c]
-                step(x[0], x[1], x[2], cache, seqlens, h=x[3] if len(x) > 3 else None,
-                     block_table=block_table, scales=scales)
-                self.stages[c].copy_(step.out)
-                if after is not None:
-                    after()
-                main.wait_stream(self.in_stream)
-                main.wait_stream(self.out_stream)
-            self.graphs.append(g)
+        # Each graph's step writes its output straight into its own stage (the
+        # step's output buffer is pointed at the stage while the graph is
+        # recorded), so no device copy sits between the step and the next
+        # device->host copy.
+        out = step.out
+        try:
+            for c in range(2):
+                step.out = self.stages[c]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    main = torch.cuda.current_stream()
+                    self.in_stream.wait_stream(main)
+                    self.out_stream.wait_stream(main)
+                    with torch.cuda.stream(self.in_stream):
+                        for d_t, h_t in zip(self.sets[1 - c], self.host_in):
+                            d_t.copy_(h_t, non_blocking=True)
+                    with torch.cuda.stream(self.out_stream):
+                        self.host_out.copy_(self.stages[1 - c], non_blocking=True)
+                    x = self.sets[c]
+                    step(x[0], x[1], x[2], cache, seqlens, h=x[3] if len(x) > 3 else None,
+                         block_table=block_table, scales=scales)
+                    if after is not None:
+                        after()
+                    main.wait_stream(self.in_stream)
+                    main.wait_stream(self.out_stream)
+                self.graphs.append(g)
+        finally:
+            step.out = out
 
     def run(self, n: int):
         for d_t, h_t in zip(self.sets[0], self.host_in):
