@@ -257,11 +257,12 @@ MLA_API int mla_out_proj_folded(const mla_dims* dims, int32_t d_model, const flo
  * workspace, partial layout; mla_combine merges as usual).  Rows past L_b
  * (codes and scales) may hold anything.
  * Precision: its tensor-core products take fp16 operands (fp32 accumulation):
- * c~ (the code times its power-of-two scale, exact while |c~| >= 2^-14), the
- * query and k^R (converted from bf16; exact for |x| in [2^-14, 65504)) and
- * the probabilities.  So q_cat and k^R must stay below 65504 in magnitude
- * (as for mla_prefill's fp16 scores), and scales must lie in [2^-24, 2^15]
- * (every row the append writes from a normalised latent does). */
+ * c~ (the code times its power-of-two scale), the query and k^R (converted
+ * from bf16) and the probabilities.  Each is exact in fp16 for magnitudes in
+ * [2^-14, 65504); smaller ones keep fp16's subnormal resolution of 2^-24.
+ * So c~, q_cat and k^R must stay below 65504 in magnitude (as for
+ * mla_prefill's fp16 scores); every row the append writes from a normalised
+ * latent does. */
 MLA_API int64_t mla_cache_fp8_row_bytes(int32_t d_c, int32_t d_r);
 MLA_API int mla_cache_append_fp8(const mla_dims* dims, int32_t hidden, const void* h,
                                  const void* W_DKV, const float* gamma, float eps,

@@ -106,6 +106,35 @@ def test_decode_fp8(name, w, lens, nsplit, boost):
     assert np.max(np.abs(f64(l2)[fin] - got_l[fin])) < tol(w)
 
 
+def test_decode_fp8_small_scales():
+    """Scales of 2^-20 .. 2^-17: most dequantised values fall below fp16's
+    normal range and keep its subnormal step (2^-24) in the fp16 operands;
+    the output stays within the bf16 bar of the oracle over the same rows."""
+    w = W["v3_bf16"].scaled(B=3, N=500)
+    lens = np.array([500, 129, 64], dtype=np.int32)
+    cap = 503
+    d = dims_of(w, capacity=cap)
+    cache, scales = _fp8_cache(w, lens, cap)
+    scales.mul_(2.0 ** -11)                     # k in [-20, -17]
+    seq = torch.from_numpy(lens).cuda()
+    q_cat = inputs.normal((w.B, w.H, w.R), 0.5, 31, 3)
+    ws = torch.full((mla.decode_workspace_bytes(d, 0) // 4,), float("nan"), device="cuda")
+    used = mla.decode_fp8(d, dev(q_cat, w), cache, scales, seq, w.softmax_scale, ws)
+    o_lat = torch.empty(w.B, w.H, w.d_c, device="cuda")
+    lse = torch.empty(w.B, w.H, device="cuda")
+    mla.combine(d, seq, ws, used, o_lat, lse)
+    assert mla.get_device_status() == 0
+    ref_cache = np.zeros((w.B, cap, w.R))
+    for b in range(w.B):
+        L = int(lens[b])
+        codes, k, rope = inputs.fp8_cache_rows(w, b, L)
+        c = O.dequantize_latent_rows(codes, np.ldexp(1.0, k - 11))
+        ref_cache[b, :L] = np.concatenate([c, rounded(rope, w)], axis=1)
+    ref_o, ref_l = O.latent_attention(rounded(q_cat, w), ref_cache, lens, w.softmax_scale, w.d_c)
+    assert rel_l2(f64(o_lat), ref_o) < tol(w)
+    assert np.max(np.abs(f64(lse) - ref_l)) < tol(w)
+
+
 def _near_midpoint(x, rel=2e-5):
     """True where x lies within `rel` (relative) of a rounding midpoint of the
     E4M3 grid, i.e. where fp32 accumulation error may flip the rounding."""
