@@ -317,13 +317,26 @@ def test_paged_bad_page_is_reported():
     assert mla.get_device_status() == 0
 
 
-def test_combine_alone():
-    """Synthetic partials placed in the documented workspace slots; the merge
-    must equal the log-sum-exp combination of exactly those partials."""
-    B, H, d_c, Wn = 5, 16, 512, 6
-    lens = np.array([300, 0, 64, 1000, 1], dtype=np.int32)
+COMBINE_CASES = [
+    ("few-partials", 6, [300, 0, 64, 1000, 1], 0.0),
+    # 2 sequences over 100 workers (59 work units: some workers empty): the
+    # kernel whose warps split the partials, rounds of four per warp
+    ("many-partials-split-warps", 100, [3000, 200], 0.0),
+    # one long sequence among short ones: the per-column kernel with about
+    # 25 partials (7 rounds), a fifth of them empty (lse = -inf)
+    ("many-partials-rounds-with-empties", 60, [4000] + [64] * 19, 0.2),
+]
+
+
+@pytest.mark.parametrize("name,Wn,lens,empty", COMBINE_CASES, ids=[c[0] for c in COMBINE_CASES])
+def test_combine_alone(name, Wn, lens, empty):
+    """Synthetic partials (lse spread with std 3, so the running maximum moves
+    between rounds) placed in the documented workspace slots; the merge must
+    equal the log-sum-exp combination of exactly those partials."""
+    lens = np.array(lens, dtype=np.int32)
+    B, H, d_c = len(lens), 16, 512
     w = SMALL_BF16.scaled(B=B)
-    d = dims_of(w, capacity=1000)
+    d = dims_of(w, capacity=int(lens.max()))
     # The documented deal: each non-empty sequence takes 4 start-up units,
     # then one unit per 64-key tile; worker w takes units [wT/W, (w+1)T/W).
     nt = [(L + 63) // 64 for L in lens]
@@ -331,7 +344,7 @@ def test_combine_alone():
     T = sum(units)
     pre = np.concatenate([[0], np.cumsum(units)])
     slots = B + Wn - 1
-    o_all, l_all = inputs.partials(1, H, slots, d_c, seed=3, empty_frac=0.0)
+    o_all, l_all = inputs.partials(1, H, slots, d_c, seed=3, empty_frac=empty)
     ws = torch.full((mla.decode_workspace_bytes(d, Wn) // 4,), float("nan"), device="cuda")
     # documented partial layout: o_part[slot][d_c / 4][H][4]
     o_ws = o_all[0].reshape(H, slots, d_c // 4, 4).transpose(1, 2, 0, 3)
@@ -352,7 +365,7 @@ def test_combine_alone():
         ref_o, ref_l = O.combine_partials(o_all[0][:, sl].astype(np.float64),
                                           l_all[0][:, sl].astype(np.float64))
         assert rel_l2(f64(o_lat[b]), ref_o) < 1e-5
-        assert np.max(np.abs(f64(lse[b]) - ref_l)) < 1e-5
+        assert _lse_err(f64(lse[b]), ref_l) < 1e-5
 
 
 # ---------------------------------------------------------------------------
