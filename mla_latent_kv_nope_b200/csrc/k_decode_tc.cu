@@ -614,7 +614,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
       // Partials are o_part[slot][d_c / 4][H][4]: lanes 0-15 store 16
       // consecutive heads of one 4-column group (256 contiguous bytes), lanes
       // 16-31 the same heads 64 groups further on.
+      // The combine reads them right after this kernel: they are stored
+      // evict-last so that the cache rows streaming through L2 behind them
+      // do not push them out to HBM first.
       float* dst = o_part + ((int64_t(slot) * (kDc / 4) + (lo_half ? 0 : 64)) * H + head) * 4;
+      const uint64_t keep = l2_policy_evict_last();
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
         uint32_t r[32];
@@ -623,9 +627,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
         if (head < H) {
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            *reinterpret_cast<float4*>(dst + int64_t(c / 4 + e) * H * 4) =
+            st_global_f4_hint(
+                dst + int64_t(c / 4 + e) * H * 4,
                 make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
-                            __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+                            __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv),
+                keep);
         }
       }
       if (lo_half && head < H)
