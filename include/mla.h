@@ -178,12 +178,7 @@ MLA_API int mla_merge_partials(const mla_dims* dims, int n_parts, const float* o
 /* --- 5. value up-projection -------------------------------------------------
  * [MLA-とは] "Value側の吸収": o_{t,i} = W^UV_i (sum_j a_{tj,i} c^KV_j).
  *   out[b,i,v] = sum_c W_UV[i,v,c] o_lat[b,i,c]
- * o_lat [B,H,d_c] fp32; W_UV [H,d_v,d_c] dtype; out [B,H,d_v] dtype.
- * With bf16 the kernel is a programmatic dependent launch that requests its
- * W_UV block before it waits for the kernel in front of it in the stream
- * (mla_combine in a step, which lets it start early); o_lat is read after
- * that wait.  So W_UV must not be written by the kernel directly in front of
- * this call: weights loaded before the step satisfy this. */
+ * o_lat [B,H,d_c] fp32; W_UV [H,d_v,d_c] dtype; out [B,H,d_v] dtype. */
 MLA_API int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* W_UV,
                  void* out, void* stream);
 

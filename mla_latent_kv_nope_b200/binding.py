@@ -365,9 +365,7 @@ def merge_partials(dims: Dims, o_parts, lse_parts, o_lat, lse=None, stream=None)
 
 
 def out_proj(dims: Dims, o_lat, W_UV, out, stream=None):
-    """mla_out_proj: out[b,i] = W^UV_i o_lat[b,i].  W_UV must not be written
-    by the kernel issued directly before this call (the bf16 kernel requests
-    it before waiting for that kernel)."""
+    """mla_out_proj: out[b,i] = W^UV_i o_lat[b,i]."""
     dt = dims.torch_dtype
     _need(o_lat, torch.float32, (dims.B, dims.H, dims.d_c), "o_lat")
     _need(W_UV, dt, (dims.H, dims.d_v, dims.d_c), "W_UV")

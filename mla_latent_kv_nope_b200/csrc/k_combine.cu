@@ -108,8 +108,7 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
                float* __restrict__ o_lat, float* __restrict__ lse_out) {
   __shared__ float4 s_rows[kCombineHeads][kQuadsPerBlock + 1];
   __shared__ int64_t s_red[2][kCombineWarps];
-  pdl_trigger();   // the out_proj after it reads o_lat only after its own wait
-  pdl_wait();      // the partials come from the decode launched just before
+  pdl_wait();   // the partials come from the decode launched just before
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h0 = blockIdx.y * kCombineHeads;
@@ -189,8 +188,7 @@ combine_many_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int
   __shared__ float s_m[kCombineWarps][kCombineHeads];
   __shared__ float s_z[kCombineWarps][kCombineHeads];
   __shared__ int64_t s_red[2][kCombineWarps];
-  pdl_trigger();   // the out_proj after it reads o_lat only after its own wait
-  pdl_wait();      // the partials come from the decode launched just before
+  pdl_wait();   // the partials come from the decode launched just before
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h0 = blockIdx.y * kCombineHeads;
@@ -279,9 +277,11 @@ cudaError_t launch_combine(const int32_t* seqlens, int64_t cap, int B, int H, in
   // Many partials per sequence on average (few long sequences): the warps
   // split the partials.  Both are launched with programmatic overlap; the
   // decode before them triggers only by finishing, so the combine's launch
-  // overlaps the decode's drain and nothing more (an early trigger in the
-  // decode measured 1.5 us slower per step).  Each block triggers at its
-  // start, so the out_proj's weight load overlaps the combine's tail.
+  // overlaps the decode's drain and nothing more.  Early triggers measured
+  // slower on B200: in the decode 1.5 us per v3 step; in the combine (so
+  // that out_proj could load its weight during the combine's tail) 2.5 us
+  // faster on the v3 step but 7.5 us slower on the v2-lite step and 4 us
+  // slower per decode + combine pair run back to back.
   if (int64_t(B) + W - 1 > int64_t(kFastParts) * B)
     return launch_pdl(combine_many_kernel, dim3(B, hb, (nq + kManyQuads - 1) / kManyQuads),
                       dim3(kCombineThreads), 0, stream, seqlens, cap, B, H, d_c, W, o_part,

@@ -69,10 +69,9 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __rest
   uint32_t* tbase = reinterpret_cast<uint32_t*>(bars + 2);
   const int i = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // The weight block is requested before the wait for the kernel in front
-  // (the combine, which lets this grid start as soon as all of its blocks
-  // run): W_UV is not one of its outputs, so the 128 KB load overlaps the
-  // combine's tail.  o_lat, its output, is read only after the wait.
+  // Nothing is read before the kernel in front (the combine) has finished:
+  // the weight could have been written by stream work before this call too.
+  pdl_wait();
   if (threadIdx.x == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
@@ -85,7 +84,6 @@ out_proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const float* __rest
     tmem_alloc(tbase, kOpN);
     tmem_relinquish();
   }
-  pdl_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

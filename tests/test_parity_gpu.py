@@ -67,10 +67,7 @@ def test_out_proj(w):
     _, Wuv = inputs.weights(w)
     o_lat = inputs.normal((w.B, w.H, w.d_c), 0.05, 123, 1)
     out = torch.empty(w.B, w.H, w.d_v, dtype=torch_dtype(w), device="cuda")
-    # The weight is in place before the kernel in front of out_proj runs
-    # (out_proj may request it before that kernel has finished).
-    W_UV = dev(Wuv, w)
-    mla.out_proj(dims_of(w), dev(o_lat, w, torch.float32), W_UV, out)
+    mla.out_proj(dims_of(w), dev(o_lat, w, torch.float32), dev(Wuv, w), out)
     ref = O.out_proj(o_lat.astype(np.float64), rounded(Wuv, w))
     assert rel_l2(f64(out), ref) < tol(w)
 
