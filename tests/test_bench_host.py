@@ -1,6 +1,7 @@
 """Host-side parts of bench.py that need no GPU: the clock sampler's
-in-process polling and summary (with a fake NVML), and the bounded reference
-arm's per-step budget."""
+in-process polling and summary (with a fake NVML), the bounded reference
+arm's per-step budget, the `--gpus` launcher, and the inputs of the roofline
+object (peak source, traffic record validity, algorithmic bytes and FLOPs)."""
 import importlib.util
 import os
 import sys
@@ -127,3 +128,54 @@ def test_gpus_flag_must_match_the_launcher():
                        capture_output=True, text=True, timeout=120, env=env, cwd=ROOT)
     assert r.returncode != 0 and "launcher started 1 rank" in r.stderr
     assert not _json_lines(r.stdout)
+
+
+def test_peaks_measured_file_else_fallback(tmp_path, monkeypatch):
+    """The roofline denominators come from MEASURED_PEAKS.json when it is
+    present and are labelled as the fallback otherwise."""
+    b = _bench()
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    hbm, tf, tf_sus, src = b._peaks()
+    assert (hbm, tf, src) == (b.FALLBACK_HBM_GBS, b.FALLBACK_BF16_TFLOPS, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(
+        '{"hbm_gbs": 6552.0, "bf16_tflops": 1638.5, "bf16_tflops_sustained": 1368.2}')
+    assert b._peaks() == (6552.0, 1638.5, 1368.2, "measured")
+
+
+def test_traffic_record_only_for_the_kernel_it_was_taken_on(tmp_path, monkeypatch):
+    """A DRAM-traffic record is reported only while the decode kernel's
+    sources hash to the value stored beside it."""
+    import json
+    import shutil
+    b = _bench()
+    csrc = tmp_path / "mla_latent_kv_nope_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in ("k_decode_tc.cu", "tile_deal.cuh", "common.cuh", "sm100.cuh"):
+        shutil.copy(os.path.join(ROOT, "mla_latent_kv_nope_b200", "csrc", name), csrc / name)
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(b, "ROOT", str(tmp_path))
+    rec = {"v3_bf16": {"source_hash": b._decode_source_hash(), "traffic_bytes_per_launch": 123.0}}
+    (tmp_path / "profiles" / "decode_traffic.json").write_text(json.dumps(rec))
+    assert b._ncu_traffic("v3_bf16") == 123.0
+    assert b._ncu_traffic("longctx_bf16") is None
+    with open(csrc / "k_decode_tc.cu", "a") as f:
+        f.write("\n")
+    assert b._ncu_traffic("v3_bf16") is None
+
+
+def test_algorithmic_counts_are_the_closed_forms():
+    """Per cached row the decode reads one latent row (576 bf16 = 1152 B, or
+    512 E4M3 codes + 64 bf16 RoPE keys + a 4-byte scale = 644 B) and does
+    2 H (576 + 512) FLOPs (QK^T over d_c + d_r, P.c over d_c)."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    from mla_latent_kv_nope_b200 import inputs
+    b = _bench()
+    w = inputs.WORKLOADS["v3_bf16"]
+    lens = np.full(32, 8193)
+    byts, flops, rows = b._algorithmic(w, lens)
+    assert rows == 32 * 8193
+    assert byts == rows * 1152
+    assert flops == 2 * 128 * rows * (576 + 512)
+    byts8, flops8, _ = b._algorithmic(w, lens, fp8=True)
+    assert byts8 == rows * 644 and flops8 == flops
