@@ -60,6 +60,27 @@ __device__ __forceinline__ void lse_round(const float (&lv)[kRound], const float
   }
 }
 
+// The partials are dead once this kernel has read them: its loads mark their
+// L2 lines evict-first (the decode stored them evict-last so that they would
+// wait in L2 for this kernel), so they leave L2 before any other data.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ float4 ld_last_use(const float4* p, uint64_t policy) {
+  float4 v;
+  asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
+__device__ __forceinline__ float ld_last_use(const float* p, uint64_t policy) {
+  float v;
+  asm volatile("ld.global.L2::cache_hint.f32 %0, [%1], %2;" : "=f"(v) : "l"(p), "l"(policy));
+  return v;
+}
+
 // Units before sequence b and in the whole batch (every thread of the block
 // takes part; one round trip over the lengths).
 __device__ __forceinline__ void unit_prefix(const int32_t* seqlens, int64_t cap, int B, int b,
@@ -138,6 +159,7 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
   // Column groups of this thread: q_base + warp + 8 j, j < 4.
   const float4* src0 = reinterpret_cast<const float4*>(o_part) + int64_t(q_base + warp) * H + i;
   const int64_t slot_stride = int64_t(nq) * H;   // float4 units
+  const uint64_t dead = l2_policy_evict_first();
   float4 acc[kQuadsPerWarp];
 #pragma unroll
   for (int j = 0; j < kQuadsPerWarp; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -149,12 +171,13 @@ combine_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int H, i
     for (int k = 0; k < kRound; ++k) {
       const int w = w0 + k;
       const bool use = w <= w_last && head_ok && live(w);
-      lv[k] = use ? lse_part[int64_t(b + w) * H + i] : -INFINITY;
+      lv[k] = use ? ld_last_use(lse_part + int64_t(b + w) * H + i, dead) : -INFINITY;
       const float4* sk = src0 + int64_t(b + (use ? w : w_first)) * slot_stride;
 #pragma unroll
       for (int j = 0; j < kQuadsPerWarp; ++j)
-        v[k][j] = (use && warp + kCombineWarps * j < nqb) ? sk[int64_t(kCombineWarps * j) * H]
-                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[k][j] = (use && warp + kCombineWarps * j < nqb)
+                      ? ld_last_use(sk + int64_t(kCombineWarps * j) * H, dead)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     lse_round(lv, v, m, z, acc);
   }
@@ -216,6 +239,7 @@ combine_many_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int
   };
   const float4* src0 = reinterpret_cast<const float4*>(o_part) + int64_t(q_base) * H + i;
   const int64_t slot_stride = int64_t(nq) * H;   // float4 units
+  const uint64_t dead = l2_policy_evict_first();
   float4 acc[kManyQuads];
 #pragma unroll
   for (int q = 0; q < kManyQuads; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -227,11 +251,12 @@ combine_many_kernel(const int32_t* __restrict__ seqlens, int64_t cap, int B, int
     for (int k = 0; k < kRound; ++k) {
       const int w = w0 + kCombineWarps * k;
       const bool use = w <= w_last && head_ok && live(w);
-      lv[k] = use ? lse_part[int64_t(b + w) * H + i] : -INFINITY;
+      lv[k] = use ? ld_last_use(lse_part + int64_t(b + w) * H + i, dead) : -INFINITY;
       const float4* sw = src0 + int64_t(b + (use ? w : w_first)) * slot_stride;
 #pragma unroll
       for (int q = 0; q < kManyQuads; ++q)
-        v[k][q] = (use && q < nqb) ? sw[int64_t(q) * H] : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[k][q] = (use && q < nqb) ? ld_last_use(sw + int64_t(q) * H, dead)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     lse_round(lv, v, m, z, acc);
   }
