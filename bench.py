@@ -140,14 +140,18 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
-        rows = list(self.inproc)
+    def summary(self, window=None):
+        """Median SM clock and the reasons seen in the timed window, or, with
+        ``window = (t0, t1)`` (host times), in that window from the separate
+        process's samples alone."""
+        rows = list(self.inproc) if window is None else []
+        t_start, t_stop = window if window is not None else (self.t_start, self.t_stop)
         for ln in getattr(self, "lines", []):
             f = ln.split()
             if len(f) != 3:
                 continue
             t, sm, rs = float(f[0]), int(f[1]), int(f[2])
-            if self.t_start is not None and not (self.t_start <= t <= self.t_stop):
+            if t_start is not None and not (t_start <= t <= t_stop):
                 continue
             rows.append((sm, rs))
         if not rows:
@@ -158,10 +162,12 @@ class ClockSampler:
             for bit, name in self.REASONS.items():
                 if rs & bit:
                     reasons.add(name)
+        source = ("NVML during the timed steps (this process while they run, and a "
+                  "separate process every ~2 ms inside the window)" if window is None else
+                  "NVML every ~2 ms (a separate process) during this pass")
         return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": getattr(self, "max_mhz", None),
                 "sm_min_mhz": sms[0], "samples": len(rows), "reasons": sorted(reasons),
-                "source": "NVML during the timed steps (this process while they run, and a "
-                          "separate process every ~2 ms inside the window)"}
+                "source": source}
 
 
 # ---------------------------------------------------------------------------
@@ -343,7 +349,9 @@ def run_ours(args, rank, world, local_rank):
         clk.stop()
         barrier()
         ms_total = t0.elapsed_time(t1)
+        t_dec = time.time()
         dec_avg, decomb_avg = decode_only(max(args.steps, 5 * kRep))
+        t_dec = (t_dec, time.time())
     ms_total = mdist.max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
 
@@ -445,6 +453,9 @@ def run_ours(args, rank, world, local_rank):
             "frac_of_roofline_with_combine": t_roof / (decomb_avg * 1e-3),
             "hbm_frac": achieved_gbs / hbm, "tensor_frac_burst": achieved_tf / tf_burst,
             "tensor_frac_sustained": achieved_tf / tf_sus,
+            # This pass runs right after the timed steps; under that much
+            # back-to-back decode work the power cap can lower the SM clock.
+            "clocks": clk.summary(t_dec),
         },
         "roofline": {
             "kernel": "mla_decode (split-KV latent attention)",

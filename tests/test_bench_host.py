@@ -179,3 +179,19 @@ def test_algorithmic_counts_are_the_closed_forms():
     assert flops == 2 * 128 * rows * (576 + 512)
     byts8, flops8, _ = b._algorithmic(w, lens, fp8=True)
     assert byts8 == rows * 644 and flops8 == flops
+
+
+def test_clock_summary_of_a_second_window():
+    """The decode-only pass gets its own clock summary from the separate
+    sampler's lines inside its window; the in-process samples belong to the
+    timed steps only."""
+    b = _bench()
+    clk = b.ClockSampler(0)
+    clk.poll_until(lambda: len(clk.inproc) >= 3, nvml=FakeNvml(mhz=1965, reasons=0))
+    clk.start(); clk.t_start, clk.t_stop = 10.0, 20.0
+    clk.lines = ["12.0 1965 0", "25.0 1800 4", "26.0 1812 4", "40.0 1500 8", "bad line"]
+    main = clk.summary()
+    assert main["samples"] == 4 and main["reasons"] == []
+    dec = clk.summary((24.0, 30.0))
+    assert dec["samples"] == 2 and dec["sm_min_mhz"] == 1800 and dec["reasons"] == ["sw_power_cap"]
+    assert clk.summary((50.0, 60.0)) is None
